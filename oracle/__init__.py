@@ -1,0 +1,129 @@
+"""fp64 CPU oracle for the KDA operator -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library
+(``gated_delta_rule_86_b200``) never imports it, and the two share no code:
+the only module both sides use is the seeded input generator, which holds none
+of the method's arithmetic.
+
+Contents
+  * :func:`recurrent` -- the token-by-token recurrence of the "Stage 3: KDA's
+    fused design" equation ("Hybrid Linear Attention Architectures: Breaking
+    Through the Long-Context Engineering Bottleneck in LLMs"), in plain C
+    (``kda_oracle.c``), fp64, threaded over (sequence, head) pairs.
+  * :func:`decode_step` -- one iteration of the same loop body, in place.
+  * :func:`chunkwise` (``chunkwise.py``) -- an independent fp64 NumPy
+    restatement of the chunkwise formulas ("Hardware-Aware Chunkwise
+    Parallelism" on the same page; section 3 of "Linear Attention KDA Gating in
+    a 3:1 Hybrid Architecture").  It is not the oracle; the tests use it to pin
+    the garbled chunk formulas against the recurrence.
+
+Pins: every function here is checked by ``tests/test_oracle_pins.py`` against
+closed forms and brute-force constructions that share no code with it
+(DeltaNet reduction, exact overwrite with a unit key, the unrolled operator
+product for short sequences, beta = 0 decay-only closed form, scalar-gate
+reduction, linearity, non-expansion, chunkwise equivalence, composition).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile ``kda_oracle.c`` into ``libkda_oracle.so`` with gcc (plain C)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build_oracle()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        i64 = ctypes.c_int64
+        lib.kda_oracle_recurrent.argtypes = [dp, dp, dp, dp, dp, dp, i64p, i64, i64, i64, i64,
+                                             i64, i64, dp, dp, ctypes.c_int]
+        lib.kda_oracle_recurrent.restype = ctypes.c_int
+        lib.kda_oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, i64, i64, i64, i64]
+        lib.kda_oracle_decode_step.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def recurrent(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, nthreads=None):
+    """Token recurrence over [B, T, H, d] inputs; returns ``(out, final_state)`` in fp64.
+
+    ``q, k, log_alpha``: [B, T, H, d_k]; ``v``: [B, T, H, d_v]; ``beta``: [B, T, H];
+    ``init_state``: [N, H, d_k, d_v] or None (zeros); ``cu_seqlens``: int [N+1]
+    with B == 1, or None (N = B).  Inputs of any float dtype are widened to fp64
+    exactly (bf16 values are taken as the bf16 numbers they are).
+    """
+    q, k, v, log_alpha, beta = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and log_alpha.shape == q.shape
+    assert v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+        assert B == 1
+    else:
+        N = B
+    s0 = None if init_state is None else _f64(init_state)
+    if s0 is not None:
+        assert s0.shape == (N, H, dk, dv)
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    fs = np.zeros((N, H, dk, dv), dtype=np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().kda_oracle_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                      _ptr(s0), _ptr(cu, ctypes.c_int64), N, B, T, H, dk, dv,
+                                      _ptr(out), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out, fs
+
+
+def decode_step(q, k, v, log_alpha, beta, state):
+    """One recurrence step for [B, H, d] inputs; returns ``(out, new_state)`` (fp64 copies)."""
+    q, k, v, log_alpha, beta = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    S = _f64(state).copy()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    assert S.shape == (B, H, dk, dv) and beta.shape == (B, H)
+    out = np.zeros((B, H, dv), dtype=np.float64)
+    rc = _load().kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                        _ptr(S), _ptr(out), B, H, dk, dv)
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out, S
+
+
+from .chunkwise import chunkwise  # noqa: E402  (NumPy restatement, see module docstring)
+
+__all__ = ["build_oracle", "recurrent", "decode_step", "chunkwise"]
