@@ -1,0 +1,383 @@
+"""Benchmark of the KDA operator on B200: prefill tokens/s and decode steps/s.
+
+One bench step = one chunkwise prefill (kda_chunk_fwd) over the long-context
+workload: B=1, H=32, T=65536, d_k=d_v=128, bf16 inputs, fp32 state, N(0,0.1)
+initial state, log_alpha = logsigmoid(N(4,1)).  The decode workload (B=256,
+H=32, d=128, fp32 state updated in place, 1024 distinct tokens) is timed in
+the same run and reported in the "decode" object.
+
+Usage:
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {kda,reference}]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own copy of the workload (weak scaling: the (sequence, head) units are
+independent, no data-path collective), the timed region is bracketed by a
+barrier and cuda synchronize, and the step time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the reference arm: there is no
+installable reference implementation) on a bounded sample of the same
+workload on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s & % tensor roofline; decode steps/s & % HBM GB/s"
+PREFILL_WORKLOAD = "long_bf16"
+DECODE_WORKLOAD = "decode_bf16"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---- algorithmic work per unit (d = 128, C = 64) ---------------------------------------------------
+
+def prefill_alg_bytes(tokens_heads, heads_total, dk=128, dv=128, in_bytes=2, out_bytes=4):
+    """q, k, log_alpha (d_k each), v (d_v), beta, out (d_v) per token-head, plus the
+    fp32 state read and written once per sequence-head."""
+    per_th = (3 * dk + dv + 1) * in_bytes + dv * out_bytes
+    return tokens_heads * per_th + heads_total * 2 * dk * dv * 4
+
+
+def prefill_alg_flops(tokens_heads, dk=128, dv=128, C=64):
+    """Triangular products counted as triangular: A, P, W, U, P U~ give 5 C d; W S, Q S,
+    Kd^T U~ give 6 d^2 (d_k = d_v = d) per token-head."""
+    return tokens_heads * (5 * C * dk + 2 * dk * dv * 3)
+
+
+def decode_alg_bytes(heads, dk=128, dv=128, in_bytes=2, out_bytes=4):
+    return heads * (2 * dk * dv * 4 + (3 * dk + dv + 1) * in_bytes + dv * out_bytes)
+
+
+# ---- clocks -----------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        self.device_index = device_index
+
+    def __enter__(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(self.device_index)
+        fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", ident], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---- distributed plumbing ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}; launch with torch.distributed.run")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- the reference arm: the fp64 oracle on the host ----------------------------------------------------
+
+def time_oracle(workload, seed_offset=0, target_s=10.0, max_tokens=None):
+    """Oracle tokens/s on the first T_s tokens of the prefill workload (all heads),
+    doubling T_s until one run takes >= target_s.  Returns (tokens/s, sample text, threads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from gated_delta_rule_86_b200 import inputs
+    w = inputs.WORKLOADS[workload]
+    threads = os.cpu_count() or 1
+    T_s = 256
+    while True:
+        x = inputs.make_prefill(w, device="cpu", T=T_s, seed=inputs.BASE_SEED + w.wid + seed_offset)
+        args = [x[n].float().numpy().astype(np.float64) for n in ("q", "k", "v", "log_alpha", "beta")]
+        s0 = None if x["init_state"] is None else x["init_state"].numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.recurrent(*args, init_state=s0, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or T_s >= (max_tokens or w.T):
+            break
+        T_s = min(T_s * 2, max_tokens or w.T)
+    del torch
+    tok = w.B * T_s
+    sample = f"first {T_s} of {w.T} tokens, all {w.H} heads, B={w.B} ({tok * w.H} token-heads), fp64 C oracle"
+    return tok / dt, sample, threads, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_delta_rule_86_b200 import inputs
+    w = inputs.WORKLOADS[PREFILL_WORKLOAD]
+    per_step = []
+    sample = threads = None
+    for i in range(args.warmup + args.steps):
+        tps, sample, threads, dt = time_oracle(PREFILL_WORKLOAD, seed_offset=i, target_s=args.ref_seconds)
+        if i >= args.warmup:
+            per_step.append(tps)
+    value = statistics.median(per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.B * w.T / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL_WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                       "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- the kda arm ----------------------------------------------------------------------------------------
+
+def event_time_ms(fn, n):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        fn(i)
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_kda(args):
+    import torch
+
+    from gated_delta_rule_86_b200 import inputs, kda_chunk_fwd, kda_decode_step, device_error
+    rank, world, local = dist_setup(args.gpus)
+    peaks, peaks_src = load_peaks()
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak_burst = peaks["bf16_tflops"]
+    tc_peak_sust = peaks.get("bf16_tflops_sustained", tc_peak_burst)
+
+    # ---------------- prefill ----------------
+    w = inputs.WORKLOADS[PREFILL_WORKLOAD]
+    x = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank)
+    names = ("q", "k", "v", "log_alpha", "beta")
+    a = [x[n] for n in names]
+    s0 = x["init_state"]
+    tokens = w.B * w.T
+    token_heads = tokens * w.H
+
+    def prefill_step(_i):
+        return kda_chunk_fwd(*a, initial_state=s0)
+
+    for _ in range(args.warmup):
+        prefill_step(0)
+    assert device_error() == 0, "device error during warm-up"
+    with ClockSampler(local) as clk:
+        barrier(world)
+        ms = event_time_ms(prefill_step, args.steps)
+        barrier(world)
+    clocks = clk.summary()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    value = world * tokens / (ms_step * 1e-3)
+    alg_bytes = prefill_alg_bytes(token_heads, w.B * w.H)
+    alg_flops = prefill_alg_flops(token_heads)
+    achieved_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
+    dense_flops = token_heads * (12 * w.chunk * w.dk + 6 * w.dk * w.dv)
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": None,
+                "peak_source": f"{peaks_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks_src == "measured" else "fallback 6650 GB/s",
+                "kernel": "kda_chunk_tc_kernel", "alg_bytes_per_launch": alg_bytes,
+                "tensor": {"alg_flops_per_launch": alg_flops,
+                           "achieved_tflops": alg_flops / (ms_step * 1e-3) / 1e12,
+                           "frac_of_burst_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst,
+                           "frac_of_sustained_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_sust,
+                           "dense_tile_frac_of_burst_peak":
+                               dense_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst}}
+    # end to end through the public API from pinned host memory
+    host = [t.cpu().pin_memory() for t in a]
+    s0_h = s0.cpu().pin_memory()
+
+    def e2e_step(_i):
+        out, fs = kda_chunk_fwd(*host, initial_state=s0_h)
+        return out
+
+    e2e_step(0)
+    barrier(world)
+    t0 = time.perf_counter()
+    e2e_ms = event_time_ms(e2e_step, max(1, args.steps // 2))
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_ms / max(1, args.steps // 2), world)
+    h2d = sum(t.numel() * t.element_size() for t in host) + s0_h.numel() * 4
+    d2h = token_heads * w.dv * 4 + w.B * w.H * w.dk * w.dv * 4
+    del host, s0_h, x, a, s0
+    torch.cuda.empty_cache()
+
+    # ---------------- decode ----------------
+    dw = inputs.WORKLOADS[DECODE_WORKLOAD]
+    d = inputs.make_decode(dw, device="cuda", seed=inputs.BASE_SEED + dw.wid + 1000 * rank)
+    state = d["state"]
+    nsteps = dw.decode_steps
+
+    def decode_step(i):
+        return kda_decode_step(d["q"][i], d["k"][i], d["v"][i], d["log_alpha"][i], d["beta"][i], state)
+
+    for i in range(3):
+        decode_step(i)
+    barrier(world)
+    dms = event_time_ms(decode_step, nsteps)
+    barrier(world)
+    dms_step = max_over_ranks(dms / nsteps, world)
+    heads = dw.B * dw.H
+    d_bytes = decode_alg_bytes(heads)
+    d_gbs = d_bytes / (dms_step * 1e-3) / 1e9
+    decode = {"workload": DECODE_WORKLOAD, "B": dw.B, "H": dw.H, "d_k": dw.dk, "d_v": dw.dv, "steps": nsteps,
+              "steps_per_s": world * 1e3 / dms_step, "tokens_per_s": world * dw.B * 1e3 / dms_step,
+              "us_per_step": dms_step * 1e3,
+              "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": hbm_peak, "unit": "GB/s",
+                           "frac": d_gbs / hbm_peak, "traffic": None, "kernel": "kda_decode_kernel",
+                           "alg_bytes_per_launch": d_bytes}}
+    # decode end to end: tokens from pinned host memory each step, output read back each step
+    hq = [d[n][:64].cpu().pin_memory() for n in names]
+    hout = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, pin_memory=True)
+
+    def decode_e2e(i):
+        kda_decode_step(hq[0][i], hq[1][i], hq[2][i], hq[3][i], hq[4][i], state, out=hout)
+
+    barrier(world)
+    de2e = event_time_ms(decode_e2e, 64) / 64
+    barrier(world)
+    de2e = max_over_ranks(de2e, world)
+    decode["e2e"] = {"value": world * 1e3 / de2e, "unit": "steps/s",
+                     "h2d_bytes_per_step": sum(t[0].numel() * t.element_size() for t in hq),
+                     "d2h_bytes_per_step": hout.numel() * 4}
+    assert device_error() == 0, "device error during the timed region"
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tps, sample, threads, _ = time_oracle(PREFILL_WORKLOAD, target_s=args.ref_seconds)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": PREFILL_WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                           "chunk": w.chunk, "io": "bf16 q/k/v/log_alpha/beta, fp32 out and state",
+                           "init_state": "N(0,0.1)", "log_alpha": "logsigmoid(N(4,1))",
+                           "l2": "inputs larger than L2 (2.1 GB of q/k/v/log_alpha per step)",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": args.steps, "clocks": clocks, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--ref-seconds", type=float, default=10.0, help="target CPU seconds per oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_kda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,10 @@
+"""B200-native (sm_100a) KDA operator: chunkwise prefill and recurrent decode.
+
+The computation lives in ``libkda_b200.so`` (C ABI in ``include/kda.h``);
+``ops`` is its thin Python binding.  Importing the package does not load the
+library; the first call does, and fails loudly if it has not been built.
+"""
+from ._lib import EXPORTED, KdaError, load  # noqa: F401
+from .ops import device_error, kda_chunk_fwd, kda_decode_step, kda_recurrent_fwd  # noqa: F401
+
+__all__ = ["kda_chunk_fwd", "kda_recurrent_fwd", "kda_decode_step", "device_error", "KdaError", "load"]

@@ -1,0 +1,179 @@
+// kda_api.cu -- the C ABI of libkda_b200.so (declared in include/kda.h).
+//
+// Host side only: argument validation, kernel selection and launch on the
+// caller's stream.  The whole library is this one translation unit; the
+// kernels live in the headers included below.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+#include "kda_chunk_tc.cuh"
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_recurrent.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_ok(int d) { return d == 64 || d == 128; }
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Checks shared by kda_chunk_fwd and kda_recurrent_fwd.  Returns KDA_OK when
+// the call is well-formed.
+kda_status check_prefill(const void *q, const void *k, const void *v, const void *la, const void *beta,
+                         const float *init_state, const int32_t *cu, int32_t num_seqs, int32_t B, int32_t T,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, kda_dtype out_dtype,
+                         const void *out, const float *final_state) {
+    if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+    // token tensors may be empty (NULL) only when there are no tokens
+    if (T > 0 && (!q || !k || !v || !la || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (cu) {
+        if (B != 1 || num_seqs < 1) return KDA_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return KDA_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {q, k, v, la, beta, out, init_state, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    // an in-place state update must alias exactly
+    if (init_state && final_state && init_state != final_state) {
+        const int64_t N = cu ? num_seqs : B;
+        const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
+        const char *a = reinterpret_cast<const char *>(init_state), *b = reinterpret_cast<const char *>(final_state);
+        if (a < b + bytes && b < a + bytes) return KDA_ERR_INVALID_ARG;
+    }
+    // 64-bit element counts must stay addressable by the kernels' index math
+    const int64_t tokens = (int64_t)B * T * H;
+    if (tokens * (dk > dv ? dk : dv) > (int64_t(1) << 46)) return KDA_ERR_UNSUPPORTED;
+    if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    const int64_t ctas = (int64_t)(cu ? num_seqs : B) * H * (dv / 32);
+    if (ctas > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+template <typename TIO, typename TOUT>
+cudaError_t dispatch_recurrent_t(const void *q, const void *k, const void *v, const void *la, const void *beta,
+                                 const float *s0, const int32_t *cu, int ns, int B, int T, int H, int dk, int dv,
+                                 void *out, float *fs, cudaStream_t st) {
+    if (dk == 64) return kda::launch_recurrent<64, TIO, TOUT>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
+    return kda::launch_recurrent<128, TIO, TOUT>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
+}
+
+cudaError_t dispatch_recurrent(kda_dtype dt, kda_dtype odt, const void *q, const void *k, const void *v,
+                               const void *la, const void *beta, const float *s0, const int32_t *cu, int ns, int B,
+                               int T, int H, int dk, int dv, void *out, float *fs, cudaStream_t st) {
+    if (dt == KDA_F32 && odt == KDA_F32)
+        return dispatch_recurrent_t<float, float>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs, st);
+    if (dt == KDA_F32)
+        return dispatch_recurrent_t<float, __nv_bfloat16>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs,
+                                                          st);
+    if (odt == KDA_F32)
+        return dispatch_recurrent_t<__nv_bfloat16, float>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs,
+                                                          st);
+    return dispatch_recurrent_t<__nv_bfloat16, __nv_bfloat16>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
+                                                              fs, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+const char *kda_version(void) { return "kda_b200 0.1.0 sm_100a"; }
+
+kda_status kda_get_last_device_error(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+    int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, kda::g_device_error, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(kda::g_device_error, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    return word == 0 ? KDA_OK : static_cast<kda_status>(word);
+}
+
+kda_status kda_recurrent_fwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                             const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                             int32_t T, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                             kda_dtype out_dtype, void *out, float *final_state, void *stream) {
+    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
+                                 dtype, out_dtype, out, final_state);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return from_cuda(dispatch_recurrent(dtype, out_dtype, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                                        B, T, H, d_k, d_v, out, final_state, st));
+}
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                         const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
+                         kda_dtype out_dtype, void *out, float *final_state, void *stream) {
+    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
+                                 dtype, out_dtype, out, final_state);
+    if (s != KDA_OK) return s;
+    if (chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == KDA_F32) {
+        // fp32 I/O asks for fp32 accuracy, which bf16 tensor-core operands
+        // cannot give: evaluate on CUDA cores with the fp32 state.
+        return from_cuda(dispatch_recurrent(dtype, out_dtype, q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                            num_seqs, B, T, H, d_k, d_v, out, final_state, st));
+    }
+    if (d_k != 128) return KDA_ERR_UNSUPPORTED;
+    if (out_dtype == KDA_F32)
+        return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
+                                                     T, H, d_v, out, final_state, st));
+    return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                                                         B, T, H, d_v, out, final_state, st));
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                           float *state, void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                           kda_dtype out_dtype, void *stream) {
+    if (!q || !k || !v || !log_alpha || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, state, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+#define KDA_DECODE_CASE(DK, DV)                                                                            \
+    if (d_k == DK && d_v == DV) {                                                                          \
+        if (dtype == KDA_F32)                                                                              \
+            e = out_dtype == KDA_F32                                                                       \
+                    ? kda::launch_decode<DK, DV, float, float>(q, k, v, log_alpha, beta, state, out, B, H, st) \
+                    : kda::launch_decode<DK, DV, float, __nv_bfloat16>(q, k, v, log_alpha, beta, state, out, B, \
+                                                                       H, st);                             \
+        else                                                                                               \
+            e = out_dtype == KDA_F32                                                                       \
+                    ? kda::launch_decode<DK, DV, __nv_bfloat16, float>(q, k, v, log_alpha, beta, state, out, B, \
+                                                                       H, st)                              \
+                    : kda::launch_decode<DK, DV, __nv_bfloat16, __nv_bfloat16>(q, k, v, log_alpha, beta, state, \
+                                                                               out, B, H, st);             \
+        return from_cuda(e);                                                                               \
+    }
+    KDA_DECODE_CASE(128, 128)
+    KDA_DECODE_CASE(128, 64)
+    KDA_DECODE_CASE(64, 128)
+    KDA_DECODE_CASE(64, 64)
+#undef KDA_DECODE_CASE
+    return KDA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,41 @@
+// Shared device helpers for the KDA kernels: element access for the two I/O
+// dtypes, the device-side error word and bounded waits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Error codes recorded in the device error word (mirror kda_status values).
+constexpr int kDevErrTimeout = 4;
+
+// Device-side error word (one per device and per translation unit that
+// includes this header; the library is a single translation unit).  Kernels
+// set it with atomicMax when a bounded wait runs out;
+// kda_get_last_device_error reads and clears it.
+static __device__ int g_device_error = 0;
+
+__device__ __forceinline__ void record_device_error(int code) { atomicMax(&g_device_error, code); }
+
+// Iteration limit of every spin on an mbarrier phase.  A try_wait suspends the
+// thread for up to a system-dependent time per call, so this bounds a wait to
+// well under a few seconds while never triggering on a healthy kernel.
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// log2(e), used to turn exp(x) into exp2(x * log2e) for the ex2 unit.
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
+
+}  // namespace kda

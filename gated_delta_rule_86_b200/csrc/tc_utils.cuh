@@ -1,0 +1,186 @@
+// Thin inline-PTX wrappers for the sm_100a features the chunk kernel uses:
+// mbarriers, the async-proxy fence, Tensor Memory (TMEM) allocation and loads,
+// tcgen05.mma with shared-memory operand descriptors, and tcgen05.commit.
+//
+// Operand layouts used throughout (bf16, 128-byte swizzle, "SW128"): a tile is
+// stored as 8-row groups of 128-byte rows; inside a group, row r's 16-byte
+// chunk c lives at chunk position c ^ (r % 8).  Groups are 1024 bytes apart and
+// every group is 1024-byte aligned.  A [rows x 64] bf16 block therefore takes
+// rows * 128 bytes; wider tiles are stored as consecutive 64-column blocks.
+// The same bytes serve as a K-major operand (rows = M or N, columns = K) or as
+// an MN-major operand (rows = K, columns = M or N); only the descriptor
+// differs.  SW64 is the 64-byte-row analogue (32 bf16 columns, 512-byte groups,
+// chunk position c ^ ((r / 2) % 4)).
+#pragma once
+
+#include <stdint.h>
+
+#include "kda_common.cuh"
+
+namespace kda {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier ---------------------------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete, at most kSpinLimit
+// polls.  On timeout records the error word, sets *abort (shared) and returns
+// false; also returns false at once if *abort is already set.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+    }
+    record_device_error(kDevErrTimeout);
+    *abort = 1;
+    return false;
+}
+
+// Make generic-proxy shared-memory writes visible to the async proxy (the
+// tensor cores read operands through it).
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- TMEM -------------------------------------------------------------------------------------
+
+// Whole-warp operations.  `dst` receives the TMEM base address.
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Load 32 lanes x 16 consecutive 32-bit columns: thread i of the warp receives
+// lane (warp's lane base + i), columns [col, col + 16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]),
+          "=r"(u[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Lane field of a TMEM address for the 32-lane subpartition a warp may access.
+__device__ __forceinline__ uint32_t tmem_lane_base(int warp) { return static_cast<uint32_t>((warp & 3) * 32) << 16; }
+
+// ---- descriptors ------------------------------------------------------------------------------
+
+enum Swz : uint32_t { kSwzNone = 0, kSwz128 = 2, kSwz64 = 4, kSwz32 = 6 };
+
+// Shared-memory matrix descriptor (sm_100 format): start address, leading- and
+// stride-dimension byte offsets (all >> 4), version 1 at bit 46, swizzle mode
+// at bits 61-63.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                               uint32_t swz) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(swz & 7) << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16 with an fp32 accumulator.  `fmt`
+// selects the operand type of both A and B (kF16 or kBF16: one tcgen05.mma
+// never mixes them); a_mn / b_mn select MN-major operands; neg_a negates A.
+enum OpFmt : uint32_t { kF16 = 0, kBF16 = 1 };
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t fmt, bool a_mn, bool b_mn,
+                                                  bool neg_a = false) {
+    return (1u << 4)                       // D format: f32
+           | (fmt << 7)                    // A format
+           | (fmt << 10)                   // B format
+           | ((neg_a ? 1u : 0u) << 13)     // negate A
+           | ((a_mn ? 1u : 0u) << 15)      // A major
+           | ((b_mn ? 1u : 0u) << 16)      // B major
+           | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false) {
+    return make_idesc(M, N, kBF16, a_mn, b_mn, neg_a);
+}
+
+// D[tmem] (+)= A[smem] * B[smem] (kind::f16: fp16 or bf16 operands); issued by one thread.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// Arrive once on `bar` when all previously issued tcgen05.mma of this thread complete.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// ---- swizzled byte offsets --------------------------------------------------------------------
+
+// Byte offset of (row, 16-byte chunk) inside a SW128 block of 128-byte rows.
+__host__ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+// Byte offset of (row, 16-byte chunk) inside a SW64 block of 64-byte rows.
+__host__ __device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t chunk) {
+    return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
+}  // namespace tc
+}  // namespace kda

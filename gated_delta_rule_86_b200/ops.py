@@ -1,0 +1,164 @@
+"""Python binding of the KDA C ABI (include/kda.h).
+
+Argument marshalling only: shapes are checked, outputs are allocated with
+torch (device memory is the only thing torch provides), pointers and the
+current CUDA stream are passed to libkda_b200.so, and a non-OK status becomes
+a :class:`KdaError`.  Every step of the computation runs in the library's
+kernels; there is no CPU path.
+
+Inputs that live in host memory (pinned CPU tensors) are copied to the current
+CUDA device, and results are copied back into host tensors, on the same
+stream: this is the end-to-end form of each call.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import KdaError  # noqa: F401  (re-exported)
+
+_DTYPES = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _io_dtype(*ts):
+    dt = ts[0].dtype
+    if dt not in _DTYPES:
+        raise TypeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
+    for t in ts:
+        if t.dtype != dt:
+            raise TypeError("q, k, v, log_alpha and beta must share one dtype")
+    return _DTYPES[dt]
+
+
+def _to_device(t, dev):
+    if t is None or t.is_cuda:
+        return t
+    return t.to(dev, non_blocking=True)
+
+
+def _prefill_prepare(q, k, v, log_alpha, beta, initial_state, cu_seqlens):
+    on_host = not q.is_cuda
+    dev = torch.device("cuda", torch.cuda.current_device()) if on_host else q.device
+    q, k, v, log_alpha, beta, initial_state, cu_seqlens = (
+        _to_device(x, dev) for x in (q, k, v, log_alpha, beta, initial_state, cu_seqlens))
+    q, k, v, log_alpha, beta = (x.contiguous() for x in (q, k, v, log_alpha, beta))
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, log_alpha must be [B, T, H, d_k] and v [B, T, H, d_v]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    if cu_seqlens is not None:
+        cu_seqlens = cu_seqlens.to(torch.int32).contiguous()
+        if B != 1:
+            raise ValueError("cu_seqlens requires B == 1")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if initial_state is not None:
+        initial_state = initial_state.to(torch.float32).contiguous()
+        if initial_state.shape != (N, H, dk, dv):
+            raise ValueError(f"initial_state must be [{N}, {H}, {dk}, {dv}]")
+    return on_host, (q, k, v, log_alpha, beta, initial_state, cu_seqlens), (B, T, H, dk, dv, N)
+
+
+def _out_dtype(out_dtype):
+    if out_dtype not in _DTYPES:
+        raise TypeError(f"unsupported out_dtype {out_dtype}; use torch.float32 or torch.bfloat16")
+    return _DTYPES[out_dtype]
+
+
+def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state, chunk_size,
+             out_dtype):
+    lib = _lib.load()
+    on_host, (q, k, v, la, beta, s0, cu), (B, T, H, dk, dv, N) = _prefill_prepare(
+        q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    dt = _io_dtype(q, k, v, la, beta)
+    odt = _out_dtype(out_dtype)
+    out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
+    fs = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if output_final_state else None
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(s0), _ptr(cu),
+            ctypes.c_int32(N if cu is not None else 0), B, T, H, dk, dv]
+    if fn_name == "kda_chunk_fwd":
+        status = lib.kda_chunk_fwd(*args, ctypes.c_int32(chunk_size), dt, odt, _ptr(out), _ptr(fs),
+                                   _stream_handle())
+    else:
+        status = lib.kda_recurrent_fwd(*args, dt, odt, _ptr(out), _ptr(fs), _stream_handle())
+    _lib.check(status, fn_name)
+    if on_host:
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_h.copy_(out, non_blocking=True)
+        fs_h = None
+        if fs is not None:
+            fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+            fs_h.copy_(fs, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return out_h, fs_h
+    return out, fs
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
+                  chunk_size=64, out_dtype=torch.float32):
+    """Chunkwise-parallel KDA prefill; returns ``(out, final_state)``.
+
+    q, k, log_alpha: [B, T, H, d_k]; v: [B, T, H, d_v]; beta: [B, T, H] (one
+    dtype: bf16 or fp32).  initial_state: fp32 [N, H, d_k, d_v] or None;
+    cu_seqlens: int32 [N+1] for packed sequences (B == 1) or None.  out has
+    dtype ``out_dtype`` (fp32 by default, the accumulator precision).
+    """
+    return _prefill("kda_chunk_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state,
+                    chunk_size, out_dtype)
+
+
+def kda_recurrent_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
+                      out_dtype=torch.float32):
+    """Token-by-token KDA prefill on CUDA cores (same contract as :func:`kda_chunk_fwd`)."""
+    return _prefill("kda_recurrent_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state,
+                    64, out_dtype)
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, out_dtype=torch.float32):
+    """One decode step; ``state`` (fp32 [B, H, d_k, d_v], on the GPU) is updated in place.
+
+    q, k, log_alpha: [B, H, d_k]; v: [B, H, d_v]; beta: [B, H].  Returns out
+    [B, H, d_v] of ``out_dtype`` (a host tensor when the token inputs were host
+    tensors; ``out``, if given, receives the result).
+    """
+    lib = _lib.load()
+    if not state.is_cuda or state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError("state must be a contiguous fp32 CUDA tensor (it is updated in place)")
+    on_host = not q.is_cuda
+    q, k, v, la, beta = (_to_device(x, state.device).contiguous() for x in (q, k, v, log_alpha, beta))
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or la.shape != q.shape or v.shape != (B, H, dv) or beta.shape != (B, H) \
+            or state.shape != (B, H, dk, dv):
+        raise ValueError("inconsistent shapes for kda_decode_step")
+    dt = _io_dtype(q, k, v, la, beta)
+    if out is not None:
+        out_dtype = out.dtype
+    odt = _out_dtype(out_dtype)
+    o = out if (out is not None and out.is_cuda) else torch.empty((B, H, dv), dtype=out_dtype, device=state.device)
+    status = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(state), _ptr(o),
+                                 B, H, dk, dv, dt, odt, _stream_handle())
+    _lib.check(status, "kda_decode_step")
+    if on_host:
+        oh = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        oh.copy_(o, non_blocking=True)
+        return oh
+    return o
+
+
+def device_error() -> int:
+    """Sync the current stream and return-and-clear the device error word (KDA_OK or KDA_ERR_TIMEOUT)."""
+    return _lib.load().kda_get_last_device_error(_stream_handle())

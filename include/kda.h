@@ -1,0 +1,142 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) KDA operator library, libkda_b200.so.
+ *
+ * KDA (Kimi Delta Attention) is the linear-attention recurrence of
+ * "Hybrid Linear Attention Architectures: Breaking Through the Long-Context
+ * Engineering Bottleneck in LLMs", section "Core Module Design", Stage 3:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,      alpha_t = exp(log_alpha_t)  (per key channel)
+ *
+ * S is d_k x d_v (rows = key channels).  The write term is read as k v^T (the
+ * printed "v k^T" cannot be left-multiplied by the d_k x d_k erase matrix);
+ * the decay acts before the erase (section 2.5 of "Linear Attention KDA Gating
+ * in a 3:1 Hybrid Architecture"); the output is read after the write; q is not
+ * scaled.
+ *
+ * Conventions for every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory and keeps no pointer after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    means the legacy default stream).  Arguments are validated on the host
+ *    before anything is launched; a rejected call launches nothing.
+ *  - Tensors are dense, row-major, with every pointer 16-byte aligned.
+ *  - `dtype` is the element type of q, k, v, log_alpha and beta; `out_dtype`
+ *    that of out (KDA_F32 keeps the full accuracy of the fp32 accumulators:
+ *    rounding the output to bf16 alone moves it by up to 2^-8 of its
+ *    magnitude).  Recurrent states are always fp32.
+ *  - No call throws across the ABI or exits the process; every failure is a
+ *    kda_status.  KDA_ERR_CUDA means a launch or runtime call failed (use
+ *    cudaGetLastError for details).
+ *  - Kernels bound every wait they perform.  A wait that runs out records
+ *    KDA_ERR_TIMEOUT in a device-side error word and the kernel returns early
+ *    (its outputs are then undefined); kda_get_last_device_error reads it.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misaligned pointer, bad cu_seqlens size */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head size, chunk size, dtype */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4        /* a kernel gave up on a bounded wait (device error word) */
+} kda_status;
+
+typedef enum {
+    KDA_F32 = 0,   /* float32 I/O */
+    KDA_BF16 = 1   /* bfloat16 I/O (fp32 accumulation and fp32 state) */
+} kda_dtype;
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel prefill.
+ *
+ * Computes, for every sequence and head, the outputs o_t of all tokens and the
+ * state after the last token, using the chunkwise form of the recurrence
+ * ("Hardware-Aware Chunkwise Parallelism" on the page named above: the
+ * inter-chunk state update and the intra-chunk output equations; section 3 of
+ * "Linear Attention KDA Gating in a 3:1 Hybrid Architecture").  Within a chunk
+ * the per-channel log decays are summed, the WY factors W and U come from the
+ * UT transform T = (I + strict_tril(diag(beta)(K*Gamma)(K/Gamma)^T))^{-1}, and
+ *     U~ = U - W S,   O = (Q*Gamma) S + tril((Q*Gamma)(K/Gamma)^T) U~,
+ *     S <- Diag(gamma) S + (K*gamma/Gamma)^T U~.
+ * The result equals the token recurrence up to rounding.
+ *
+ *   q, k, log_alpha : [B, T, H, d_k]  dtype.  log_alpha <= 0 (alpha in (0, 1]).
+ *   v               : [B, T, H, d_v]  dtype.
+ *   beta            : [B, T, H]       dtype, in [0, 1].
+ *   init_state      : [N, H, d_k, d_v] fp32, or NULL for zero initial states.
+ *   cu_seqlens      : NULL, or int32 [num_seqs + 1] (device) with B == 1:
+ *                     packed sequences, sequence n = tokens cu_seqlens[n] ..
+ *                     cu_seqlens[n+1]-1; ascending, cu_seqlens[0] == 0,
+ *                     cu_seqlens[num_seqs] == T (not checked on the host:
+ *                     reading it would need a device sync).  Chunks never
+ *                     cross sequences; empty sequences are allowed.
+ *   N               : num_seqs when cu_seqlens is given, else B.
+ *   chunk           : chunk length; 64 is supported.
+ *   out             : [B, T, H, d_v] out_dtype (written).
+ *   final_state     : [N, H, d_k, d_v] fp32, or NULL to skip.  It may alias
+ *                     init_state exactly (in-place state update); partial
+ *                     overlap is invalid.
+ * Supported: d_k == 128 and d_v in {64, 128} for bf16 (tensor-core path);
+ * d_k, d_v in {64, 128} for fp32 (fp32 CUDA-core path, fp32 accuracy).
+ * T == 0 is valid (final_state = init_state or zeros).
+ */
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                         const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                         int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k,
+                         int32_t d_v, int32_t chunk, kda_dtype dtype, kda_dtype out_dtype,
+                         void *out, float *final_state, void *stream);
+
+/*
+ * kda_recurrent_fwd -- the same operation as kda_chunk_fwd, evaluated token by
+ * token on CUDA cores with the state in fp32 registers (the RNN mode that
+ * section 3 of "Linear Attention KDA Gating in a 3:1 Hybrid Architecture"
+ * contrasts with the chunked algorithm).  Same arguments and layouts as
+ * kda_chunk_fwd without `chunk`; d_k, d_v in {64, 128}; either dtype.
+ */
+kda_status kda_recurrent_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                             const void *beta, const float *init_state,
+                             const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                             int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                             kda_dtype out_dtype, void *out, float *final_state, void *stream);
+
+/*
+ * kda_decode_step -- one recurrent step for one new token per sequence, with
+ * the fp32 state updated in place (the memory-bound decode step: every state
+ * element is read once and written once).
+ *
+ *   q, k, log_alpha : [B, H, d_k] dtype;  v : [B, H, d_v] dtype;  beta : [B, H] dtype.
+ *   state           : [B, H, d_k, d_v] fp32, read and overwritten.
+ *   out             : [B, H, d_v] out_dtype (written).
+ * Supported: d_k, d_v in {64, 128}.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
+                           const void *beta, float *state, void *out, int32_t B, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, kda_dtype out_dtype,
+                           void *stream);
+
+/* Human-readable name of a status (static string, never NULL). */
+const char *kda_status_string(kda_status s);
+
+/*
+ * Synchronises `stream`, then returns and clears the device-side error word
+ * of the current device: KDA_OK, or KDA_ERR_TIMEOUT if a kernel gave up on a
+ * bounded wait since the last call.  KDA_ERR_CUDA if the sync or read failed.
+ */
+kda_status kda_get_last_device_error(void *stream);
+
+/* Library version string, e.g. "kda_b200 0.1.0 sm_100a". */
+const char *kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H */

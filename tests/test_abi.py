@@ -1,0 +1,84 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects malformed calls on the host before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_86_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_86_b200 import build
+    build.build_library()
+    return _lib.load()
+
+
+def test_header_matches_binding_list():
+    assert declared_symbols() == sorted(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    names = [lib.kda_status_string(i).decode() for i in range(5)]
+    assert names == ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]
+    assert lib.kda_version().decode().startswith("kda_b200")
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: every call below is rejected first
+ODD = ctypes.c_void_p((1 << 20) + 8)   # 8-byte aligned only
+
+
+def chunk(lib, q=FAKE, B=1, T=128, H=2, dk=128, dv=128, chunk_size=64, dtype=_lib.KDA_BF16, cu=None, ns=0,
+          s0=None, fs=None, out=FAKE, odt=_lib.KDA_F32):
+    return lib.kda_chunk_fwd(q, FAKE, FAKE, FAKE, FAKE, s0, cu, ns, B, T, H, dk, dv, chunk_size, dtype, odt, out,
+                             fs, None)
+
+
+def test_rejects_bad_arguments(lib):
+    E, U = _lib.KDA_ERR_INVALID_ARG, _lib.KDA_ERR_UNSUPPORTED
+    assert chunk(lib, q=None) == E
+    assert chunk(lib, out=None) == E
+    assert chunk(lib, B=0) == E
+    assert chunk(lib, T=-1) == E
+    assert chunk(lib, H=0) == E
+    assert chunk(lib, q=ODD) == E
+    assert chunk(lib, dtype=7) == E
+    assert chunk(lib, odt=5) == E
+    assert chunk(lib, chunk_size=0) == E
+    assert chunk(lib, B=2, cu=FAKE, ns=3) == E          # packed batch needs B == 1
+    assert chunk(lib, cu=FAKE, ns=0) == E
+    assert chunk(lib, s0=FAKE, fs=ctypes.c_void_p((1 << 20) + 4096)) == E   # partial overlap
+    assert chunk(lib, dk=96) == U
+    assert chunk(lib, dv=256) == U
+    assert chunk(lib, chunk_size=128) == U
+    assert chunk(lib, dk=64, dtype=_lib.KDA_BF16) == U   # tensor-core path needs d_k = 128
+    rec = lib.kda_recurrent_fwd(FAKE, FAKE, FAKE, FAKE, None, None, None, 0, 1, 8, 1, 64, 64, _lib.KDA_F32,
+                                _lib.KDA_F32, FAKE, None, None)
+    assert rec == E
+    dec = lib.kda_decode_step
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 32, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == U
+    assert dec(ODD, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libkda_b200.so"))
+    with pytest.raises(ImportError):
+        _lib.load()

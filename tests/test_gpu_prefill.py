@@ -1,0 +1,141 @@
+"""Prefill parity against the fp64 oracle (GPU): chunked tensor-core path and
+token-recurrent CUDA-core path, small ragged cases and full-size workloads."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_86_b200 import device_error, inputs, kda_chunk_fwd, kda_recurrent_fwd
+from parity import BF16_TOL, FP32_TOL, NAMES, heads_slice, np64, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_check(fn, x, tol, heads=None):
+    xs = x if heads is None else heads_slice(x, heads)
+    dev = torch.device("cuda")
+    args = [x[n].to(dev) for n in NAMES]
+    s0 = None if x["init_state"] is None else x["init_state"].to(dev)
+    cu = None if x["cu_seqlens"] is None else x["cu_seqlens"].to(dev)
+    out, fs = fn(*args, initial_state=s0, cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    ref_o, ref_s = oracle.recurrent(*(np64(xs[n]) for n in NAMES), init_state=np64(xs["init_state"]),
+                                    cu_seqlens=None if xs["cu_seqlens"] is None else xs["cu_seqlens"].cpu().numpy())
+    if heads is not None:
+        idx = torch.as_tensor(heads, device=dev)
+        out, fs = out.index_select(2, idx), fs.index_select(1, idx)
+    eo, es = rel_err(out, ref_o), rel_err(fs, ref_s)
+    assert eo <= tol and es <= tol, f"out {eo:.3e} state {es:.3e} (tol {tol})"
+    return eo, es
+
+
+# ---- the fp32 workload (Tiny fp32 check) -------------------------------------------------------
+
+def test_tiny_fp32_chunk(cuda_lib):
+    x = inputs.make_prefill("tiny_fp32", device="cpu")
+    run_and_check(kda_chunk_fwd, x, FP32_TOL)
+
+
+def test_tiny_fp32_recurrent(cuda_lib):
+    x = inputs.make_prefill("tiny_fp32", device="cpu")
+    run_and_check(kda_recurrent_fwd, x, FP32_TOL)
+
+
+# ---- small ragged bf16 cases -------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 200, 333])
+@pytest.mark.parametrize("H", [2, 80])   # 2 pairs -> 32-wide d_v slices, 80 pairs -> 64-wide
+def test_chunk_bf16_ragged(cuda_lib, T, H):
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=T, H=H, init_state=True)
+    run_and_check(kda_chunk_fwd, x, BF16_TOL, heads=[0, H - 1] if H > 2 else None)
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+def test_chunk_bf16_batch_dv(cuda_lib, dv):
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=3, T=150, H=3, dv=dv, init_state=False)
+    run_and_check(kda_chunk_fwd, x, BF16_TOL)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128)])
+def test_recurrent_bf16(cuda_lib, dk, dv):
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=97, H=3, dk=dk, dv=dv, init_state=True)
+    run_and_check(kda_recurrent_fwd, x, BF16_TOL)
+
+
+def test_chunk_varlen_small(cuda_lib):
+    lens = [1, 0, 64, 130, 7, 65, 0, 200]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    y = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=int(cu[-1]), H=4, init_state=False)
+    y["cu_seqlens"] = cu
+    y["init_state"] = torch.randn((len(lens), 4, 128, 128), generator=torch.Generator().manual_seed(3)) * 0.1
+    run_and_check(kda_chunk_fwd, y, BF16_TOL)
+    run_and_check(kda_recurrent_fwd, y, BF16_TOL)
+
+
+def test_chunk_strong_decay_fallback(cuda_lib):
+    """Gates with mean log-decay near -3 per token exceed the rebasing range: the kernel
+    takes its exact token-by-token branch for those chunks and must still match."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=300, H=2, mu=-3.0, init_state=True)
+    run_and_check(kda_chunk_fwd, x, BF16_TOL)
+
+
+def test_chunk_mixed_decay(cuda_lib):
+    """Half the heads decay slowly, half extremely fast; per-chunk branch selection."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=256, H=4, init_state=True)
+    fast = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=256, H=4, mu=-4.0, seed=77)
+    x["log_alpha"][:, :, 2:] = fast["log_alpha"][:, :, 2:]
+    run_and_check(kda_chunk_fwd, x, BF16_TOL)
+
+
+def test_chunk_zero_length(cuda_lib):
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=0, H=2, init_state=True)
+    dev = torch.device("cuda")
+    out, fs = kda_chunk_fwd(*(x[n].to(dev) for n in NAMES), initial_state=x["init_state"].to(dev))
+    torch.cuda.synchronize()
+    assert out.shape == (2, 0, 2, 128)
+    assert torch.equal(fs.cpu(), x["init_state"])
+
+
+def test_split_prefill_matches_whole(cuda_lib):
+    """State handoff: prefill(T1) then prefill(T2 | final state) == prefill(T1 + T2)."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=320, H=2, init_state=True)
+    dev = torch.device("cuda")
+    a = [x[n].to(dev) for n in NAMES]
+    o, f = kda_chunk_fwd(*a, initial_state=x["init_state"].to(dev))
+    o1, f1 = kda_chunk_fwd(*(t[:, :128] for t in a), initial_state=x["init_state"].to(dev))
+    o2, f2 = kda_chunk_fwd(*(t[:, 128:] for t in a), initial_state=f1)
+    torch.cuda.synchronize()
+    assert (torch.cat([o1, o2], 1).float() - o.float()).abs().max().item() < 1e-2
+    assert (f2 - f).abs().max().item() < 1e-3
+
+
+# ---- full-size workloads, sampled heads --------------------------------------------------------
+
+def test_prefill_bf16_full(cuda_lib):
+    x = inputs.make_prefill("prefill_bf16", device="cuda")
+    run_and_check(kda_chunk_fwd, x, BF16_TOL, heads=[0, 5, 15])
+
+
+def test_long_bf16_full(cuda_lib):
+    x = inputs.make_prefill("long_bf16", device="cuda")
+    run_and_check(kda_chunk_fwd, x, BF16_TOL, heads=[0, 31])
+
+
+def test_varlen_bf16_full(cuda_lib):
+    x = inputs.make_prefill("varlen_bf16", device="cuda")
+    run_and_check(kda_chunk_fwd, x, BF16_TOL, heads=[3, 20])
+
+
+@pytest.mark.parametrize("fn", [kda_chunk_fwd, kda_recurrent_fwd])
+def test_bf16_output_is_rounded_fp32_output(cuda_lib, fn):
+    """out_dtype=bf16 stores the same fp32 accumulators, rounded to nearest: bit-exact."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=130, H=3, init_state=True)
+    dev = torch.device("cuda")
+    a = [x[n].to(dev) for n in NAMES]
+    o32, f32 = fn(*a, initial_state=x["init_state"].to(dev))
+    o16, f16 = fn(*a, initial_state=x["init_state"].to(dev), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(f16, f32)
