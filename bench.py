@@ -151,20 +151,27 @@ def dist_setup(n_gpus):
     return rank, world, local
 
 
-def barrier(world):
+def barrier(world, device="cuda"):
     import torch
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if device == "cuda":
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a per-rank scalar (the step time) over all ranks; every rank gets it."""
     import torch
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, ms_step_max):
+    """Whole-job throughput: units processed by all ranks / the slowest rank's step time."""
+    return world * units_per_rank / (ms_step_max * 1e-3)
 
 
 # ---- the reference arm: the fp64 oracle on the host ----------------------------------------------------
@@ -265,7 +272,7 @@ def run_kda(args):
         barrier(world)
     clocks = clk.summary()
     ms_step = max_over_ranks(ms / args.steps, world)
-    value = world * tokens / (ms_step * 1e-3)
+    value = weak_scaling_value(tokens, world, ms_step)
     alg_bytes = prefill_alg_bytes(token_heads, w.B * w.H)
     alg_flops = prefill_alg_flops(token_heads)
     achieved_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
@@ -363,6 +370,30 @@ def run_kda(args):
     return 0
 
 
+def run_profile_case(args):
+    """One small launch set for ncu: warm-up launches then the profiled ones.
+
+    chunk:  kda_chunk_fwd on B=1, H=32, T=16384 (0.54 GB of bf16 inputs, above L2).
+    decode: kda_decode_step on the full decode workload state (B=256, H=32, 512 MiB fp32).
+    """
+    import torch
+
+    from gated_delta_rule_86_b200 import inputs, kda_chunk_fwd, kda_decode_step
+    torch.cuda.set_device(0)
+    if args.profile == "chunk":
+        x = inputs.make_prefill(PREFILL_WORKLOAD, device="cuda", T=16384)
+        a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+        for _ in range(3):
+            kda_chunk_fwd(*a, initial_state=x["init_state"])
+    else:
+        d = inputs.make_decode(DECODE_WORKLOAD, device="cuda", steps=4)
+        for i in range(4):
+            kda_decode_step(d["q"][i], d["k"][i], d["v"][i], d["log_alpha"][i], d["beta"][i], d["state"])
+    torch.cuda.synchronize()
+    print(f"profile case {args.profile} done", flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -371,7 +402,11 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--ref-seconds", type=float, default=10.0, help="target CPU seconds per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["chunk", "decode"], default=None,
+                    help="run a small fixed launch set for an ncu capture (no timing output)")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile_case(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
