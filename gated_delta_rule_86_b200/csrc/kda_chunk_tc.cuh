@@ -16,6 +16,15 @@
 //   S    <- Diag(exp(G_last)) S + (K * exp(G_last - G))^T U~
 // which equals the token recurrence exactly in exact arithmetic.
 //
+// Pipeline.  Everything up to W and U depends only on the chunk's own inputs;
+// only the last three lines touch S.  A CTA therefore runs two warp roles:
+//   * prep (warps 4-11): decays, rebased operands, A/P, UT transform, W, U of
+//     chunk n+1, loading chunk n+2's inputs into registers meanwhile;
+//   * chain (warps 0-3): the state-dependent MMAs, output rows and the fp32
+//     state update of chunk n.
+// They hand chunks over through two operand slots (mbarriers full[] / done[]),
+// so the serial state chain only waits on prep when prep is the slower role.
+//
 // Precision (fp32 accumulation in TMEM, fp32 master state in registers, fp32
 // decays and substitution, fp32 or bf16 output):
 //   * A and P need the rebased factors below, whose range exceeds fp16: they are
@@ -36,11 +45,12 @@
 // exceed that (extremely fast forgetting) is evaluated token by token in fp32
 // instead, so every input with finite log_alpha gets a correct result.
 //
-// Work decomposition: one CTA per (sequence, head, NV-wide slice of d_v).  The
+// Work decomposition: one CTA per (sequence, head, 32-wide slice of d_v).  The
 // d_v columns of S evolve independently (column j of U~ depends only on
 // column j of S), so slicing d_v multiplies the parallelism of the sequential
-// chunk chain; the d_v-independent work (decays, A, P, T, W) is recomputed per
-// slice.  Packed variable-length batches are scheduled longest-first.
+// chunk chain; the d_v-independent prep is recomputed per slice (moving it
+// between SMs would cost more than recomputing it).  Packed variable-length
+// batches are scheduled longest-first.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -54,48 +64,64 @@ namespace kda {
 
 constexpr int kChunk = 64;
 constexpr int kDK = 128;
+constexpr int kNV = 32;  // value columns per CTA
 // Largest per-channel cumulative decay (in natural-log units) allowed on either
 // side of the chunk's middle token for the tensor-core path.  Factors of the
 // rebased products stay within exp(+-40); their sums stay far below the fp32
 // and bf16 overflow threshold exp(88.7).
 constexpr float kRangeLimit = 40.f;
 
-// ---- shared-memory plan (bytes, all blocks 1024-aligned) ----------------------------------------
-template <int NV>
+constexpr int kChainThreads = 128;  // warps 0-3
+constexpr int kPrepThreads = 256;   // warps 4-11
+constexpr int kThreads = kChainThreads + kPrepThreads;
+constexpr uint32_t kBarPrep = 1, kBarChain = 2;  // named barrier ids
+
+// ---- shared-memory plan (byte offsets; operand tiles 1024-aligned) -------------------------------
 struct ChunkSmem {
-    static constexpr int kTile = kChunk * kDK * 2;   // one [64 x 128] 16-bit operand (16 KB)
-    // bf16 operands of A_raw and P_raw; dead once those MMAs complete, then
-    // reused as fp32 scratch for the UT transform (A and T, 2 x 16 KB).
+    static constexpr int kTile = kChunk * kDK * 2;   // [64 x 128] 16-bit operand (16 KB)
+    // prep: bf16 operands of A_raw and P_raw; dead once those MMAs complete,
+    // then reused as fp32 scratch of the UT transform
     static constexpr int kKr = 0;                    // K exp(G - Gref)            A of A_raw
-    static constexpr int kQrHi = kKr + kTile;        // Q exp(G - Gref), hi part   A of P_raw
-    static constexpr int kQrLo = kQrHi + kTile;      //                 lo part
-    static constexpr int kKnHi = kQrLo + kTile;      // K exp(Gref - G), hi part   B of A_raw, P_raw
-    static constexpr int kKnLo = kKnHi + kTile;      //                 lo part    B of P_raw
-    // fp16 operands
-    static constexpr int kKg = kKnLo + kTile;        // K exp(G)                   B of W (MN-major)
-    static constexpr int kQg = kKg + kTile;          // Q exp(G)                   A of Q S
-    static constexpr int kKd = kQg + kTile;          // K exp(Glast - G)           A of Kd^T U~ (MN-major)
-    static constexpr int kT = kKd + kTile;           // T diag(beta) [64 x 64]     A of W, U
-    static constexpr int kP = kT + kChunk * kChunk * 2;           // tril(P) [64 x 64]   A of P U~
-    static constexpr int kV = kP + kChunk * kChunk * 2;           // V slice [64 x NV]   B of U
-    static constexpr int kW = kV + kChunk * NV * 2;               // W [64 x 128]        A of -W S
-    static constexpr int kS = kW + kTile;                         // S [128 x NV]        B of W S, Q S
-    static constexpr int kUt = kS + kDK * NV * 2;                 // U~ [64 x NV]        B of P U~, Kd^T U~
-    static constexpr int kX = kUt + kChunk * NV * 2;              // fp32 [16 x 48] substitution scratch
-    static constexpr int kBeta = kX + 16 * 48 * 4;                // fp32 [64]
-    static constexpr int kG0 = kBeta + 64 * 4;                    // fp32 [128] decay after token 0
-    static constexpr int kGref = kG0 + kDK * 4;                   // fp32 [128] decay after token 31
-    static constexpr int kGlast = kGref + kDK * 4;                // fp32 [128] decay after token 63
-    static constexpr int kTot = kGlast + kDK * 4;                 // fp32 [8][128] scan totals
-    static constexpr int kEnd = kTot + 8 * kDK * 4;
-    static constexpr int kBytes = kEnd + 1024;  // + alignment slack
-    // exact-path scratch: [128][2 NV] fp32 partial products inside the A/P region
-    static_assert(kDK * 2 * NV * 4 <= kKg, "exact-path scratch must fit the A/P operand region");
+    static constexpr int kQrHi = kKr + kTile;        // Q exp(G - Gref), hi        A of P_raw
+    static constexpr int kQrLo = kQrHi + kTile;      //                  lo
+    static constexpr int kKnHi = kQrLo + kTile;      // K exp(Gref - G), hi        B of A_raw, P_raw
+    static constexpr int kKnLo = kKnHi + kTile;      //                  lo
+    static constexpr int kLd = 68;                   // fp32 row stride of A and T (bank spread, 16-B rows)
+    static constexpr int kA32 = 0;                   // fp32 [64][kLd] beta_r A_rs (strict lower)
+    static constexpr int kT32 = kA32 + kChunk * kLd * 4;     // fp32 [64][kLd] T
+    static constexpr int kX32 = kT32 + kChunk * kLd * 4;     // fp32 [3][16][16] block products
+    // prep-internal fp16 operands
+    static constexpr int kKg = kKnLo + kTile;        // K exp(G) [64 x 128]        B of W (MN-major)
+    static constexpr int kTb = kKg + kTile;          // T diag(beta) [64 x 64]     A of W, U
+    static constexpr int kV = kTb + kChunk * kChunk * 2;          // V slice [64 x 32]  B of U
+    // hand-over slots (fp16): Qg, Kd double-buffered; P, W single
+    static constexpr int kQg0 = kV + kChunk * kNV * 2;            // Q exp(G)          A of Q S
+    static constexpr int kQg1 = kQg0 + kTile;
+    static constexpr int kKd0 = kQg1 + kTile;                     // K exp(Glast - G)  A of Kd^T U~
+    static constexpr int kKd1 = kKd0 + kTile;
+    static constexpr int kP = kKd1 + kTile;                       // tril(P) [64 x 64] A of P U~
+    static constexpr int kW = kP + kChunk * kChunk * 2;           // W [64 x 128]      A of -W S
+    // chain-internal fp16 operands
+    static constexpr int kS = kW + kTile;                         // S [128 x 32]      B of W S, Q S
+    static constexpr int kUt = kS + kDK * kNV * 2;                // U~ [64 x 32]      B of P U~, Kd^T U~
+    // small fp32 arrays
+    static constexpr int kGamma = kUt + kChunk * kNV * 2;         // [2][128] exp(Glast), per slot
+    static constexpr int kBeta = kGamma + 2 * kDK * 4;            // [64]
+    static constexpr int kG0 = kBeta + kChunk * 4;                // [128] decay after token 0
+    static constexpr int kGref = kG0 + kDK * 4;                   // [128] decay after token 31
+    static constexpr int kGlast = kGref + kDK * 4;                // [128] decay after token 63
+    static constexpr int kTot = kGlast + kDK * 4;                 // [16][128] scan totals
+    static constexpr int kRed = kTot + 16 * kDK * 4;              // chain exact path: 292 floats
+    static constexpr int kFlags = kRed + 300 * 4;                 // int[2] exact-path flags
+    static constexpr int kEnd = kFlags + 16;
+    static constexpr int kBytes = kEnd + 1024;                    // + alignment slack
+    static_assert(kX32 + 3 * 256 * 4 <= kKg, "UT scratch must fit the A/P operand region");
+    static_assert(kBytes <= 232448, "shared memory plan exceeds 227 KB");
 };
 
 // TMEM columns (fp32 accumulators).  M=64 tiles use lanes 0-15 of each 32-lane
 // subpartition (row m -> lane (m % 16) + 32 (m / 16)); M=128 tiles use all lanes.
-constexpr uint32_t kTmA = 0, kTmP = 64, kTmSn = 0, kTmW = 128, kTmU = 256, kTmO = 384;
+constexpr uint32_t kTmA = 0, kTmP = 64, kTmW = 128, kTmU0 = 256, kTmO = 320, kTmSn = 352;
 constexpr uint32_t kTmCols = 512;
 
 // Descriptor of k-step `kk` (16 elements along K) of a K-major SW128 operand with `rows` rows.
@@ -138,12 +164,16 @@ __device__ __forceinline__ uint4 pack8_bf16(const float *f) {
 __device__ __forceinline__ uint4 pack8_h(const float *f) {
     return make_uint4(pack_h(f[0], f[1]), pack_h(f[2], f[3]), pack_h(f[4], f[5]), pack_h(f[6], f[7]));
 }
-// bf16 hi part and the bf16 rounding of the remainder (x ~= hi + lo to ~16 bits).
+// Two-term bf16 split x ~= hi + lo: hi is x truncated to bf16 (exact in fp32),
+// lo the bf16 rounding of the exact remainder; |x - hi - lo| <= 2^-15 |x|.
 __device__ __forceinline__ void split8_bf16(const float *f, uint4 &hi, uint4 &lo) {
     float r[8];
+    uint32_t h[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) r[i] = f[i] - __bfloat162float(__float2bfloat16_rn(f[i]));
-    hi = pack8_bf16(f);
+    for (int i = 0; i < 8; ++i) r[i] = f[i] - __uint_as_float(__float_as_uint(f[i]) & 0xffff0000u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __byte_perm(__float_as_uint(f[2 * i]), __float_as_uint(f[2 * i + 1]), 0x7632);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
     lo = pack8_bf16(r);
 }
 
@@ -158,43 +188,66 @@ template <> __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16
     reinterpret_cast<uint4 *>(dst)[1] = pack8_bf16(f + 8);
 }
 
-// Wait for the next completion of the CTA's MMA barrier, then make every
-// thread agree on whether the wait succeeded.  Returns false on timeout.
-__device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t &phase, volatile int *abort_flag) {
-    tc::mbar_wait(bar, phase, abort_flag);
-    phase ^= 1u;
-    tc::tc_fence_after();
-    __syncthreads();
-    return *abort_flag == 0;
+// Sum 32 per-lane values across the warp so that lane l ends with the warp-wide
+// sum of value l (recursive halving: 31 shuffles for 32 values).
+__device__ __forceinline__ void warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = upper ? v[i] : v[i + off];
+            const float keep = upper ? v[i + off] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
 }
 
-template <int NV, typename TO>
-__global__ void __launch_bounds__(128, 1)
+// One thread of a role waits on an mbarrier phase (bounded), then the role's
+// named barrier spreads the outcome.  Returns false on timeout or abort.
+__device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, bool leader, uint32_t bar_id,
+                                          uint32_t nthreads, volatile int *abort_flag) {
+    bool ok = true;
+    if (leader) ok = tc::mbar_wait(bar, parity, abort_flag);
+    const bool failed = tc::named_sync_or(bar_id, nthreads, !ok);
+    tc::tc_fence_after();
+    return !failed;
+}
+
+struct ChunkArgs {
+    const __nv_bfloat16 *q, *k, *v, *log_alpha, *beta;
+    const float *init_state;
+    float *final_state;
+    int H, DV;
+};
+
+template <typename TO>
+__global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ log_alpha,
                     const __nv_bfloat16 *__restrict__ beta, const float *init_state,
                     const int32_t *__restrict__ cu_seqlens, int num_seqs, int T, int H, int DV,
                     TO *__restrict__ out, float *final_state) {
-    using SM = ChunkSmem<NV>;
+    using SM = ChunkSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = tc::smem_u32(sm);
-    float *sX = reinterpret_cast<float *>(sm + SM::kX);
+    float *sGamma = reinterpret_cast<float *>(sm + SM::kGamma);
     float *sBeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *sG0 = reinterpret_cast<float *>(sm + SM::kG0);
     float *sGref = reinterpret_cast<float *>(sm + SM::kGref);
     float *sGlast = reinterpret_cast<float *>(sm + SM::kGlast);
     float *sTot = reinterpret_cast<float *>(sm + SM::kTot);
-    float *sA = reinterpret_cast<float *>(sm + SM::kKr);                   // fp32 [64][64]
-    float *sT = reinterpret_cast<float *>(sm + SM::kKr) + kChunk * kChunk;  // fp32 [64][64]
+    float *sRed = reinterpret_cast<float *>(sm + SM::kRed);
+    volatile int *sFlags = reinterpret_cast<volatile int *>(sm + SM::kFlags);
 
-    __shared__ uint64_t bar_mma;
+    __shared__ uint64_t bar_m1, bar_m1p, bar_m2, bar_m3, bar_m4, full[2], done[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ int s_slot;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nslices = DV / NV;
+    const int nslices = DV / kNV;
     const int slice = blockIdx.x % nslices;
     const int pair = blockIdx.x / nslices;
     const int h = pair % H;
@@ -208,12 +261,19 @@ kda_chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         t0 = (int64_t)n * T;
         t1 = t0 + T;
     }
-    const int64_t len = t1 - t0;
-    const int nchunks = static_cast<int>((len + kChunk - 1) / kChunk);
-    const int vcol0 = slice * NV;  // first value column of this slice
+    const int nchunks = static_cast<int>((t1 - t0 + kChunk - 1) / kChunk);
+    const int vcol0 = slice * kNV;
 
     if (tid == 0) {
-        tc::mbar_init(&bar_mma, 1);
+        tc::mbar_init(&bar_m1, 1);
+        tc::mbar_init(&bar_m1p, 1);
+        tc::mbar_init(&bar_m2, 1);
+        tc::mbar_init(&bar_m3, 1);
+        tc::mbar_init(&bar_m4, 1);
+        tc::mbar_init(&full[0], 1);
+        tc::mbar_init(&full[1], 1);
+        tc::mbar_init(&done[0], 1);
+        tc::mbar_init(&done[1], 1);
         tc::fence_mbar_init();
         abort_flag = 0;
     }
@@ -226,455 +286,554 @@ kda_chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     tc::tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
     const uint32_t tl = tc::tmem_lane_base(warp);
-    uint32_t phase = 0;
 
-    // ---- fp32 master state: thread i owns key row i, NV value columns -----------------------------
-    float S[NV];
-    const size_t state_base = ((size_t)n * H + h) * kDK * DV;
+    if (warp < 4) {
+        // ===================================== chain role =====================================
+        const bool leader = tid == 0;
+        float S[kNV];  // fp32 master state: key row tid, this slice's value columns
+        const size_t state_base = ((size_t)n * H + h) * kDK * DV + (size_t)tid * DV + vcol0;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) S[j] = init_state ? init_state[state_base + (size_t)tid * DV + vcol0 + j] : 0.f;
-
-    // fp16 copy of S as the MN-major B operand [128 K-rows x NV]
-    auto write_state_operand = [&]() {
+        for (int j = 0; j < kNV; ++j) S[j] = init_state ? init_state[state_base + j] : 0.f;
+        auto write_state_operand = [&]() {
 #pragma unroll
-        for (int j = 0; j < NV / 8; ++j)
-            *reinterpret_cast<uint4 *>(sm + SM::kS + tile_chunk(tid, j, kDK, NV)) = pack8_h(&S[8 * j]);
-    };
-    write_state_operand();
-
-    // Exact evaluation of one chunk, token by token in fp32 (the recurrence
-    // itself), starting from the state in registers.  Used when the chunk's
-    // decays exceed the rebasing range or an fp16 operand overflowed.
-    auto exact_chunk = [&](int64_t tok0, int L) {
-        float *red = reinterpret_cast<float *>(sm + SM::kKr);  // [128][2 NV]
-        float *col = reinterpret_cast<float *>(sm + SM::kKg);  // [2 NV]
-        for (int r = 0; r < L; ++r) {
-            const int64_t row = (tok0 + r) * H + h;
-            const float a = expf(__bfloat162float(log_alpha[row * kDK + tid]));
-            const float kk = __bfloat162float(k[row * kDK + tid]);
-            const float qq = __bfloat162float(q[row * kDK + tid]);
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                S[j] *= a;
-                red[tid * (2 * NV) + j] = S[j] * kk;
-                red[tid * (2 * NV) + NV + j] = S[j] * qq;
-            }
-            float kq = kk * qq;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
-            if (lane == 0) sX[warp] = kq;
-            __syncthreads();
-            if (tid < 2 * NV) {
-                float acc = 0.f;
-                for (int i = 0; i < kDK; ++i) acc += red[i * (2 * NV) + tid];
-                col[tid] = acc;
-            }
-            __syncthreads();
-            const float kqs = sX[0] + sX[1] + sX[2] + sX[3];
-            const float b = __bfloat162float(beta[row]);
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const float u = b * (__bfloat162float(v[row * DV + vcol0 + j]) - col[j]);
-                if (tid == j) out[row * DV + vcol0 + j] = from_f32<TO>(fmaf(u, kqs, col[NV + j]));
-                S[j] = fmaf(kk, u, S[j]);
-            }
-            __syncthreads();
-        }
+            for (int j = 0; j < kNV / 8; ++j)
+                *reinterpret_cast<uint4 *>(sm + SM::kS + tile_chunk(tid, j, kDK, kNV)) = pack8_h(&S[8 * j]);
+            tc::fence_async_smem();
+        };
         write_state_operand();
-        __syncthreads();
-    };
 
-    for (int c = 0; c < nchunks; ++c) {
-        const int64_t tok0 = t0 + (int64_t)c * kChunk;  // first token of the chunk
-        const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
-
-        // ================= phase E: decays, range check, rebased operands =================
-        const int cg = tid & 15, tg = tid >> 4;  // 8 channels [8cg, 8cg+8), 8 tokens [8tg, 8tg+8)
-        float G[8][8];                            // cumulative decay, this thread's 8 x 8 block
-        {
-            float run[8];
+        // token-by-token fp32 evaluation of one chunk from the state in registers
+        auto exact_chunk = [&](int64_t tok0, int L) {
+            for (int r = 0; r < L; ++r) {
+                const int64_t row = (tok0 + r) * H + h;
+                const float a = expf(__bfloat162float(log_alpha[row * kDK + tid]));
+                const float kk = __bfloat162float(k[row * kDK + tid]);
+                const float qq = __bfloat162float(q[row * kDK + tid]);
+                float va[32], vb[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) run[i] = 0.f;
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const int r = tg * 8 + rr;
-                float g8[8];
-                if (r < L) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(log_alpha + ((tok0 + r) * H + h) * kDK + cg * 8);
-                    unpack8(u, g8);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) g8[i] = 0.f;
+                for (int j = 0; j < kNV; ++j) {
+                    S[j] *= a;
+                    va[j] = S[j] * kk;
+                    vb[j] = S[j] * qq;
                 }
+                warp_transpose_sum32(va, lane);
+                warp_transpose_sum32(vb, lane);
+                float kq = kk * qq;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
+                sRed[warp * 64 + lane] = va[0];
+                sRed[warp * 64 + 32 + lane] = vb[0];
+                if (lane == 0) sRed[256 + warp] = kq;
+                tc::named_sync(kBarChain, kChainThreads);
+                if (warp == 0) {
+                    float aa = 0.f, bb = 0.f, kqs = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        aa += sRed[w * 64 + lane];
+                        bb += sRed[w * 64 + 32 + lane];
+                        kqs += sRed[256 + w];
+                    }
+                    const float u = __bfloat162float(beta[row]) *
+                                    (__bfloat162float(v[row * DV + vcol0 + lane]) - aa);
+                    sRed[260 + lane] = u;
+                    out[row * DV + vcol0 + lane] = from_f32<TO>(fmaf(u, kqs, bb));
+                }
+                tc::named_sync(kBarChain, kChainThreads);
+#pragma unroll
+                for (int j = 0; j < kNV; ++j) S[j] = fmaf(kk, sRed[260 + j], S[j]);
+                tc::named_sync(kBarChain, kChainThreads);
+            }
+            write_state_operand();
+        };
+
+        uint32_t ph_m3 = 0, ph_m4 = 0;
+        tc::named_sync(kBarChain, kChainThreads);
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            const int64_t tok0 = t0 + (int64_t)c * kChunk;
+            const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
+            if (!role_wait(&full[b], (c >> 1) & 1, leader, kBarChain, kChainThreads, &abort_flag)) break;
+            const bool exact = sFlags[b] != 0;
+            const float gam = sGamma[b * kDK + tid];
+            bool released = false;
+            bool bad = exact;
+            if (!exact) {
+                // ---- M3: U~ = U - W S (accumulated onto U),  O = Qg S ----
+                const uint32_t tU = kTmU0 + b * kNV;
+                const uint32_t sQg = b ? SM::kQg1 : SM::kQg0, sKd = b ? SM::kKd1 : SM::kKd0;
+                if (leader) {
+                    constexpr uint32_t idNeg = tc::make_idesc(64, kNV, tc::kF16, false, true, true);
+                    constexpr uint32_t idO = tc::make_idesc(64, kNV, tc::kF16, false, true);
+#pragma unroll
+                    for (int kk = 0; kk < kDK / 16; ++kk) {
+                        const uint64_t bdesc = desc_mnmajor(sbase + SM::kS, kDK, kNV, kk);
+                        tc::mma_f16(tmem + tU, desc_kmajor(sbase + SM::kW, kChunk, kk), bdesc, idNeg, true);
+                        tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + sQg, kChunk, kk), bdesc, idO, kk > 0);
+                    }
+                    tc::mma_commit(&bar_m3);
+                }
+                if (!role_wait(&bar_m3, ph_m3, leader, kBarChain, kChainThreads, &abort_flag)) break;
+                ph_m3 ^= 1u;
+                // U~ -> fp16 B operand; a value outside the fp16 range sends the chunk to the exact path
+                {
+                    const int r = warp * 16 + lane;
+#pragma unroll
+                    for (int c16 = 0; c16 < kNV / 16; ++c16) {
+                        float u16[16];
+                        tc::tmem_ld16(tmem + tl + tU + c16 * 16, u16);
+                        tc::tmem_ld_wait();
+                        if (lane < 16) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) bad |= !(fabsf(u16[i]) <= 65000.f);
+                            *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16, kChunk, kNV)) =
+                                pack8_h(u16);
+                            *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16 + 1, kChunk, kNV)) =
+                                pack8_h(u16 + 8);
+                        }
+                    }
+                    tc::fence_async_smem();
+                    tc::tc_fence_before();
+                    bad = tc::named_sync_or(kBarChain, kChainThreads, bad);
+                }
+                if (!bad) {
+                    // ---- M4: O += P U~,  Sn = Kd^T U~ ----
+                    if (leader) {
+                        tc::tc_fence_after();
+                        constexpr uint32_t idO = tc::make_idesc(64, kNV, tc::kF16, false, true);
+                        constexpr uint32_t idS = tc::make_idesc(128, kNV, tc::kF16, true, true);
+#pragma unroll
+                        for (int kk = 0; kk < kChunk / 16; ++kk) {
+                            const uint64_t bdesc = desc_mnmajor(sbase + SM::kUt, kChunk, kNV, kk);
+                            tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + SM::kP, kChunk, kk), bdesc, idO, true);
+                            tc::mma_f16(tmem + kTmSn, desc_mnmajor(sbase + sKd, kChunk, kDK, kk), bdesc, idS,
+                                        kk > 0);
+                        }
+                        tc::mma_commit(&bar_m4);
+                    }
+                    if (!role_wait(&bar_m4, ph_m4, leader, kBarChain, kChainThreads, &abort_flag)) break;
+                    ph_m4 ^= 1u;
+                    // every MMA that read the slot has completed: hand it back to prep
+                    if (leader) tc::mbar_arrive(&done[b]);
+                    released = true;
+                    // ---- epilogue: output rows, state update ----
+                    const int r = warp * 16 + lane;
+                    float o[kNV];
+#pragma unroll
+                    for (int c16 = 0; c16 < kNV / 16; ++c16) {
+                        float o16[16];
+                        tc::tmem_ld16(tmem + tl + kTmO + c16 * 16, o16);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[c16 * 16 + i] = o16[i];
+                    }
+                    float sn[kNV];
+#pragma unroll
+                    for (int c16 = 0; c16 < kNV / 16; ++c16) {
+                        float s16[16];
+                        tc::tmem_ld16(tmem + tl + kTmSn + c16 * 16, s16);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) sn[c16 * 16 + i] = s16[i];
+                    }
+                    bool obad = false;
+                    if (lane < 16)
+#pragma unroll
+                        for (int i = 0; i < kNV; ++i) obad |= !(fabsf(o[i]) <= 3.0e38f);
+                    tc::tc_fence_before();
+                    bad = tc::named_sync_or(kBarChain, kChainThreads, obad);
+                    if (!bad) {
+                        if (lane < 16 && r < L) {
+                            TO *dst = out + ((tok0 + r) * H + h) * DV + vcol0;
+#pragma unroll
+                            for (int c16 = 0; c16 < kNV / 16; ++c16) store16<TO>(dst + c16 * 16, &o[c16 * 16]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < kNV; ++j) S[j] = fmaf(gam, S[j], sn[j]);
+                        write_state_operand();
+                        tc::tc_fence_before();
+                        tc::named_sync(kBarChain, kChainThreads);
+                        continue;
+                    }
+                }
+            }
+            // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
+            if (!released && leader) tc::mbar_arrive(&done[b]);
+            exact_chunk(tok0, L);
+            tc::tc_fence_before();
+            tc::named_sync(kBarChain, kChainThreads);
+        }
+        if (final_state && abort_flag == 0) {
+#pragma unroll
+            for (int j = 0; j < kNV; ++j) final_state[state_base + j] = S[j];
+        }
+    } else {
+        // ===================================== prep role ======================================
+        const int tp = tid - kChainThreads;      // 0..255
+        const bool leader = tp == 0;
+        const int cg = tp & 15, tg = tp >> 4;    // 8 channels [8cg, 8cg+8), 4 tokens [4tg, 4tg+4)
+        uint4 rg[4], rk[4], rq[4], rv;
+        float rb = 0.f;
+        auto load_raw = [&](int c) {
+            const int64_t tok0 = t0 + (int64_t)c * kChunk;
+            const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = tg * 4 + rr;
+                if (r < L) {
+                    const int64_t off = ((tok0 + r) * H + h) * kDK + cg * 8;
+                    rg[rr] = *reinterpret_cast<const uint4 *>(log_alpha + off);
+                    rk[rr] = *reinterpret_cast<const uint4 *>(k + off);
+                    rq[rr] = *reinterpret_cast<const uint4 *>(q + off);
+                } else {
+                    rg[rr] = rk[rr] = rq[rr] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            const int vr = tp >> 2, vj = tp & 3;
+            rv = (vr < L) ? *reinterpret_cast<const uint4 *>(v + ((tok0 + vr) * H + h) * DV + vcol0 + vj * 8)
+                          : make_uint4(0, 0, 0, 0);
+            rb = (tp < kChunk && tp < L) ? __bfloat162float(beta[(tok0 + tp) * H + h]) : 0.f;
+        };
+        uint32_t ph_m1 = 0, ph_m1p = 0, ph_m2 = 0;
+        float *sA = reinterpret_cast<float *>(sm + SM::kA32);
+        float *sT = reinterpret_cast<float *>(sm + SM::kT32);
+        float *sX = reinterpret_cast<float *>(sm + SM::kX32);
+        if (nchunks > 0) load_raw(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            // slot b (Qg[b], Kd[b], U[b], flags, gamma) is free once the chain finished chunk c-2
+            if (c >= 2 && !role_wait(&done[b], ((c - 2) >> 1) & 1, leader, kBarPrep, kPrepThreads, &abort_flag))
+                break;
+
+            // ---- decays (fp32 scan over the chunk, per channel) ----
+            float G[4][8];
+            {
+                float run[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) run[i] = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    float g8[8];
+                    unpack8(rg[rr], g8);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        run[i] += g8[i];
+                        G[rr][i] = run[i];
+                    }
+                }
+                // lanes 16-31 hold the odd token group of the warp's pair: add the even one's total
+                const int w4 = warp - 4;
+                float pair_tot[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    run[i] += g8[i];
-                    G[rr][i] = run[i];
+                    const float lower = __shfl_up_sync(0xffffffffu, run[i], 16);
+                    const float add = (lane >= 16) ? lower : 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) G[rr][i] += add;
+                    pair_tot[i] = run[i] + add;  // lanes 16-31: total of the warp's 8 tokens
+                }
+                if (lane >= 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sTot[w4 * kDK + cg * 8 + i] = pair_tot[i];
+                }
+                if (tp < kChunk) sBeta[tp] = rb;
+                {
+                    float f[8];
+                    unpack8(rv, f);
+                    *reinterpret_cast<uint4 *>(sm + SM::kV + tile_chunk(tp >> 2, tp & 3, kChunk, kNV)) = pack8_h(f);
+                }
+                tc::named_sync(kBarPrep, kPrepThreads);
+                float off[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) off[i] = 0.f;
+                for (int p = 0; p < w4; ++p)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) off[i] += sTot[p * kDK + cg * 8 + i];
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) G[rr][i] += off[i];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (tg == 0) sG0[cg * 8 + i] = G[0][i];
+                    if (tg == 7) sGref[cg * 8 + i] = G[3][i];
+                    if (tg == 15) sGlast[cg * 8 + i] = G[3][i];
                 }
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sTot[tg * kDK + cg * 8 + i] = run[i];
-            __syncthreads();
-            float off[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) off[i] = 0.f;
-            for (int p = 0; p < tg; ++p)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) off[i] += sTot[p * kDK + cg * 8 + i];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) G[rr][i] += off[i];
-            // decays after tokens 0, 31 and 63 (padding rows carry log_alpha = 0)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (tg == 0) sG0[cg * 8 + i] = G[0][i];
-                if (tg == 3) sGref[cg * 8 + i] = G[7][i];
-                if (tg == 7) sGlast[cg * 8 + i] = G[7][i];
+            tc::named_sync(kBarPrep, kPrepThreads);
+            bool bad = false;
+            if (tp < kDK) {
+                const float g0 = sG0[tp], gr = sGref[tp], gl = sGlast[tp];
+                bad = !((g0 - gr <= kRangeLimit) && (gr - gl <= kRangeLimit));
             }
-        }
-        if (tid < 64) sBeta[tid] = (tid < L) ? __bfloat162float(beta[(tok0 + tid) * H + h]) : 0.f;
-        __syncthreads();
-        {
-            const float g0 = sG0[tid], gr = sGref[tid], gl = sGlast[tid];
-            const bool bad = !((g0 - gr <= kRangeLimit) && (gr - gl <= kRangeLimit));
-            if (__syncthreads_or(bad)) {
-                exact_chunk(tok0, L);
+            if (tc::named_sync_or(kBarPrep, kPrepThreads, bad)) {
+                // decays too fast for the rebased products: the chain evaluates it exactly
+                if (c + 1 < nchunks) load_raw(c + 1);
+                if (leader) {
+                    sFlags[b] = 1;
+                    tc::mbar_arrive(&full[b]);
+                }
                 continue;
             }
-        }
-        {
-            float gref[8], erefabs[8], elast[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                gref[i] = sGref[cg * 8 + i];
-                erefabs[i] = expf(gref[i]);                       // exp(Gref)
-                elast[i] = expf(sGlast[cg * 8 + i] - gref[i]);   // exp(Glast - Gref)
-            }
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const int r = tg * 8 + rr;
-                float kf[8], qf[8];
-                if (r < L) {
-                    const int64_t row = (tok0 + r) * H + h;
-                    unpack8(*reinterpret_cast<const uint4 *>(k + row * kDK + cg * 8), kf);
-                    unpack8(*reinterpret_cast<const uint4 *>(q + row * kDK + cg * 8), qf);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) kf[i] = qf[i] = 0.f;
-                }
-                float kr[8], qr[8], kn[8], kg[8], qg[8], kd[8];
+
+            // ---- rebased and decayed operands ----
+            {
+                float gref[8], erefabs[8], elast[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float dg = G[rr][i] - gref[i];
-                    const float e1 = fast_exp(dg), e2 = fast_exp(-dg);
-                    kr[i] = kf[i] * e1;
-                    qr[i] = qf[i] * e1;
-                    kn[i] = kf[i] * e2;
-                    kg[i] = kr[i] * erefabs[i];
-                    qg[i] = qr[i] * erefabs[i];
-                    kd[i] = kn[i] * elast[i];
+                    gref[i] = sGref[cg * 8 + i];
+                    erefabs[i] = fast_exp(gref[i]);                       // exp(Gref)
+                    elast[i] = fast_exp(sGlast[cg * 8 + i] - gref[i]);   // exp(Glast - Gref)
                 }
-                const uint32_t off = tile_chunk(r, cg, kChunk, kDK);
-                uint4 hi, lo;
-                *reinterpret_cast<uint4 *>(sm + SM::kKr + off) = pack8_bf16(kr);
-                split8_bf16(qr, hi, lo);
-                *reinterpret_cast<uint4 *>(sm + SM::kQrHi + off) = hi;
-                *reinterpret_cast<uint4 *>(sm + SM::kQrLo + off) = lo;
-                split8_bf16(kn, hi, lo);
-                *reinterpret_cast<uint4 *>(sm + SM::kKnHi + off) = hi;
-                *reinterpret_cast<uint4 *>(sm + SM::kKnLo + off) = lo;
-                *reinterpret_cast<uint4 *>(sm + SM::kKg + off) = pack8_h(kg);
-                *reinterpret_cast<uint4 *>(sm + SM::kQg + off) = pack8_h(qg);
-                *reinterpret_cast<uint4 *>(sm + SM::kKd + off) = pack8_h(kd);
-            }
-            // V slice [64 x NV] (fp16) as the MN-major B operand of U
-            for (int idx = tid; idx < kChunk * (NV / 8); idx += 128) {
-                const int r = idx / (NV / 8), j = idx % (NV / 8);
-                float f[8];
-                if (r < L) {
-                    unpack8(*reinterpret_cast<const uint4 *>(v + ((tok0 + r) * H + h) * DV + vcol0 + j * 8), f);
-                } else {
+                const uint32_t sQg = b ? SM::kQg1 : SM::kQg0, sKd = b ? SM::kKd1 : SM::kKd0;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] = 0.f;
-                }
-                *reinterpret_cast<uint4 *>(sm + SM::kV + tile_chunk(r, j, kChunk, NV)) = pack8_h(f);
-            }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ================= M1: A_raw = Kr Kn^T,  P_raw = Qr Kn^T (split) =================
-        if (tid == 0) {
-            tc::tc_fence_after();
-            constexpr uint32_t id = tc::make_idesc(64, 64, tc::kBF16, false, false);
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int r = tg * 4 + rr;
+                    float kf[8], qf[8];
+                    unpack8(rk[rr], kf);
+                    unpack8(rq[rr], qf);
+                    float kr[8], qr[8], kn[8], kg[8], qg[8], kd[8];
 #pragma unroll
-            for (int kk = 0; kk < kDK / 16; ++kk) {
-                const uint64_t bhi = desc_kmajor(sbase + SM::kKnHi, kChunk, kk);
-                const uint64_t blo = desc_kmajor(sbase + SM::kKnLo, kChunk, kk);
-                const uint64_t qhi = desc_kmajor(sbase + SM::kQrHi, kChunk, kk);
-                tc::mma_f16(tmem + kTmA, desc_kmajor(sbase + SM::kKr, kChunk, kk), bhi, id, kk > 0);
-                tc::mma_f16(tmem + kTmP, qhi, bhi, id, kk > 0);
-                tc::mma_f16(tmem + kTmP, qhi, blo, id, true);
-                tc::mma_f16(tmem + kTmP, desc_kmajor(sbase + SM::kQrLo, kChunk, kk), bhi, id, true);
-            }
-            tc::mma_commit(&bar_mma);
-        }
-        if (!wait_mma(&bar_mma, phase, &abort_flag)) break;
-
-        // ================= phase S: masks, UT transform =================
-        {
-            const bool owner = lane < 16;
-            const int r = warp * 16 + lane;
-            float a16[16], p16[16];
-#pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
-                tc::tmem_ld16(tmem + tl + kTmA + c16 * 16, a16);
-                tc::tmem_ld16(tmem + tl + kTmP + c16 * 16, p16);
-                tc::tmem_ld_wait();
-                if (owner) {
-                    const float br = sBeta[r];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int s = c16 * 16 + i;
-                        sA[r * kChunk + s] = (s < r) ? br * a16[i] : 0.f;
-                        p16[i] = (s <= r) ? p16[i] : 0.f;
+                    for (int i = 0; i < 8; ++i) {
+                        const float dg = G[rr][i] - gref[i];
+                        const float e1 = fast_exp(dg), e2 = fast_exp(-dg);
+                        kr[i] = kf[i] * e1;
+                        qr[i] = qf[i] * e1;
+                        kn[i] = kf[i] * e2;
+                        kg[i] = kr[i] * erefabs[i];
+                        qg[i] = qr[i] * erefabs[i];
+                        kd[i] = kn[i] * elast[i];
                     }
-                    *reinterpret_cast<uint4 *>(sm + SM::kP + tile_chunk(r, 2 * c16, kChunk, kChunk)) = pack8_h(p16);
-                    *reinterpret_cast<uint4 *>(sm + SM::kP + tile_chunk(r, 2 * c16 + 1, kChunk, kChunk)) =
-                        pack8_h(p16 + 8);
+                    const uint32_t off = tile_chunk(r, cg, kChunk, kDK);
+                    uint4 hi, lo;
+                    *reinterpret_cast<uint4 *>(sm + SM::kKr + off) = pack8_bf16(kr);
+                    split8_bf16(qr, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + SM::kQrHi + off) = hi;
+                    *reinterpret_cast<uint4 *>(sm + SM::kQrLo + off) = lo;
+                    split8_bf16(kn, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + SM::kKnHi + off) = hi;
+                    *reinterpret_cast<uint4 *>(sm + SM::kKnLo + off) = lo;
+                    *reinterpret_cast<uint4 *>(sm + SM::kKg + off) = pack8_h(kg);
+                    *reinterpret_cast<uint4 *>(sm + sQg + off) = pack8_h(qg);
+                    *reinterpret_cast<uint4 *>(sm + sKd + off) = pack8_h(kd);
                 }
             }
-            for (int i = tid; i < kChunk * kChunk; i += 128) sT[i] = 0.f;
-        }
-        tc::tc_fence_before();
-        __syncthreads();
-        // diagonal 16x16 blocks: thread (b, cc) computes column cc of (I + A_bb)^{-1}
-        if (tid < 64) {
-            const int b = tid >> 4, cc = tid & 15;
-            float x[16];
+            // the raw registers are consumed: fetch the next chunk while this one computes
+            if (c + 1 < nchunks) load_raw(c + 1);
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::named_sync(kBarPrep, kPrepThreads);
+
+            // ---- M1: A_raw = Kr Kn^T (committed first: the UT transform needs it),
+            //          P_raw = Qr Kn^T (two-term split, completes during the transform) ----
+            if (leader) {
+                tc::tc_fence_after();
+                constexpr uint32_t id = tc::make_idesc(64, 64, tc::kBF16, false, false);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
+                for (int kk = 0; kk < kDK / 16; ++kk)
+                    tc::mma_f16(tmem + kTmA, desc_kmajor(sbase + SM::kKr, kChunk, kk),
+                                desc_kmajor(sbase + SM::kKnHi, kChunk, kk), id, kk > 0);
+                tc::mma_commit(&bar_m1);
 #pragma unroll
-                for (int s = 0; s < 15; ++s)
-                    if (s < r && s >= cc) acc = fmaf(sA[(16 * b + r) * kChunk + 16 * b + s], x[s], acc);
-                x[r] = (r == cc) ? 1.f : ((r > cc) ? -acc : 0.f);
+                for (int kk = 0; kk < kDK / 16; ++kk) {
+                    const uint64_t bhi = desc_kmajor(sbase + SM::kKnHi, kChunk, kk);
+                    const uint64_t blo = desc_kmajor(sbase + SM::kKnLo, kChunk, kk);
+                    const uint64_t qhi = desc_kmajor(sbase + SM::kQrHi, kChunk, kk);
+                    tc::mma_f16(tmem + kTmP, qhi, bhi, id, kk > 0);
+                    tc::mma_f16(tmem + kTmP, qhi, blo, id, true);
+                    tc::mma_f16(tmem + kTmP, desc_kmajor(sbase + SM::kQrLo, kChunk, kk), bhi, id, true);
+                }
+                tc::mma_commit(&bar_m1p);
             }
+            if (!role_wait(&bar_m1, ph_m1, leader, kBarPrep, kPrepThreads, &abort_flag)) break;
+            ph_m1 ^= 1u;
+
+            // ---- A (fp32, beta-scaled, strict lower) from TMEM: warps 4-7 ----
+            constexpr int ld = SM::kLd;
+            if (warp < 8) {
+                const int r = (warp & 3) * 16 + lane;
+                const float br = (lane < 16) ? sBeta[r] : 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[(16 * b + r) * kChunk + 16 * b + cc] = x[r];
-        }
-        __syncthreads();
-        // off-diagonal row blocks: T[i, 0:16i] = -D_i (A[i, 0:16i] T[0:16i, 0:16i])
-        for (int ib = 1; ib < 4; ++ib) {
-            const int w = 16 * ib;
-            for (int e = tid; e < 16 * w; e += 128) {
-                const int r = e / w, cc = e % w;
-                float acc = 0.f;
-                for (int m = cc; m < w; ++m) acc = fmaf(sA[(w + r) * kChunk + m], sT[m * kChunk + cc], acc);
-                sX[r * 48 + cc] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < 16 * w; e += 128) {
-                const int r = e / w, cc = e % w;
-                float acc = 0.f;
-                for (int m = 0; m <= r; ++m) acc = fmaf(sT[(w + r) * kChunk + w + m], sX[m * 48 + cc], acc);
-                sT[(w + r) * kChunk + cc] = -acc;
-            }
-            __syncthreads();
-        }
-        // T diag(beta) -> fp16 A operand [64 x 64]
-        {
-            const int r = tid >> 1, half = tid & 1;
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float x16[16];
+                    tc::tmem_ld16(tmem + tl + kTmA + c16 * 16, x16);
+                    tc::tmem_ld_wait();
+                    if (lane < 16) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<float4 *>(&sA[r * ld + c16 * 16 + i]) =
+                                make_float4((c16 * 16 + i < r) ? br * x16[i] : 0.f,
+                                            (c16 * 16 + i + 1 < r) ? br * x16[i + 1] : 0.f,
+                                            (c16 * 16 + i + 2 < r) ? br * x16[i + 2] : 0.f,
+                                            (c16 * 16 + i + 3 < r) ? br * x16[i + 3] : 0.f);
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            tc::named_sync(kBarPrep, kPrepThreads);
+
+            // ---- UT transform T = (I + A)^{-1} ----
+            // (a) 16x16 diagonal blocks: thread (bb, cc) solves column cc of (I + A_bb) x = e_cc by
+            //     forward substitution; the zeros above the diagonal are written too.
+            if (tp < 64) {
+                const int bb = tp >> 4, cc = tp & 15;
+                const float *arow = sA + (16 * bb) * ld + 16 * bb;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int s2 = 0; s2 < 15; ++s2)
+                        if (s2 < r) {
+                            const float term = arow[r * ld + s2] * ((s2 >= cc) ? x[s2] : 0.f);
+                            if (s2 & 1) acc1 += term; else acc0 += term;
+                        }
+                    x[r] = (r == cc) ? 1.f : ((r > cc) ? -(acc0 + acc1) : 0.f);
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) sT[(16 * bb + r) * ld + 16 * bb + cc] = x[r];
+            }
+            tc::named_sync(kBarPrep, kPrepThreads);
+            // (b) off-diagonal blocks by distance d = i - j: T_ij = -T_ii sum_{j<=m<i} A_im T_mj.
+            //     The 4 - d blocks of one distance are independent; 256 threads = one 16x16 block.
+#pragma unroll
+            for (int d = 1; d < 4; ++d) {
+                const int r = tp >> 4, cc = tp & 15;
+#pragma unroll
+                for (int blk = 0; blk < 4 - d; ++blk) {
+                    const int j = blk, i = blk + d;
+                    const float *arow = sA + (16 * i + r) * ld + 16 * j;
+                    const float *tcol = sT + (16 * j) * ld + 16 * j + cc;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 16 * d; m += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
+                        acc[0] = fmaf(a4.x, tcol[(m + 0) * ld], acc[0]);
+                        acc[1] = fmaf(a4.y, tcol[(m + 1) * ld], acc[1]);
+                        acc[2] = fmaf(a4.z, tcol[(m + 2) * ld], acc[2]);
+                        acc[3] = fmaf(a4.w, tcol[(m + 3) * ld], acc[3]);
+                    }
+                    sX[blk * 256 + r * 16 + cc] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                }
+                tc::named_sync(kBarPrep, kPrepThreads);
+#pragma unroll
+                for (int blk = 0; blk < 4 - d; ++blk) {
+                    const int j = blk, i = blk + d;
+                    const float *drow = sT + (16 * i + r) * ld + 16 * i;  // row r of T_ii (zero above the diagonal)
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 16; m += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
+                        acc[0] = fmaf(t4.x, sX[blk * 256 + (m + 0) * 16 + cc], acc[0]);
+                        acc[1] = fmaf(t4.y, sX[blk * 256 + (m + 1) * 16 + cc], acc[1]);
+                        acc[2] = fmaf(t4.z, sX[blk * 256 + (m + 2) * 16 + cc], acc[2]);
+                        acc[3] = fmaf(t4.w, sX[blk * 256 + (m + 3) * 16 + cc], acc[3]);
+                    }
+                    sT[(16 * i + r) * ld + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                }
+                tc::named_sync(kBarPrep, kPrepThreads);
+            }
+            // T diag(beta) -> fp16 A operand [64 x 64]: 2 chunks of 8 per thread; the strictly
+            // upper blocks are never written, so the mask j*8 + i <= r is applied here
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int idx = tp * 2 + e, r = idx >> 3, j = idx & 7;
                 float f[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s = half * 32 + j * 8 + i;
-                    f[i] = sT[r * kChunk + s] * sBeta[s];
-                }
-                *reinterpret_cast<uint4 *>(sm + SM::kT + tile_chunk(r, half * 4 + j, kChunk, kChunk)) = pack8_h(f);
+                for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? sT[r * ld + j * 8 + i] * sBeta[j * 8 + i] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + SM::kTb + tile_chunk(r, j, kChunk, kChunk)) = pack8_h(f);
             }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ================= M2: W = (T b) Kg,  U = (T b) V =================
-        if (tid == 0) {
-            tc::tc_fence_after();
-            constexpr uint32_t idW = tc::make_idesc(64, kDK, tc::kF16, false, true);
-            constexpr uint32_t idU = tc::make_idesc(64, NV, tc::kF16, false, true);
+            // ---- P: wait for its MMAs and for the chain to release P and W (chunk c-1) ----
+            if (!role_wait(&bar_m1p, ph_m1p, leader, kBarPrep, kPrepThreads, &abort_flag)) break;
+            ph_m1p ^= 1u;
+            if (c >= 1 &&
+                !role_wait(&done[(c - 1) & 1], ((c - 1) >> 1) & 1, leader, kBarPrep, kPrepThreads, &abort_flag))
+                break;
+            if (warp >= 8) {
+                const int r = (warp & 3) * 16 + lane;
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk) {
-                const uint64_t adesc = desc_kmajor(sbase + SM::kT, kChunk, kk);
-                tc::mma_f16(tmem + kTmW, adesc, desc_mnmajor(sbase + SM::kKg, kChunk, kDK, kk), idW, kk > 0);
-                tc::mma_f16(tmem + kTmU, adesc, desc_mnmajor(sbase + SM::kV, kChunk, NV, kk), idU, kk > 0);
-            }
-            tc::mma_commit(&bar_mma);
-        }
-        if (!wait_mma(&bar_mma, phase, &abort_flag)) break;
-
-        // W -> fp16 A operand [64 x 128]
-        {
-            const bool owner = lane < 16;
-            const int r = warp * 16 + lane;
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float x16[16];
+                    tc::tmem_ld16(tmem + tl + kTmP + c16 * 16, x16);
+                    tc::tmem_ld_wait();
+                    if (lane < 16) {
 #pragma unroll
-            for (int c16 = 0; c16 < kDK / 16; ++c16) {
-                float w16[16];
-                tc::tmem_ld16(tmem + tl + kTmW + c16 * 16, w16);
-                tc::tmem_ld_wait();
-                if (owner) {
-                    *reinterpret_cast<uint4 *>(sm + SM::kW + tile_chunk(r, 2 * c16, kChunk, kDK)) = pack8_h(w16);
-                    *reinterpret_cast<uint4 *>(sm + SM::kW + tile_chunk(r, 2 * c16 + 1, kChunk, kDK)) =
-                        pack8_h(w16 + 8);
-                }
-            }
-        }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ================= M3: U~ = U - W S (into U),  O = Qg S =================
-        if (tid == 0) {
-            tc::tc_fence_after();
-            constexpr uint32_t idNeg = tc::make_idesc(64, NV, tc::kF16, false, true, true);
-            constexpr uint32_t idO = tc::make_idesc(64, NV, tc::kF16, false, true);
-#pragma unroll
-            for (int kk = 0; kk < kDK / 16; ++kk) {
-                const uint64_t bdesc = desc_mnmajor(sbase + SM::kS, kDK, NV, kk);
-                tc::mma_f16(tmem + kTmU, desc_kmajor(sbase + SM::kW, kChunk, kk), bdesc, idNeg, true);
-                tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + SM::kQg, kChunk, kk), bdesc, idO, kk > 0);
-            }
-            tc::mma_commit(&bar_mma);
-        }
-        if (!wait_mma(&bar_mma, phase, &abort_flag)) break;
-
-        // U~ -> fp16 MN-major B operand [64 x NV]; a value outside the fp16
-        // range sends the chunk to the exact path
-        {
-            const bool owner = lane < 16;
-            const int r = warp * 16 + lane;
-            bool bad = false;
-#pragma unroll
-            for (int c16 = 0; c16 < NV / 16; ++c16) {
-                float u16[16];
-                tc::tmem_ld16(tmem + tl + kTmU + c16 * 16, u16);
-                tc::tmem_ld_wait();
-                if (owner) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) bad |= !(fabsf(u16[i]) <= 65000.f);
-                    *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16, kChunk, NV)) = pack8_h(u16);
-                    *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16 + 1, kChunk, NV)) =
-                        pack8_h(u16 + 8);
+                        for (int i = 0; i < 16; ++i) x16[i] = (c16 * 16 + i <= r) ? x16[i] : 0.f;
+                        *reinterpret_cast<uint4 *>(sm + SM::kP + tile_chunk(r, 2 * c16, kChunk, kChunk)) =
+                            pack8_h(x16);
+                        *reinterpret_cast<uint4 *>(sm + SM::kP + tile_chunk(r, 2 * c16 + 1, kChunk, kChunk)) =
+                            pack8_h(x16 + 8);
+                    }
                 }
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            if (__syncthreads_or(bad)) {
-                exact_chunk(tok0, L);
-                continue;
-            }
-        }
+            tc::named_sync(kBarPrep, kPrepThreads);
 
-        // ================= M4: O += P U~,  Sn = Kd^T U~ =================
-        if (tid == 0) {
-            tc::tc_fence_after();
-            constexpr uint32_t idO = tc::make_idesc(64, NV, tc::kF16, false, true);
-            constexpr uint32_t idS = tc::make_idesc(128, NV, tc::kF16, true, true);
+            // ---- M2: W = (T b) Kg,  U[b] = (T b) V ----
+            if (leader) {
+                tc::tc_fence_after();
+                constexpr uint32_t idW = tc::make_idesc(64, kDK, tc::kF16, false, true);
+                constexpr uint32_t idU = tc::make_idesc(64, kNV, tc::kF16, false, true);
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk) {
-                const uint64_t bdesc = desc_mnmajor(sbase + SM::kUt, kChunk, NV, kk);
-                tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + SM::kP, kChunk, kk), bdesc, idO, true);
-                tc::mma_f16(tmem + kTmSn, desc_mnmajor(sbase + SM::kKd, kChunk, kDK, kk), bdesc, idS, kk > 0);
+                for (int kk = 0; kk < kChunk / 16; ++kk) {
+                    const uint64_t adesc = desc_kmajor(sbase + SM::kTb, kChunk, kk);
+                    tc::mma_f16(tmem + kTmW, adesc, desc_mnmajor(sbase + SM::kKg, kChunk, kDK, kk), idW, kk > 0);
+                    tc::mma_f16(tmem + kTmU0 + b * kNV, adesc, desc_mnmajor(sbase + SM::kV, kChunk, kNV, kk), idU,
+                                kk > 0);
+                }
+                tc::mma_commit(&bar_m2);
             }
-            tc::mma_commit(&bar_mma);
-        }
-        if (!wait_mma(&bar_mma, phase, &abort_flag)) break;
+            if (!role_wait(&bar_m2, ph_m2, leader, kBarPrep, kPrepThreads, &abort_flag)) break;
+            ph_m2 ^= 1u;
 
-        // ================= epilogue: output rows, state update =================
-        {
-            const bool owner = lane < 16;
-            const int r = warp * 16 + lane;
-            float o[NV];
-            bool bad = false;
+            // ---- W -> fp16 A operand [64 x 128]; gamma; hand the slot to the chain ----
+            {
+                const int w4 = warp - 4;
+                const int half = w4 >> 2;            // columns [64 half, 64 half + 64)
+                const int r = (warp & 3) * 16 + lane;
 #pragma unroll
-            for (int c16 = 0; c16 < NV / 16; ++c16) {
-                float o16[16];
-                tc::tmem_ld16(tmem + tl + kTmO + c16 * 16, o16);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[c16 * 16 + i] = o16[i];
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float w16[16];
+                    tc::tmem_ld16(tmem + tl + kTmW + half * 64 + c16 * 16, w16);
+                    tc::tmem_ld_wait();
+                    if (lane < 16) {
+                        const int j = half * 8 + 2 * c16;
+                        *reinterpret_cast<uint4 *>(sm + SM::kW + tile_chunk(r, j, kChunk, kDK)) = pack8_h(w16);
+                        *reinterpret_cast<uint4 *>(sm + SM::kW + tile_chunk(r, j + 1, kChunk, kDK)) =
+                            pack8_h(w16 + 8);
+                    }
+                }
             }
-            if (owner)
-#pragma unroll
-                for (int i = 0; i < NV; ++i) bad |= !(fabsf(o[i]) <= 3.0e38f);
+            if (tp < kDK) sGamma[b * kDK + tp] = fast_exp(sGlast[tp]);
+            if (leader) sFlags[b] = 0;
+            tc::fence_async_smem();
             tc::tc_fence_before();
-            if (__syncthreads_or(bad)) {
-                exact_chunk(tok0, L);
-                continue;
-            }
-            if (owner && r < L) {
-                TO *dst = out + ((tok0 + r) * H + h) * DV + vcol0;
-#pragma unroll
-                for (int c16 = 0; c16 < NV / 16; ++c16) store16<TO>(dst + c16 * 16, &o[c16 * 16]);
-            }
-            const float gam = expf(sGlast[tid]);
-#pragma unroll
-            for (int c16 = 0; c16 < NV / 16; ++c16) {
-                float s16[16];
-                tc::tmem_ld16(tmem + tl + kTmSn + c16 * 16, s16);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) S[c16 * 16 + i] = fmaf(gam, S[c16 * 16 + i], s16[i]);
-            }
-            write_state_operand();
+            tc::named_sync(kBarPrep, kPrepThreads);
+            if (leader) tc::mbar_arrive(&full[b]);
         }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
     }
 
-    if (final_state && abort_flag == 0) {
-#pragma unroll
-        for (int j = 0; j < NV; ++j) final_state[state_base + (size_t)tid * DV + vcol0 + j] = S[j];
-    }
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmCols);
 }
 
-template <int NV, typename TO>
-cudaError_t launch_chunk_tc_nv(const void *q, const void *k, const void *v, const void *la, const void *beta,
-                               const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
-                               void *out, float *final_state, cudaStream_t stream) {
-    auto kern = kda_chunk_tc_kernel<NV, TO>;
-    const int smem = ChunkSmem<NV>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    const int N = cu ? num_seqs : B;
-    const unsigned grid = static_cast<unsigned>(N) * H * (DV / NV);
-    kern<<<grid, 128, smem, stream>>>(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                                      static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(la),
-                                      static_cast<const __nv_bfloat16 *>(beta), init_state, cu, num_seqs, T, H, DV,
-                                      static_cast<TO *>(out), final_state);
-    return cudaGetLastError();
-}
-
-// Slice width: narrow slices when there are few (sequence, head) pairs, so the
-// grid still covers the SMs.
 template <typename TO>
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *la, const void *beta,
                             const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
                             void *out, float *final_state, cudaStream_t stream) {
-    const int64_t pairs = (int64_t)(cu ? num_seqs : B) * H;
-    if (pairs * (DV / 64) < 148)
-        return launch_chunk_tc_nv<32, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, DV, out, final_state,
-                                          stream);
-    return launch_chunk_tc_nv<64, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, DV, out, final_state,
-                                      stream);
+    auto kern = kda_chunk_tc_kernel<TO>;
+    const int smem = ChunkSmem::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int N = cu ? num_seqs : B;
+    const unsigned grid = static_cast<unsigned>(N) * H * (DV / kNV);
+    kern<<<grid, kThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                                           static_cast<const __nv_bfloat16 *>(v),
+                                           static_cast<const __nv_bfloat16 *>(la),
+                                           static_cast<const __nv_bfloat16 *>(beta), init_state, cu, num_seqs, T, H,
+                                           DV, static_cast<TO *>(out), final_state);
+    return cudaGetLastError();
 }
 
 }  // namespace kda

@@ -36,6 +36,12 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // log2(e), used to turn exp(x) into exp2(x * log2e) for the ex2 unit.
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ float fast_exp(float x) { return exp2f(x * kLog2e); }
+// 2^x on the SFU (ex2.approx: relative error ~2^-22, flushes subnormal results).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_exp(float x) { return ex2_approx(x * kLog2e); }
 
 }  // namespace kda
