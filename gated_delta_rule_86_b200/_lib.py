@@ -11,8 +11,8 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT 
 KDA_F32, KDA_BF16 = 0, 1
 
 # every symbol include/kda.h declares
-EXPORTED = ("kda_chunk_fwd", "kda_recurrent_fwd", "kda_decode_step", "kda_status_string",
-            "kda_get_last_device_error", "kda_version")
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_recurrent_fwd", "kda_decode_step",
+            "kda_status_string", "kda_get_last_device_error", "kda_version")
 
 _lib = None
 
@@ -37,8 +37,10 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, f32p = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     prefill_args = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, i32, i32]
-    lib.kda_chunk_fwd.argtypes = prefill_args + [i32, ctypes.c_int, ctypes.c_int, vp, f32p, vp]
+    lib.kda_chunk_fwd.argtypes = prefill_args + [i32, ctypes.c_int, ctypes.c_int, vp, f32p, vp, ctypes.c_size_t, vp]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_int
     lib.kda_recurrent_fwd.argtypes = prefill_args + [ctypes.c_int, ctypes.c_int, vp, f32p, vp]
     lib.kda_recurrent_fwd.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,

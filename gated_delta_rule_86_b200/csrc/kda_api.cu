@@ -115,10 +115,21 @@ kda_status kda_recurrent_fwd(const void *q, const void *k, const void *v, const 
                                         B, T, H, d_k, d_v, out, final_state, st));
 }
 
+kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                                        size_t *bytes) {
+    if (!bytes || N < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if (dtype == KDA_BF16) *bytes = kda::chunk_tc_workspace_bytes((int64_t)N * H, d_v);
+    return KDA_OK;
+}
+
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
                          const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                          int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
-                         kda_dtype out_dtype, void *out, float *final_state, void *stream) {
+                         kda_dtype out_dtype, void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                         void *stream) {
     kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
                                  dtype, out_dtype, out, final_state);
     if (s != KDA_OK) return s;
@@ -132,11 +143,13 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                                             num_seqs, B, T, H, d_k, d_v, out, final_state, st));
     }
     if (d_k != 128) return KDA_ERR_UNSUPPORTED;
+    const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
     if (out_dtype == KDA_F32)
         return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
-                                                     T, H, d_v, out, final_state, st));
+                                                     T, H, d_v, out, final_state, workspace, st));
     return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                                         B, T, H, d_v, out, final_state, st));
+                                                         B, T, H, d_v, out, final_state, workspace, st));
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,

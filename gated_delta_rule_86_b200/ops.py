@@ -90,8 +90,12 @@ def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, outpu
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(s0), _ptr(cu),
             ctypes.c_int32(N if cu is not None else 0), B, T, H, dk, dv]
     if fn_name == "kda_chunk_fwd":
-        status = lib.kda_chunk_fwd(*args, ctypes.c_int32(chunk_size), dt, odt, _ptr(out), _ptr(fs),
-                                   _stream_handle())
+        ws_bytes = ctypes.c_size_t(0)
+        _lib.check(lib.kda_chunk_fwd_workspace_size(N, H, dk, dv, dt, ctypes.byref(ws_bytes)),
+                   "kda_chunk_fwd_workspace_size")
+        ws = torch.empty(ws_bytes.value, dtype=torch.uint8, device=q.device) if ws_bytes.value else None
+        status = lib.kda_chunk_fwd(*args, ctypes.c_int32(chunk_size), dt, odt, _ptr(out), _ptr(fs), _ptr(ws),
+                                   ctypes.c_size_t(ws_bytes.value), _stream_handle())
     else:
         status = lib.kda_recurrent_fwd(*args, dt, odt, _ptr(out), _ptr(fs), _stream_handle())
     _lib.check(status, fn_name)

@@ -35,6 +35,7 @@
 #ifndef KDA_B200_KDA_H
 #define KDA_B200_KDA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -84,6 +85,11 @@ typedef enum {
  *   final_state     : [N, H, d_k, d_v] fp32, or NULL to skip.  It may alias
  *                     init_state exactly (in-place state update); partial
  *                     overlap is invalid.
+ *   workspace       : device scratch of at least the size that
+ *                     kda_chunk_fwd_workspace_size reports (16-byte aligned);
+ *                     may be NULL when that size is 0.  Owned by the caller,
+ *                     used only during the call; calls that overlap on the
+ *                     GPU must not share one workspace.
  * Supported: d_k == 128 and d_v in {64, 128} for bf16 (tensor-core path);
  * d_k, d_v in {64, 128} for fp32 (fp32 CUDA-core path, fp32 accuracy).
  * T == 0 is valid (final_state = init_state or zeros).
@@ -92,7 +98,18 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                          const void *beta, const float *init_state, const int32_t *cu_seqlens,
                          int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k,
                          int32_t d_v, int32_t chunk, kda_dtype dtype, kda_dtype out_dtype,
-                         void *out, float *final_state, void *stream);
+                         void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * Workspace kda_chunk_fwd needs, in bytes, for N sequences (B, or num_seqs with
+ * cu_seqlens) of H heads: on the tensor-core path, one 65 KB chunk image per
+ * (sequence, head, 32-column value slice), through which the CTAs of one head
+ * hand each other the per-chunk operands (see kda_chunk_fwd); 0 on the fp32
+ * path.  Pure host computation, never fails for valid sizes.
+ */
+kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                                        kda_dtype dtype, size_t *bytes);
 
 /*
  * kda_recurrent_fwd -- the same operation as kda_chunk_fwd, evaluated token by

@@ -44,9 +44,9 @@ ODD = ctypes.c_void_p((1 << 20) + 8)   # 8-byte aligned only
 
 
 def chunk(lib, q=FAKE, B=1, T=128, H=2, dk=128, dv=128, chunk_size=64, dtype=_lib.KDA_BF16, cu=None, ns=0,
-          s0=None, fs=None, out=FAKE, odt=_lib.KDA_F32):
+          s0=None, fs=None, out=FAKE, odt=_lib.KDA_F32, ws=FAKE, ws_bytes=1 << 30):
     return lib.kda_chunk_fwd(q, FAKE, FAKE, FAKE, FAKE, s0, cu, ns, B, T, H, dk, dv, chunk_size, dtype, odt, out,
-                             fs, None)
+                             fs, ws, ws_bytes, None)
 
 
 def test_rejects_bad_arguments(lib):
@@ -67,6 +67,8 @@ def test_rejects_bad_arguments(lib):
     assert chunk(lib, dv=256) == U
     assert chunk(lib, chunk_size=128) == U
     assert chunk(lib, dk=64, dtype=_lib.KDA_BF16) == U   # tensor-core path needs d_k = 128
+    assert chunk(lib, ws=None) == E                      # tensor-core path needs its workspace
+    assert chunk(lib, ws_bytes=1024) == E
     rec = lib.kda_recurrent_fwd(FAKE, FAKE, FAKE, FAKE, None, None, None, 0, 1, 8, 1, 64, 64, _lib.KDA_F32,
                                 _lib.KDA_F32, FAKE, None, None)
     assert rec == E
@@ -75,6 +77,19 @@ def test_rejects_bad_arguments(lib):
     assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
     assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 32, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == U
     assert dec(ODD, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+
+
+def test_workspace_size(lib):
+    n = ctypes.c_size_t(7)
+    assert lib.kda_chunk_fwd_workspace_size(2, 16, 128, 128, _lib.KDA_BF16, ctypes.byref(n)) == _lib.KDA_OK
+    per = n.value // (2 * 16 * 4)
+    assert per * 2 * 16 * 4 == n.value and per >= 64 * 1024      # one chunk image per (seq, head, slice)
+    assert lib.kda_chunk_fwd_workspace_size(2, 16, 128, 64, _lib.KDA_BF16, ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == per * 2 * 16 * 2
+    assert lib.kda_chunk_fwd_workspace_size(2, 16, 64, 64, _lib.KDA_F32, ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == 0
+    assert lib.kda_chunk_fwd_workspace_size(0, 16, 128, 128, _lib.KDA_BF16, ctypes.byref(n)) == \
+        _lib.KDA_ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch):
