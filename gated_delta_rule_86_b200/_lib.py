@@ -11,8 +11,8 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT 
 KDA_F32, KDA_BF16 = 0, 1
 
 # every symbol include/kda.h declares
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_recurrent_fwd", "kda_decode_step",
-            "kda_status_string", "kda_get_last_device_error", "kda_version")
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_static_ws", "kda_recurrent_fwd",
+            "kda_decode_step", "kda_status_string", "kda_get_last_device_error", "kda_version")
 
 _lib = None
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/kda.h"
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
@@ -75,6 +77,31 @@ cudaError_t dispatch_recurrent(kda_dtype dt, kda_dtype odt, const void *q, const
                                                           st);
     return dispatch_recurrent_t<__nv_bfloat16, __nv_bfloat16>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
                                                               fs, st);
+}
+
+// Handoff buffer of kda_chunk_fwd_static_ws: a fixed array in device memory,
+// one copy per GPU that loads the library.  In host code `g_static_ws` only
+// names the symbol; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_static_ws[KDA_STATIC_WS_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void *g_static_ws_addr[kMaxDevices] = {};
+
+// Device address of the current device's copy of g_static_ws, looked up once
+// per device (with that device current) and cached.
+kda_status static_ws_address(void **addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return KDA_ERR_CUDA;
+        g_static_ws_addr[dev] = p;
+    }
+    *addr = g_static_ws_addr[dev];
+    return KDA_OK;
 }
 
 }  // namespace
@@ -150,6 +177,29 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                                                      T, H, d_v, out, final_state, workspace, st));
     return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
                                                          B, T, H, d_v, out, final_state, workspace, st));
+}
+
+kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, const void *log_alpha,
+                                   const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                                   int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                   int32_t chunk, kda_dtype dtype, kda_dtype out_dtype, void *out,
+                                   float *final_state, void *stream) {
+    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
+                                 dtype, out_dtype, out, final_state);
+    if (s != KDA_OK) return s;
+    if (chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64 || dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
+    const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
+    if (need > KDA_STATIC_WS_BYTES) return KDA_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    s = static_ws_address(&ws);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (out_dtype == KDA_F32)
+        return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
+                                                     T, H, d_v, out, final_state, ws, st));
+    return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                                                         B, T, H, d_v, out, final_state, ws, st));
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,

@@ -139,6 +139,42 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
                            int32_t d_k, int32_t d_v, kda_dtype dtype, kda_dtype out_dtype,
                            void *stream);
 
+/*
+ * kda_chunk_fwd_static_ws -- kda_chunk_fwd for callers that cannot allocate
+ * device memory when they call it.  Examples: an inference engine that has
+ * reserved all device memory up front in its own pool and forbids further
+ * allocations, or code running inside an allocation callback, where calling
+ * back into the allocator is not allowed.  Such a caller has no way to
+ * provide the workspace argument of kda_chunk_fwd.  This call instead takes
+ * the chunk-image handoff buffer from a fixed array built into the library
+ * (KDA_STATIC_WS_BYTES per GPU; every GPU that loads the library holds it
+ * until the process exits).  The pages describe nothing like it; it exists
+ * only for such callers.
+ *
+ * Same arguments, layouts and results as kda_chunk_fwd, without workspace /
+ * workspace_bytes.  Only the tensor-core path: dtype KDA_BF16, d_k == 128,
+ * d_v in {64, 128}.  It allocates nothing (no cudaMalloc, no library
+ * allocator).  KDA_ERR_UNSUPPORTED if the problem needs more than
+ * KDA_STATIC_WS_BYTES of handoff buffer, i.e. more than
+ * KDA_STATIC_WS_BYTES / (65 KB * d_v / 32) (sequence, head) pairs: 63 at
+ * d_v = 128, 126 at d_v = 64.
+ *
+ * The first call on a device looks up that device's copy of the array (with
+ * the device current), so make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its last contents
+ * there; nothing in it needs to start at zero, since each chunk image is
+ * written before it is read.  Two calls that run on the same GPU at the same
+ * time (different streams, or graph replays in flight together) use the same
+ * array and race: serialise them.
+ */
+#define KDA_STATIC_WS_BYTES (16u << 20)
+kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, const void *log_alpha,
+                                   const void *beta, const float *init_state,
+                                   const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                                   int32_t T, int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
+                                   kda_dtype dtype, kda_dtype out_dtype, void *out,
+                                   float *final_state, void *stream);
+
 /* Human-readable name of a status (static string, never NULL). */
 const char *kda_status_string(kda_status s);
 
