@@ -170,6 +170,7 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                                             num_seqs, B, T, H, d_k, d_v, out, final_state, st));
     }
     if (d_k != 128) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
     const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
     if (out_dtype == KDA_F32)
@@ -189,6 +190,7 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
     if (s != KDA_OK) return s;
     if (chunk < 1) return KDA_ERR_INVALID_ARG;
     if (chunk != 64 || dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
     const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
     if (need > KDA_STATIC_WS_BYTES) return KDA_ERR_UNSUPPORTED;
     void *ws = nullptr;

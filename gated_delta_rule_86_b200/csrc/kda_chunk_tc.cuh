@@ -16,32 +16,33 @@
 //   S    <- Diag(exp(G_last)) S + (K * exp(G_last - G))^T U~
 // which equals the token recurrence exactly in exact arithmetic.
 //
-// Pipeline.  Everything up to W and U depends only on the chunk's own inputs;
-// only the last three lines touch S.  One cluster of CL = d_v / 32 CTAs handles
-// one (sequence, head); CTA r owns value columns [32 r, 32 r + 32) and runs
-// three roles:
-//   * prep (warps 4-11): for every CL-th chunk (c = r mod CL): decays, rebased
-//     operands, A/P, UT transform and W.  The finished operands of the chunk
-//     (Kd, P, Qg, W, T diag(beta), gamma and a flag) form one contiguous image,
-//     which is bulk-stored to a per-producer region of a global workspace and
-//     announced to every CTA of the cluster through remote mbarrier arrives;
-//   * chain (warps 0-3): for every chunk, bulk-loads the image (in two parts,
-//     so the next chunk's loads overlap this chunk's MMAs), computes U on its
-//     own value slice, then the state-dependent MMAs, output rows and the fp32
-//     state update, and tells the producer when the region may be reused.
-// The prep of a chunk is thus computed once per head instead of once per
-// slice, and each CTA spends only 1/CL of its time on it.
-
+// Work split.  Only U~ and the state update sit on the sequential chain; every
+// other quantity depends on the chunk's own inputs alone.  One cluster of
+// 1 + kNP CTAs handles one (sequence, head):
+//   * prep CTAs (ranks 1..kNP): CTA 1 + p prepares chunks c = p mod kNP: decays,
+//     rebased operands, A and P, the UT transform, then W and U on the tensor
+//     cores.  The finished chunk image (-W, U, Qg = Q exp(G), Kd = K exp(G_last - G),
+//     P, gamma = exp(G_last) and a flag) is bulk-stored to this producer's region
+//     of a global workspace (it stays in L2) and announced to the chain CTA
+//     through a remote mbarrier arrive;
+//   * the chain CTA (rank 0) bulk-loads each image into a two-deep shared-memory
+//     ring and runs, per chunk, one MMA group [-W ; Qg] S (rows 0-63 give
+//     U~ - U, rows 64-127 give Qg S), the U~ epilogue, the MMAs Kd^T U~ and
+//     [. ; P] U~ (adding P U~ to rows 64-127) and the fp32 state update, while
+//     dedicated warps store the output rows.
+// The chain CTA computes all d_v columns of S at once: a tcgen05.mma costs about
+// the same for N = 32 and N = 128 value columns, so slicing d_v across CTAs would
+// multiply the tensor-core time of the chain without shortening it.
+//
 // Precision (fp32 accumulation in TMEM, fp32 master state in registers, fp32
 // decays and substitution, fp32 or bf16 output):
 //   * A and P need the rebased factors below, whose range exceeds fp16: they are
 //     bf16 operands, and P (which feeds the output directly) uses a two-term
 //     bf16 split of both operands (hi*hi + hi*lo + lo*hi), ~16-bit accuracy.
-//   * Every other product (W, U, U~, Q S, P U~, Kd^T U~) has operands bounded by
-//     the inputs and runs on fp16 operands (11-bit significand, same tensor
-//     rate as bf16).  If any of those values leaves the fp16 range, the chunk's
-//     U~ or O turns non-finite; that is detected and the chunk is recomputed on
-//     the exact path below.
+//   * Every other product has operands bounded by the inputs and runs on fp16
+//     operands (11-bit significand, same tensor rate as bf16).  A value outside
+//     the fp16 range turns U~ or O non-finite; that is detected and the chunk is
+//     recomputed on the exact path below.
 //
 // Exponent range ("log-domain accumulation", section 3 of "Designing and
 // Deploying Hybrid MLA and Linear Attention Architectures for LLMs"): the
@@ -50,16 +51,19 @@
 // stays within exp(+-kRangeLimit) whenever the chunk's per-channel decay on
 // either side of the middle stays within kRangeLimit.  A chunk whose decays
 // exceed that (extremely fast forgetting) is evaluated token by token in fp32
-// instead, so every input with finite log_alpha gets a correct result.
+// by the chain CTA instead, so every input with finite log_alpha gets a correct
+// result.
 //
-// Work decomposition: the d_v columns of S evolve independently (column j of U~
-// depends only on column j of S), so slicing d_v across the CTAs of a cluster
-// multiplies the parallelism of the sequential chunk chain.  Packed
-// variable-length batches are scheduled longest-first.
+// Packed variable-length batches are scheduled longest-first.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
 
 #include "kda_common.cuh"
 #include "kda_recurrent.cuh"
@@ -69,95 +73,112 @@ namespace kda {
 
 constexpr int kChunk = 64;
 constexpr int kDK = 128;
-constexpr int kNV = 32;  // value columns per CTA
 // Largest per-channel cumulative decay (in natural-log units) allowed on either
 // side of the chunk's middle token for the tensor-core path.  Factors of the
 // rebased products stay within exp(+-40); their sums stay far below the fp32
 // and bf16 overflow threshold exp(88.7).
 constexpr float kRangeLimit = 40.f;
 
-constexpr int kChainThreads = 128;  // warps 0-3
-constexpr int kPrepThreads = 256;   // warps 4-11
-constexpr int kThreads = kChainThreads + kPrepThreads;
-constexpr uint32_t kBarPrep = 1, kBarChain = 2;  // named barrier ids
+constexpr int kNP = 3;                // prep CTAs per cluster
+constexpr int kCL = kNP + 1;          // cluster: chain CTA (rank 0) + prep CTAs
+constexpr int kThreads = 384;         // 12 warps in every CTA of the cluster
+constexpr int kRoleThreads = 256;     // warps 0-7 run the role; warp 8 moves images
+constexpr uint32_t kBarRole = 1, kBarU = 2, kBarOut = 3;  // named barriers: warps 0-7, U~ warps, output warps
 
-// ---- chunk image: the prep results of one chunk, in their MMA layouts (fp16) -----------------
-// part 2 (consumed by the second chain MMA group) first, part 1 after it.
-struct ChunkImage {
-    static constexpr int kTile = kChunk * kDK * 2;      // [64 x 128] 16-bit tile
-    static constexpr int kKd = 0;                       // K exp(Glast - G)   A of Kd^T U~ (MN-major)
-    static constexpr int kP = kKd + kTile;              // tril(P) [64 x 64]  A of P U~
-    static constexpr int kPart1 = kP + kChunk * kChunk * 2;
-    static constexpr int kQg = kPart1;                  // Q exp(G)           A of Q S
-    static constexpr int kW = kQg + kTile;              // W [64 x 128]       A of -W S
-    static constexpr int kTb = kW + kTile;              // T diag(beta)       A of U
-    static constexpr int kGamma = kTb + kChunk * kChunk * 2;   // fp32 [128] exp(Glast)
-    static constexpr int kFlag = kGamma + kDK * 4;             // int: 1 = evaluate exactly
+// ---- chunk image in the global workspace (fp16 tiles in their shared-memory layouts) ----------
+template <int DV> struct Img {
+    static constexpr int kNW = 0;                          // -W  [64 x 128]
+    static constexpr int kUT = kNW + kChunk * kDK * 2;     // U^T [DV x 64]
+    static constexpr int kQt = kUT + kChunk * DV * 2;      // Qg  [64 x 128]
+    static constexpr int kKd = kQt + kChunk * kDK * 2;     // Kd  [64 x 128]
+    static constexpr int kP = kKd + kChunk * kDK * 2;      // tril(P) [64 x 64] (after Kd: [Kd ; P] rows)
+    static constexpr int kGam = kP + kChunk * kChunk * 2;  // fp32 [128] exp(G_last)
+    static constexpr int kFlag = kGam + kDK * 4;           // int: 1 = evaluate exactly
     static constexpr int kBytes = kFlag + 16;
-    static constexpr int kPart2Bytes = kPart1;
-    static constexpr int kPart1Bytes = kBytes - kPart1;
-    static constexpr int kStride = (kBytes + 1023) / 1024 * 1024;  // workspace region stride
+    static constexpr int kStride = (kBytes + 1023) / 1024 * 1024;
 };
 
-// ---- shared-memory plan (byte offsets; operand tiles 1024-aligned) -------------------------------
-struct ChunkSmem {
-    using I = ChunkImage;
-    static constexpr int kTile = I::kTile;
-    // prep region: the image of the chunk being prepared, and its scratch
-    static constexpr int kImg = 0;
-    // bf16 operands of A_raw and P_raw (dead once those MMAs complete); they
-    // overlap the image's W/Tb/gamma/flag, which are written later
-    static constexpr int kKr = I::kW;                 // K exp(G - Gref)            A of A_raw
-    static constexpr int kQrHi = kKr + kTile;         // Q exp(G - Gref), hi        A of P_raw
-    static constexpr int kQrLo = kQrHi + kTile;       //                  lo
-    static constexpr int kKnHi = kQrLo + kTile;       // K exp(Gref - G), hi        B of A_raw, P_raw
-    static constexpr int kKnLo = kKnHi + kTile;       //                  lo
-    static constexpr int kApEnd = kKnLo + kTile;
-    // fp32 scratch of the UT transform, inside the dead A/P operands and past the image
-    static constexpr int kLd = 68;                    // fp32 row stride of A and T (bank spread, 16-B rows)
-    static constexpr int kA32 = (I::kBytes + 1023) / 1024 * 1024 + 7168;
-    static constexpr int kT32 = kA32 + kChunk * kLd * 4;
-    static constexpr int kX32 = kT32 + kChunk * kLd * 4;      // fp32 [3][16][16] block products
-    static constexpr int kTot = kA32;                          // fp32 [8][128] scan totals (decay phase only)
-    static constexpr int kKg = kApEnd;                // K exp(G) [64 x 128]        B of W (MN-major)
-    static constexpr int kPrepEnd = kKg + kTile;
-    // chain region
-    static constexpr int kSlot = kPrepEnd;            // the chain's copy of the current chunk image
-    static constexpr int kV = kSlot + I::kStride;     // V slice [64 x 32] fp16   B of U
-    static constexpr int kS = kV + kChunk * kNV * 2;  // S [128 x 32] fp16        B of W S, Q S
-    static constexpr int kUt = kS + kDK * kNV * 2;    // U~ [64 x 32] fp16        B of P U~, Kd^T U~
-    // small fp32 arrays
-    static constexpr int kBeta = kUt + kChunk * kNV * 2;      // [64]  prep
-    static constexpr int kG0 = kBeta + kChunk * 4;            // [128] decay after token 0
-    static constexpr int kGref = kG0 + kDK * 4;               // [128] decay after token 31
-    static constexpr int kGlast = kGref + kDK * 4;            // [128] decay after token 63
-    static constexpr int kRed = kGlast + kDK * 4;             // chain exact path: 292 floats
-    static constexpr int kEnd = kRed + 300 * 4;
-    static constexpr int kBytes = kEnd + 1024;                // + alignment slack
-    static_assert(kX32 + 3 * 256 * 4 <= kApEnd, "UT scratch must fit the dead A/P operands");
-    static_assert(kTot + 8 * kDK * 4 <= kApEnd, "scan totals must fit the dead A/P operands");
-    static_assert(kBytes <= 232448, "shared memory plan exceeds 227 KB");
+// ---- chain CTA shared memory ------------------------------------------------------------------
+template <int DV> struct ChainSmem {
+    using I = Img<DV>;
+    // one slot of the image ring: A1 = [-W ; Qg] as two 16 KB k-blocks of 128 rows (rows 0-63 -W,
+    // rows 64-127 Qg; the B operand of S^T A1^T), then U^T, then Kd, P, gamma, flag in image order
+    static constexpr int kA1 = 0;
+    static constexpr int kUT = 2 * kChunk * kDK * 2;
+    static constexpr int kKd = kUT + kChunk * DV * 2;
+    static constexpr int kP = kKd + (I::kP - I::kKd);
+    static constexpr int kGam = kKd + (I::kGam - I::kKd);
+    static constexpr int kFlag = kKd + (I::kFlag - I::kKd);
+    static constexpr int kTailBytes = I::kBytes - I::kKd;
+    static constexpr int kSlotBytes = (kKd + kTailBytes + 1023) / 1024 * 1024;
+    // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel half, k . q
+    static constexpr int kRedPk = 2 * kSlotBytes;
+    static constexpr int kRedPq = kRedPk + 2 * 128 * 4;
+    static constexpr int kRedKq = kRedPq + 2 * 128 * 4;
+    // output staging of a full chunk: DV / 64 blocks of [64 tokens x 64 values] (fp32 or bf16),
+    // written by a TMA tensor store per block
+    static constexpr int kOut = (kRedKq + 16 + 1023) / 1024 * 1024;
+    static constexpr int kBytes = kOut + kChunk * DV * 4;
 };
 
-// TMEM columns (fp32 accumulators).  M=64 tiles use lanes 0-15 of each 32-lane
-// subpartition (row m -> lane (m % 16) + 32 (m / 16)); M=128 tiles use all lanes.
-constexpr uint32_t kTmA = 0, kTmP = 64, kTmW = 128, kTmU = 256, kTmO = 288, kTmSn = 320;
-constexpr uint32_t kTmCols = 512;
+// ---- prep CTA shared memory -------------------------------------------------------------------
+template <int DV> struct PrepSmem {
+    using I = Img<DV>;
+    static constexpr int kTile = kChunk * kDK * 2;         // [64 x 128] 16-bit tile
+    // A operands of the A/P products, per 64-channel block b: [Kr_b | Qh_b | Ql_b]
+    // (8 KB each), so that [Kr ; Qh] and [Qh ; Ql] are 128-row operands
+    static constexpr int kKQBlk = 3 * kChunk * 128;
+    static constexpr int kKQ = 0;
+    static constexpr int kKh = 2 * kKQBlk;                 // K exp(Gref - G), hi  [64 x 128] (B)
+    static constexpr int kKl = kKh + kTile;                //                  lo
+    static constexpr int kKgV = kKl + kTile;               // [K exp(G) | V] [64 x 256], V zero past DV
+    // [Tb | Tb]: the A operand of W (both row halves give the same rows, so all warps can read
+    // them); the first Tb is also the B operand of U^T = V^T Tb^T
+    static constexpr int kTbP = kKgV + kChunk * 2 * kDK * 2;
+    static constexpr int kImg = kTbP + 2 * kChunk * kChunk * 2;  // staging image (Img layout)
+    static constexpr int kBeta = kImg + I::kStride;              // fp32 [64]
+    static constexpr int kG0 = kBeta + kChunk * 4;               // fp32 [128] decay after token 0
+    static constexpr int kGref = kG0 + kDK * 4;                  //            after token 31
+    static constexpr int kGlast = kGref + kDK * 4;               //            after token 63
+    static constexpr int kBytes = kGlast + kDK * 4;
+    // The A/P operand area also holds, in turn: the raw bf16 inputs of the chunk (bulk-loaded
+    // rows of log_alpha, k, q, v; read into registers before the operands are written) and the
+    // fp32 scratch of the UT transform (once the A/P products complete).
+    static constexpr int kRawG = 0, kRawK = kChunk * 256, kRawQ = 2 * kChunk * 256, kRawV = 3 * kChunk * 256;
+    static constexpr int kRawBytes = kChunk * (3 * kDK * 2 + DV * 2);   // one TMA box per tensor
+    static constexpr int kLd = 68;                               // row stride of A and T^T
+    static constexpr int kA32 = 0;                               // A [64][68]
+    static constexpr int kT32 = kA32 + kChunk * kLd * 4;         // T^T [64][68] (row c = column c of T)
+    static constexpr int kX32 = kT32 + kChunk * kLd * 4;         // [3][16][20] block products, transposed
+    static constexpr int kTd32 = kX32 + 3 * 16 * 20 * 4;         // [4][16][20] diagonal blocks of T
+    static_assert(kTd32 + 4 * 16 * 20 * 4 <= kKgV && kRawV + kChunk * DV * 2 <= kKgV, "A/P operand area");
+    // scan scratch inside the K exp(G) | V operand (dead from [W | U] to the next rebase)
+    static constexpr int kTot = kKgV;                            // [8][128] per-warp totals
+    static constexpr int kPre = kTot + 8 * kDK * 4;              // [8][128] per-warp prefixes
+};
+
+template <int DV> constexpr int chunk_smem_bytes() {
+    return (ChainSmem<DV>::kBytes > PrepSmem<DV>::kBytes ? ChainSmem<DV>::kBytes : PrepSmem<DV>::kBytes) + 1024;
+}
+static_assert(chunk_smem_bytes<128>() <= 232448, "shared memory plan exceeds 227 KB");
+
+// TMEM columns (fp32 accumulators, M = 128 layout: row m -> lane m).
+// chain: D1^T double-buffered (0, 128), D2^T, the S^T operand (64 columns) and the U~^T operand (32)
+constexpr uint32_t kTmD1 = 0, kTmD2 = 256, kTmS = 384, kTmUt = 448, kTmChainCols = 512;
+constexpr uint32_t kTmA = 0, kTmP2 = 64, kTmW = 256, kTmUT = 384, kTmPrepCols = 512;  // prep
 
 // Descriptor of k-step `kk` (16 elements along K) of a K-major SW128 operand with `rows` rows.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int kk) {
     return tc::make_sdesc(base + (kk >> 2) * (rows * 128) + (kk & 3) * 32, 16, 1024, tc::kSwz128);
 }
-// Descriptor of k-step `kk` of an MN-major operand stored as [K rows x MN columns]:
-// SW64 when MN == 32, else 64-column SW128 blocks.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int krows, int mn, int kk) {
-    if (mn == 32) return tc::make_sdesc(base + kk * 1024, krows * 64, 512, tc::kSwz64);
+// Descriptor of k-step `kk` of an MN-major operand stored as [K rows x MN columns] in 64-column
+// SW128 blocks of krows x 128 bytes.
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int krows, int kk) {
     return tc::make_sdesc(base + kk * 2048, krows * 128, 1024, tc::kSwz128);
 }
-// Byte offset of 16-byte chunk `j` (8 16-bit columns) of row `r` in a tile with
-// `cols` columns stored as above (SW64 for 32 columns, SW128 64-column blocks).
-__device__ __forceinline__ uint32_t tile_chunk(int r, int j, int rows, int cols) {
-    if (cols == 32) return tc::sw64(r, j);
+// Byte offset of 16-byte chunk `j` (8 16-bit columns) of row `r` in a tile with `rows` rows
+// stored as 64-column SW128 blocks.
+__device__ __forceinline__ uint32_t tile_chunk(int r, int j, int rows) {
     return (j >> 3) * (rows * 128) + tc::sw128(r, j & 7);
 }
 
@@ -174,6 +195,15 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ void unpack8_h(const uint4 &u, float *f) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 x = __half22float2(h[i]);
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
@@ -233,37 +263,809 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, bool l
     tc::tc_fence_after();
     return !failed;
 }
+// Same with a phase completed by other CTAs of the cluster.
+__device__ __forceinline__ bool role_wait_cluster(uint64_t *bar, uint32_t parity, bool leader, uint32_t bar_id,
+                                                  uint32_t nthreads, volatile int *abort_flag) {
+    bool ok = true;
+    if (leader) ok = tc::mbar_wait_cluster(bar, parity, abort_flag);
+    const bool failed = tc::named_sync_or(bar_id, nthreads, !ok);
+    tc::tc_fence_after();
+    return !failed;
+}
 
-template <int CL, typename TO>
-__global__ void __launch_bounds__(kThreads, 1)
-kda_chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                    const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ log_alpha,
-                    const __nv_bfloat16 *__restrict__ beta, const float *init_state,
-                    const int32_t *__restrict__ cu_seqlens, int num_seqs, int T, int H, int DV,
-                    TO *__restrict__ out, float *final_state, uint8_t *__restrict__ workspace) {
-    using SM = ChunkSmem;
-    using I = ChunkImage;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = tc::smem_u32(sm);
+// Wait (bounded, ignoring the abort flag) for all tcgen05 operations this thread issued.
+__device__ __forceinline__ void drain_mma(uint64_t *bar, uint32_t parity) {
+    int never = 0;
+    tc::mma_commit(bar);
+    tc::mbar_wait(bar, parity, &never);
+}
+
+// Per-CTA bookkeeping shared by both roles.
+struct ChunkCtx {
+    int n, h, H, nchunks;
+    int64_t t0, t1;
+    uint32_t sbase, tmem;
+    uint8_t *sm;
+    uint8_t *ws_pair;        // this (sequence, head)'s kNP producer regions
+    volatile int *abort_flag;
+    // chunk c: first token and valid length
+    __device__ __forceinline__ int64_t tok0(int c) const { return t0 + (int64_t)c * kChunk; }
+    __device__ __forceinline__ int len(int c) const {
+        const int64_t r = t1 - tok0(c);
+        return static_cast<int>(r < kChunk ? r : kChunk);
+    }
+};
+
+// Mbarriers of one CTA (each role uses its own subset).
+struct ChunkBars {
+    // chain: image slot full / free, MMA completions, producer publications (per producer region)
+    uint64_t full[2], slot_free[2], mma1, mma2, mma3[2], pub[kNP][2];
+    // prep: MMA completions, global region consumed by the chain (per region)
+    uint64_t m_ap, m_wu, consumed[2], staged, staging_free, raw_full, raw_free;
+    uint64_t fin;
+    int chain_ok;   // the chain leader's last MMA wait succeeded (read after a barrier)
+};
+
+// ================================== prep role (cluster ranks 1..kNP) ==================================
+// Producer p prepares chunks c = p, p + kNP, ... with warps 0-7.  Its k-th chunk is written straight
+// from registers into global region (p, k % 2) of the workspace, then announced to the chain CTA.
+// Tensor maps of the token tensors: [tokens][H][d] bf16, one box = 64 tokens x d channels of one
+// head; and of the output [tokens][H][d_v] (fp32 or bf16), one box = 64 tokens x 64 values.
+struct RowMaps {
+    CUtensorMap g, k, q, v, o;
+};
+
+template <int DV>
+__device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, int p, const RowMaps &maps,
+                                          const __nv_bfloat16 *beta) {
+    using SM = PrepSmem<DV>;
+    using I = Img<DV>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t *const sm = cx.sm;
+    const uint32_t sbase = cx.sbase, tmem = cx.tmem;
+    const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
+    volatile int *abort_flag = cx.abort_flag;
+    if (warp == 8) {
+        // ---- publisher: staged image -> the chunk's global region (one bulk store), then announce the
+        //      region to the chain CTA ----
+        if (lane == 0) {
+            int kl = 0;
+            for (int c = p; c < nchunks; c += kNP, ++kl) {
+                const int reg = kl & 1;
+                uint8_t *gimg = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
+                if (!tc::mbar_wait(&bars.staged, kl & 1, abort_flag)) break;
+                tc::bulk_store_nc(gimg, sm + SM::kImg, I::kBytes);
+                tc::bulk_commit();
+                tc::bulk_wait_read_all();
+                tc::mbar_arrive(&bars.staging_free);
+                tc::bulk_wait_all();
+                tc::fence_async_global();
+                tc::mbar_arrive_cluster(tc::mapa(tc::smem_u32(&bars.pub[p][reg]), 0));
+            }
+        }
+        return;
+    }
+    if (warp == 9) {
+        // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next chunk
+        //      (TMA; rows past the tensor end read as zero, rows past the sequence end are masked by the
+        //      readers), into the A/P operand area once the previous chunk's UT scratch is dead ----
+        int kl = 0, issued = -1;
+        for (int c = p; c < nchunks; c += kNP, ++kl) {
+            bool ok = true;
+            if (lane == 0 && kl >= 1) ok = tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            const int64_t tok0 = cx.tok0(c);
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&bars.raw_full, SM::kRawBytes);
+                const int t = static_cast<int>(tok0);
+                tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
+                tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
+                tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
+                tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
+            }
+            issued = kl;
+        }
+        // no copy may still be in flight when the CTA leaves
+        if (lane == 0 && issued >= 0) {
+            int never = 0;
+            tc::mbar_wait(&bars.raw_full, issued & 1, &never);
+        }
+        return;
+    }
+    if (warp > 9) return;
+
+    const int tp = tid;
+    const bool leader = tp == 0;
+    const int cg = tp & 15, tg = tp >> 4;   // channels [8cg, 8cg+8), tokens [4tg, 4tg+4)
+    const int sp = warp & 3, half = warp >> 2;
+    const uint32_t tl = tc::tmem_lane_base(warp);
     float *sBeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *sG0 = reinterpret_cast<float *>(sm + SM::kG0);
     float *sGref = reinterpret_cast<float *>(sm + SM::kGref);
     float *sGlast = reinterpret_cast<float *>(sm + SM::kGlast);
     float *sTot = reinterpret_cast<float *>(sm + SM::kTot);
-    float *sRed = reinterpret_cast<float *>(sm + SM::kRed);
+    float *sPre = reinterpret_cast<float *>(sm + SM::kPre);
+    constexpr int ld = SM::kLd;
+    float *sA = reinterpret_cast<float *>(sm + SM::kA32);
+    float *sT = reinterpret_cast<float *>(sm + SM::kT32);
+    float *sX = reinterpret_cast<float *>(sm + SM::kX32);
+    float *sTd = reinterpret_cast<float *>(sm + SM::kTd32);
 
-    // chain: bar_m3, bar_m4 (MMA completion), full1/full2 (image part loads), pub[p] (chunk of
-    // producer p stored); prep: bar_m1, bar_m2 (MMA completion), consumed (all CL chains loaded
-    // this producer's last chunk)
-    __shared__ uint64_t bar_m1, bar_m2, bar_m3, bar_m4, full1, full2, consumed, pub[CL];
+    // beta of the next chunk, prefetched into registers (one value per thread of warps 0-1)
+    float rb = 0.f;
+    auto load_beta = [&](int c) {
+        const int64_t tok0 = cx.tok0(c);
+        rb = (tp < kChunk && tp < cx.len(c)) ? __bfloat162float(beta[(tok0 + tp) * H + h]) : 0.f;
+    };
+    // the staged chunk image is complete: set its flag (1: some value left the fp16 range, or the
+    // decays the rebasing range; the chain then evaluates the chunk exactly) and hand it to the
+    // publisher
+    uint8_t *const img = sm + SM::kImg;
+    auto stage_done = [&](bool mybad) {
+        tc::fence_async_smem();
+        const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
+        if (leader) {
+            *reinterpret_cast<volatile int *>(img + I::kFlag) = bad ? 1 : 0;
+            tc::fence_async_smem();
+            tc::mbar_arrive(&bars.staged);
+        }
+    };
+
+    uint32_t ph_ap = 0, ph_wu = 0;
+    if (p < nchunks) load_beta(p);
+    int kl = 0;
+    for (int c = p; c < nchunks; c += kNP, ++kl) {
+        const int reg = kl & 1;
+        // region `reg` last held this producer's chunk kl - 2: the chain must have loaded it
+        if (kl >= 2 &&
+            !role_wait_cluster(&bars.consumed[reg], ((kl >> 1) - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
+            break;
+        const int L = cx.len(c);
+        // the raw inputs of this chunk are in shared memory
+        if (!role_wait(&bars.raw_full, kl & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
+        // ---- decays: fp32 scan over the chunk, per channel ----
+        float G[4][8];
+        {
+            float run[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) run[i] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = tg * 4 + rr;
+                float g8[8];
+                const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
+                                        : make_uint4(0, 0, 0, 0);
+                unpack8(raw, g8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    run[i] += g8[i];
+                    G[rr][i] = run[i];
+                }
+            }
+            // lanes 16-31 hold the odd token group of the warp's pair: add the even one's total
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float lower = __shfl_up_sync(0xffffffffu, run[i], 16);
+                const float add = (lane >= 16) ? lower : 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) G[rr][i] += add;
+                if (lane >= 16) sTot[warp * kDK + cg * 8 + i] = run[i] + add;   // the warp's 8 tokens
+            }
+            if (tg == 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sG0[cg * 8 + i] = G[0][i];             // token 0: no prefix
+            }
+            if (tp < kChunk) sBeta[tp] = rb;
+        }
+        tc::named_sync(kBarRole, kRoleThreads);
+        // per channel: exclusive prefix over the 8 warps, G after tokens 31 and 63, range check
+        bool bad = false;
+        if (tp < kDK) {
+            float run = 0.f, gref = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                sPre[w * kDK + tp] = run;
+                run += sTot[w * kDK + tp];
+                if (w == 3) gref = run;
+            }
+            sGref[tp] = gref;
+            sGlast[tp] = run;
+            bad = !((sG0[tp] - gref <= kRangeLimit) && (gref - run <= kRangeLimit));
+        }
+        if (tc::named_sync_or(kBarRole, kRoleThreads, bad)) {
+            // decays too fast for the rebased products: the chain evaluates this chunk exactly
+            if (c + kNP < nchunks) load_beta(c + kNP);
+            if (leader) tc::mbar_arrive(&bars.raw_free);
+            if (kl >= 1 &&
+                !role_wait(&bars.staging_free, (kl - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
+                break;
+            stage_done(true);
+            continue;
+        }
+        {
+            float off[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) off[i] = sPre[warp * kDK + cg * 8 + i];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) G[rr][i] += off[i];
+        }
+
+        // the publisher has read the previous image out of the staging tiles
+        if (kl >= 1 &&
+            !role_wait(&bars.staging_free, (kl - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
+            break;
+        // ---- rebased and decayed operands; Q exp(G) and Kd into the staged image ----
+        bool ovf = false;   // an fp16 operand or image value out of range
+        uint4 rk[4], rq[4], rv[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int r = tg * 4 + rr;
+            const bool in = r < L;
+            rk[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawK + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
+            rq[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawQ + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
+            rv[rr] = (in && cg * 8 < DV) ? *reinterpret_cast<const uint4 *>(sm + SM::kRawV + r * DV * 2 + cg * 16)
+                                         : make_uint4(0, 0, 0, 0);
+        }
+        tc::named_sync(kBarRole, kRoleThreads);   // the operands below overwrite the raw rows
+        {
+            float gref[8], elast[8], erefabs[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                gref[i] = sGref[cg * 8 + i];
+                erefabs[i] = fast_exp(gref[i]);                       // exp(Gref)
+                elast[i] = fast_exp(sGlast[cg * 8 + i] - gref[i]);   // exp(Glast - Gref)
+            }
+            const uint32_t okq = SM::kKQ + (cg >> 3) * SM::kKQBlk;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = tg * 4 + rr;
+                float kf[8], qf[8];
+                unpack8(rk[rr], kf);
+                unpack8(rq[rr], qf);
+                float kr[8], qr[8], kn[8], kd[8], kg[8], qg[8], vf[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float dg = G[rr][i] - gref[i];
+                    const float e1 = fast_exp(dg), e2 = fast_exp(-dg);
+                    kr[i] = kf[i] * e1;
+                    qr[i] = qf[i] * e1;
+                    kn[i] = kf[i] * e2;
+                    kd[i] = kn[i] * elast[i];
+                    kg[i] = kr[i] * erefabs[i];
+                    qg[i] = qr[i] * erefabs[i];
+                }
+                const uint32_t o128 = tile_chunk(r, cg, kChunk);   // [64 x 128] tiles
+                *reinterpret_cast<uint4 *>(sm + SM::kKgV + o128) = pack8_h(kg);
+                *reinterpret_cast<uint4 *>(img + I::kQt + o128) = pack8_h(qg);
+                unpack8(rv[rr], vf);   // zero past DV
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ovf |= !(fabsf(vf[i]) <= 65000.f);
+                *reinterpret_cast<uint4 *>(sm + SM::kKgV + tile_chunk(r, 16 + cg, kChunk)) = pack8_h(vf);
+                const uint32_t okr = okq + tc::sw128(r, cg & 7);   // [Kr | Qh | Ql] blocks
+                uint4 hi, lo;
+                *reinterpret_cast<uint4 *>(sm + okr) = pack8_bf16(kr);
+                split8_bf16(qr, hi, lo);
+                *reinterpret_cast<uint4 *>(sm + okr + 8192) = hi;
+                *reinterpret_cast<uint4 *>(sm + okr + 16384) = lo;
+                split8_bf16(kn, hi, lo);
+                *reinterpret_cast<uint4 *>(sm + SM::kKh + o128) = hi;
+                *reinterpret_cast<uint4 *>(sm + SM::kKl + o128) = lo;
+                *reinterpret_cast<uint4 *>(img + I::kKd + o128) = pack8_h(kd);
+            }
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        tc::named_sync(kBarRole, kRoleThreads);
+
+        // ---- A/P products: D_A = [Kr ; Qh] Kh^T (rows 0-63 A_raw, rows 64-127 Qh Kh^T),
+        //      D_P2 = [Kr ; Qh] Kl^T + [Qh ; Ql] Kh^T (rows 64-127 Qh Kl^T + Ql Kh^T) ----
+        if (leader) {
+            tc::tc_fence_after();
+            constexpr uint32_t id = tc::make_idesc(128, 64, tc::kBF16, false, false);
+#pragma unroll
+            for (int kk = 0; kk < kDK / 16; ++kk) {
+                const uint32_t a0 = sbase + SM::kKQ + (kk >> 2) * SM::kKQBlk + (kk & 3) * 32;
+                const uint64_t akq = tc::make_sdesc(a0, 16, 1024, tc::kSwz128);
+                const uint64_t aqq = tc::make_sdesc(a0 + 8192, 16, 1024, tc::kSwz128);
+                const uint64_t bh = desc_kmajor(sbase + SM::kKh, kChunk, kk);
+                const uint64_t bl = desc_kmajor(sbase + SM::kKl, kChunk, kk);
+                tc::mma_f16(tmem + kTmA, akq, bh, id, kk > 0);
+                tc::mma_f16(tmem + kTmP2, akq, bl, id, kk > 0);
+                tc::mma_f16(tmem + kTmP2, aqq, bh, id, true);
+            }
+            tc::mma_commit(&bars.m_ap);
+        }
+        if (c + kNP < nchunks) load_beta(c + kNP);
+        if (!role_wait(&bars.m_ap, ph_ap, leader, kBarRole, kRoleThreads, abort_flag)) break;
+        ph_ap ^= 1u;
+
+        // ---- A (fp32, beta-scaled, strict lower) and tril(P) (fp16 A operand) ----
+        {
+            const int m = sp * 32 + lane;   // accumulator row
+            const int c0 = half * 32;       // columns [c0, c0 + 32)
+            if (sp < 2) {
+                const int r = m;
+                const float br = sBeta[r];
+#pragma unroll
+                for (int c16 = 0; c16 < 2; ++c16) {
+                    float x16[16];
+                    tc::tmem_ld16(tmem + tl + kTmA + c0 + c16 * 16, x16);
+                    tc::tmem_ld_wait();
+                    const int cb = c0 + c16 * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<float4 *>(&sA[r * ld + cb + i]) =
+                            make_float4((cb + i < r) ? br * x16[i] : 0.f, (cb + i + 1 < r) ? br * x16[i + 1] : 0.f,
+                                        (cb + i + 2 < r) ? br * x16[i + 2] : 0.f,
+                                        (cb + i + 3 < r) ? br * x16[i + 3] : 0.f);
+                }
+            } else {
+                const int r = m - 64;
+#pragma unroll
+                for (int c16 = 0; c16 < 2; ++c16) {
+                    float x16[16], y16[16];
+                    tc::tmem_ld16(tmem + tl + kTmA + c0 + c16 * 16, x16);
+                    tc::tmem_ld16(tmem + tl + kTmP2 + c0 + c16 * 16, y16);
+                    tc::tmem_ld_wait();
+                    const int cb = c0 + c16 * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x16[i] = (cb + i <= r) ? x16[i] + y16[i] : 0.f;
+                    *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8, kChunk)) = pack8_h(x16);
+                    *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8 + 1, kChunk)) = pack8_h(x16 + 8);
+                }
+            }
+        }
+        tc::tc_fence_before();
+        tc::named_sync(kBarRole, kRoleThreads);
+
+        // ---- UT transform T = (I + A)^{-1} ----
+        // (a) 16x16 diagonal blocks: four threads (p = tp % 4) solve column cc of (I + A_bb) x = e_cc by
+        //     right-looking substitution: thread p keeps rows r = p + 4 k in registers, the owner of
+        //     row s finalises x_s and shuffles it to the other three, which update their later rows.
+        //     The zeros above the diagonal are written too.
+        {
+            const int col = tp >> 2, pp = tp & 3;
+            const int bb = col >> 4, cc = col & 15;
+            float a[4][16], part[4], x[4];
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                const float *arow = sA + (16 * bb + pp + 4 * kq) * ld + 16 * bb;
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(arow + 4 * s4);
+                    a[kq][4 * s4] = v4.x;
+                    a[kq][4 * s4 + 1] = v4.y;
+                    a[kq][4 * s4 + 2] = v4.z;
+                    a[kq][4 * s4 + 3] = v4.w;
+                }
+                part[kq] = 0.f;
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) {
+                float xs = (s2 == cc) ? 1.f : ((s2 < cc) ? 0.f : -part[s2 >> 2]);
+                xs = __shfl_sync(0xffffffffu, xs, (lane & ~3) | (s2 & 3));
+                if (pp == (s2 & 3)) x[s2 >> 2] = xs;
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)
+                    if (pp + 4 * kq > s2) part[kq] = fmaf(a[kq][s2], xs, part[kq]);
+            }
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                sT[(16 * bb + cc) * ld + 16 * bb + pp + 4 * kq] = x[kq];   // T^T
+                sTd[(bb * 16 + pp + 4 * kq) * 20 + cc] = x[kq];            // T_bb, row-major
+            }
+        }
+        tc::named_sync(kBarRole, kRoleThreads);
+        // (b) off-diagonal blocks by distance d = i - j: T_ij = -T_ii sum_{j<=m<i} A_im T_mj.
+        //     The 4 - d blocks of one distance are independent; 256 threads = one 16x16 block.  With T
+        //     stored transposed, both factors of every dot product are contiguous (float4 reads).
+        {
+            const int r = tp >> 4, cc = tp & 15;
+#pragma unroll 1
+            for (int d = 1; d < 4; ++d) {
+#pragma unroll 1
+                for (int blk = 0; blk < 4 - d; ++blk) {
+                    const int j = blk, i = blk + d;
+                    const float *arow = sA + (16 * i + r) * ld + 16 * j;     // A[16i + r][16j + m]
+                    const float *tcol = sT + (16 * j + cc) * ld + 16 * j;    // T[16j + m][16j + cc]
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int m = 0; m < 16 * d; m += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
+                        const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m);
+                        acc[0] = fmaf(a4.x, t4.x, acc[0]);
+                        acc[1] = fmaf(a4.y, t4.y, acc[1]);
+                        acc[2] = fmaf(a4.z, t4.z, acc[2]);
+                        acc[3] = fmaf(a4.w, t4.w, acc[3]);
+                    }
+                    sX[(blk * 16 + cc) * 20 + r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // X^T
+                }
+                tc::named_sync(kBarRole, kRoleThreads);
+#pragma unroll 1
+                for (int blk = 0; blk < 4 - d; ++blk) {
+                    const int j = blk, i = blk + d;
+                    const float *drow = sTd + (i * 16 + r) * 20;   // T_ii[r][m] (zero above the diagonal)
+                    const float *xcol = sX + (blk * 16 + cc) * 20;  // X[m][cc]
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 16; m += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
+                        const float4 x4 = *reinterpret_cast<const float4 *>(xcol + m);
+                        acc[0] = fmaf(t4.x, x4.x, acc[0]);
+                        acc[1] = fmaf(t4.y, x4.y, acc[1]);
+                        acc[2] = fmaf(t4.z, x4.z, acc[2]);
+                        acc[3] = fmaf(t4.w, x4.w, acc[3]);
+                    }
+                    sT[(16 * j + cc) * ld + 16 * i + r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));   // T^T
+                }
+                tc::named_sync(kBarRole, kRoleThreads);
+            }
+        }
+        // T diag(beta) -> fp16 A operand [64 x 64]: 2 chunks of 8 per thread; the strictly upper
+        // blocks of sT are never written, so the mask j*8 + i <= r is applied here
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int idx = tp * 2 + e, r = idx >> 3, j = idx & 7;
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? sT[(j * 8 + i) * ld + r] * sBeta[j * 8 + i] : 0.f;
+            const uint4 t8 = pack8_h(f);
+            *reinterpret_cast<uint4 *>(sm + SM::kTbP + tile_chunk(r, j, kChunk)) = t8;
+            *reinterpret_cast<uint4 *>(sm + SM::kTbP + 8192 + tile_chunk(r, j, kChunk)) = t8;
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        tc::named_sync(kBarRole, kRoleThreads);
+        if (leader) tc::mbar_arrive(&bars.raw_free);   // the UT scratch is dead: next raw rows may land
+
+        // ---- W = Tb Kg, twice (A = [Tb ; Tb]);  U^T = V^T Tb^T (A = V^T, MN-major; B = Tb) ----
+        if (leader) {
+            tc::tc_fence_after();
+            constexpr uint32_t idW = tc::make_idesc(128, kDK, tc::kF16, false, true);
+            constexpr uint32_t idUT = tc::make_idesc(128, kChunk, tc::kF16, true, false);
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk) {
+                tc::mma_f16(tmem + kTmW, tc::make_sdesc(sbase + SM::kTbP + kk * 32, 16, 1024, tc::kSwz128),
+                            desc_mnmajor(sbase + SM::kKgV, kChunk, kk), idW, kk > 0);
+                tc::mma_f16(tmem + kTmUT, desc_mnmajor(sbase + SM::kKgV + 2 * 8192, kChunk, kk),
+                            desc_kmajor(sbase + SM::kTbP, kChunk, kk), idUT, kk > 0);
+            }
+            tc::mma_commit(&bars.m_wu);
+        }
+        if (!role_wait(&bars.m_wu, ph_wu, leader, kBarRole, kRoleThreads, abort_flag)) break;
+        ph_wu ^= 1u;
+        // -W (rows 0-63, duplicated in 64-127: warp (sp, half) takes rows 32 (sp % 2) + lane, columns
+        // 32 (2 (sp / 2) + half) + [0, 32)) and U^T (value row j = 32 sp + lane, tokens 32 half + [0, 32))
+        // -> fp16 in the staged image
+        {
+            float x[32];
+            const int r = (sp & 1) * 32 + lane, qd = (sp >> 1) * 2 + half;
+            tc::tmem_ld32(tmem + tl + kTmW + qd * 32, x);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                x[i] = -x[i];
+                ovf |= !(fabsf(x[i]) <= 65000.f);
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, 4 * qd + q4, kChunk)) = pack8_h(x + 8 * q4);
+            const int j = sp * 32 + lane;
+            tc::tmem_ld32(tmem + tl + kTmUT + half * 32, x);
+            tc::tmem_ld_wait();
+            if (j < DV) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ovf |= !(fabsf(x[i]) <= 65000.f);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(img + I::kUT + tile_chunk(j, 4 * half + q4, DV)) = pack8_h(x + 8 * q4);
+            }
+        }
+        if (tp < kDK) reinterpret_cast<float *>(img + I::kGam)[tp] = fast_exp(sGlast[tp]);
+        tc::tc_fence_before();
+        stage_done(ovf);
+    }
+    if (leader) drain_mma(&bars.fin, 0);
+}
+
+// ================================== chain role (cluster rank 0) =====================================
+// The chain works on transposed tiles so that the state and U~ are the A operands of its MMAs,
+// held in TMEM:
+//   D1^T = S^T [-W ; Qg]^T        (columns 0-63: (U~ - U)^T, columns 64-127: (Qg S)^T)
+//   D2^T = U~^T Kd                 (the state increment, transposed)
+//   D1^T[:, 64:128] += U~^T P^T    (so that columns 64-127 become O^T)
+// Warps 0-7 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
+// channels [64 (w / 4), 64 (w / 4) + 64) of S^T.  Lane 0 of warp 8 loads the chunk images.
+template <int DV, typename TO>
+__device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const RowMaps &maps,
+                                           const __nv_bfloat16 *q,
+                                           const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                                           const __nv_bfloat16 *log_alpha, const __nv_bfloat16 *beta,
+                                           const float *init_state, TO *out, float *final_state) {
+    using SM = ChainSmem<DV>;
+    using I = Img<DV>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t *const sm = cx.sm;
+    const uint32_t sbase = cx.sbase, tmem = cx.tmem;
+    const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
+    volatile int *abort_flag = cx.abort_flag;
+
+    if (warp == 8) {
+        // ---- loader: producer region -> image slot c % 2, once the slot is free and the image published ----
+        if (lane == 0) {
+            int last = -1;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                if (c >= 2) {
+                    if (!tc::mbar_wait(&bars.slot_free[s], ((c >> 1) - 1) & 1, abort_flag)) break;
+                    // chunk c - 2 has long been loaded: its producer may rewrite that region
+                    const int pc = c - 2;
+                    tc::mbar_arrive_cluster_relaxed(
+                        tc::mapa(tc::smem_u32(&bars.consumed[(pc / kNP) & 1]), 1 + pc % kNP));
+                }
+                const int p = c % kNP, kq = c / kNP, reg = kq & 1;
+                if (!tc::mbar_wait_cluster(&bars.pub[p][reg], (kq >> 1) & 1, abort_flag)) break;
+                tc::fence_async_global();
+                const uint8_t *src = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
+                uint8_t *slot = sm + s * SM::kSlotBytes;
+                uint64_t *fb = &bars.full[s];
+                tc::mbar_arrive_expect_tx(fb, I::kBytes);
+                tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
+                tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
+                tc::bulk_load(slot + SM::kA1 + 8192, src + I::kQt, 8192, fb);
+                tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
+                tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
+                tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
+                last = c;
+            }
+            // no copy may still be in flight when the CTA leaves
+            int never = 0;
+            for (int c = (last >= 1 ? last - 1 : 0); c <= last; ++c)
+                tc::mbar_wait(&bars.full[c & 1], (c >> 1) & 1, &never);
+        }
+        return;
+    }
+    if (warp > 8) return;
+
+    const bool leader = tid == 0;
+    const int sp = warp & 3, half = warp >> 2;
+    const int j = sp * 32 + lane;            // value column (TMEM lane)
+    const bool jv = j < DV;
+    const int c0 = half * 64;                // key channels [c0, c0 + 64)
+    const uint32_t tl = tc::tmem_lane_base(warp);
+    float *redPk = reinterpret_cast<float *>(sm + SM::kRedPk);
+    float *redPq = reinterpret_cast<float *>(sm + SM::kRedPq);
+    float *redKq = reinterpret_cast<float *>(sm + SM::kRedKq);
+
+    float S[64];  // fp32 master state: S^T[j][c0 + i]
+    const size_t state_base = ((size_t)cx.n * H + h) * kDK * DV + (size_t)c0 * DV + j;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
+    // S^T -> fp16 A operand in TMEM (lane j, channels c0..c0+63 in 32 columns); returns whether some
+    // entry left the fp16 range
+    auto write_state_operand = [&]() -> bool {
+        bool big = false;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) big |= !(fabsf(S[i]) <= 65000.f);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            uint32_t u[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) u[i] = pack_h(S[32 * g + 2 * i], S[32 * g + 2 * i + 1]);
+            tc::tmem_st16(tmem + tl + kTmS + half * 32 + g * 16, u);
+        }
+        tc::tmem_st_wait();
+        return big;
+    };
+    tc::tc_fence_before();
+    bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
+
+    // token-by-token fp32 evaluation of one chunk from the state in registers
+    auto exact_chunk = [&](int64_t tok0, int L) -> bool {
+        for (int r = 0; r < L; ++r) {
+            const int64_t trow = (tok0 + r) * H + h;
+            const __nv_bfloat16 *gr = log_alpha + trow * kDK + c0, *kr = k + trow * kDK + c0,
+                                *qr = q + trow * kDK + c0;
+            float pk = 0.f, pq = 0.f, kq = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float a = expf(__bfloat162float(gr[i])), kk = __bfloat162float(kr[i]),
+                            qq = __bfloat162float(qr[i]);
+                S[i] *= a;
+                pk = fmaf(S[i], kk, pk);
+                pq = fmaf(S[i], qq, pq);
+                kq = fmaf(kk, qq, kq);
+            }
+            redPk[half * 128 + j] = pk;
+            redPq[half * 128 + j] = pq;
+            if (sp == 0 && lane == 0) redKq[half] = kq;
+            tc::named_sync(kBarRole, kRoleThreads);
+            const float u = jv ? __bfloat162float(beta[trow]) *
+                                     (__bfloat162float(v[trow * DV + j]) - (redPk[j] + redPk[128 + j]))
+                               : 0.f;
+            if (half == 0 && jv)
+                out[trow * DV + j] = from_f32<TO>(fmaf(u, redKq[0] + redKq[1], redPq[j] + redPq[128 + j]));
+#pragma unroll
+            for (int i = 0; i < 64; ++i) S[i] = fmaf(__bfloat162float(kr[i]), u, S[i]);
+            tc::named_sync(kBarRole, kRoleThreads);
+        }
+        return write_state_operand();
+    };
+
+    // output of a tensor-path chunk: columns 64-127 of D1^T[b] hold O^T once [. ; P] U~ completed;
+    // thread (j, half) has tokens 32 half + [0, 32) of value column j.  A full chunk is staged in
+    // shared memory (a warp writes 32 consecutive values of one token: no bank conflicts) and written
+    // by TMA tensor stores; a partial last chunk is stored directly.
+    uint32_t ph_m3[2] = {0, 0};
+    TO *const stage = reinterpret_cast<TO *>(sm + SM::kOut);
+    auto store_output = [&](int cp, int bp) -> bool {
+        if (leader) tc::bulk_wait_read_all();   // the previous chunk's stores have read the staging
+        if (!role_wait(&bars.mma3[bp], ph_m3[bp], leader, kBarRole, kRoleThreads, abort_flag)) return false;
+        ph_m3[bp] ^= 1u;
+        float o[32];
+        tc::tmem_ld32(tmem + tl + kTmD1 + bp * 128 + 64 + half * 32, o);
+        tc::tmem_ld_wait();
+        const int64_t tok0 = cx.tok0(cp);
+        const int L = cx.len(cp);
+        if (L == kChunk) {
+            if (jv) {
+                TO *col = stage + (j >> 6) * (kChunk * 64) + (j & 63);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) col[(half * 32 + i) * 64] = from_f32<TO>(o[i]);
+            }
+            tc::fence_async_smem();
+            tc::named_sync(kBarRole, kRoleThreads);
+            if (leader) {
+#pragma unroll
+                for (int blk = 0; blk < DV / 64; ++blk)
+                    tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0), stage + blk * (kChunk * 64));
+                tc::bulk_commit();
+            }
+        } else if (jv) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = half * 32 + i;
+                if (r < L) out[((tok0 + r) * H + h) * DV + j] = from_f32<TO>(o[i]);
+            }
+        }
+        return true;
+    };
+
+    uint32_t ph1 = 0, ph2 = 0;
+    bool prev_tensor = false;   // chunk c - 1 went through the tensor path: its output is pending
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1, b = c & 1;
+        const int64_t tok0 = cx.tok0(c);
+        const int L = cx.len(c);
+        const uint8_t *slot = sm + s * SM::kSlotBytes;
+        const uint32_t sslot = sbase + s * SM::kSlotBytes;
+        if (!role_wait(&bars.full[s], (c >> 1) & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
+        const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
+        if (!flagged && leader) {
+            // ---- D1^T[b] = S^T [-W ; Qg]^T ----
+            constexpr uint32_t id1 = tc::make_idesc(128, 128, tc::kF16, false, false);
+#pragma unroll
+            for (int kk = 0; kk < kDK / 16; ++kk)
+                tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8, desc_kmajor(sslot + SM::kA1, 128, kk),
+                               id1, kk > 0);
+            tc::mma_commit(&bars.mma1);
+        }
+        // the previous chunk's output, while D1^T[b] is computed; then its slot is free
+        if (prev_tensor && !store_output(c - 1, b ^ 1)) break;
+        if (c >= 1 && leader) tc::mbar_arrive(&bars.slot_free[s ^ 1]);
+        prev_tensor = false;
+        if (!flagged) {
+            if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) break;
+            ph1 ^= 1u;
+            // ---- U~^T = U^T + (-W S)^T (tokens 32 half + [0, 32)) -> fp16 A operand in TMEM ----
+            bool mybad = force_exact;
+            {
+                float x[32];
+                tc::tmem_ld32(tmem + tl + kTmD1 + b * 128 + half * 32, x);
+                tc::tmem_ld_wait();
+                uint32_t u[16];
+                if (jv) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float u8[8];
+                        unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 4 * half + q4, DV)),
+                                  u8);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) x[8 * q4 + i] += u8[i];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mybad |= !(fabsf(x[i]) <= 65000.f);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) u[i] = pack_h(x[2 * i], x[2 * i + 1]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) u[i] = 0u;
+                }
+                tc::tmem_st16(tmem + tl + kTmUt + half * 16, u);
+                tc::tmem_st_wait();
+            }
+            tc::tc_fence_before();
+            const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
+            if (leader) {
+                tc::tc_fence_after();
+                // ---- D2^T = U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
+                constexpr uint32_t id2 = tc::make_idesc(128, 128, tc::kF16, false, true);
+                constexpr uint32_t id3 = tc::make_idesc(128, kChunk, tc::kF16, false, false);
+#pragma unroll
+                for (int kk = 0; kk < kChunk / 16; ++kk)
+                    tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + SM::kKd, kChunk, kk),
+                                   id2, kk > 0);
+                tc::mma_commit(&bars.mma2);
+#pragma unroll
+                for (int kk = 0; kk < kChunk / 16; ++kk)
+                    tc::mma_f16_ta(tmem + kTmD1 + b * 128 + 64, tmem + kTmUt + kk * 8,
+                                   desc_kmajor(sslot + SM::kP, kChunk, kk), id3, true);
+                tc::mma_commit(&bars.mma3[b]);
+            }
+            if (!role_wait(&bars.mma2, ph2, leader, kBarRole, kRoleThreads, abort_flag)) break;
+            ph2 ^= 1u;
+            if (!bad) {
+                // ---- S^T = S^T Diag(gamma) + D2^T ----
+                const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float d[32];
+                    tc::tmem_ld32(tmem + tl + kTmD2 + c0 + g * 32, d);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 gg = gam4[g * 8 + i4];
+                        const int i = 32 * g + 4 * i4;
+                        S[i] = fmaf(gg.x, S[i], d[4 * i4]);
+                        S[i + 1] = fmaf(gg.y, S[i + 1], d[4 * i4 + 1]);
+                        S[i + 2] = fmaf(gg.z, S[i + 2], d[4 * i4 + 2]);
+                        S[i + 3] = fmaf(gg.w, S[i + 3], d[4 * i4 + 3]);
+                    }
+                }
+                const bool big = write_state_operand();
+                tc::tc_fence_before();
+                force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+                prev_tensor = true;
+                continue;
+            }
+            // this chunk is evaluated exactly: its pending [. ; P] U~ must still complete
+            if (!role_wait(&bars.mma3[b], ph_m3[b], leader, kBarRole, kRoleThreads, abort_flag)) break;
+            ph_m3[b] ^= 1u;
+        }
+        // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
+        const bool big = exact_chunk(tok0, L);
+        tc::tc_fence_before();
+        force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+    }
+    if (prev_tensor && nchunks > 0) store_output(nchunks - 1, (nchunks - 1) & 1);
+    if (leader) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
+    if (final_state && *abort_flag == 0 && jv) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) final_state[state_base + (size_t)i * DV] = S[i];
+    }
+    if (leader) drain_mma(&bars.fin, 0);
+}
+
+// ====================================== kernel and launch ==========================================
+template <int DV, typename TO>
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __nv_bfloat16 *__restrict__ q,
+                    const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                    const __nv_bfloat16 *__restrict__ log_alpha, const __nv_bfloat16 *__restrict__ beta,
+                    const float *init_state, const int32_t *__restrict__ cu_seqlens, int num_seqs, int T, int H,
+                    TO *__restrict__ out, float *final_state, uint8_t *__restrict__ workspace) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ ChunkBars bars;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ int s_slot;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rank = static_cast<int>(tc::cluster_ctarank());   // == value slice
-    const int pair = blockIdx.x / CL;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int rank = static_cast<int>(tc::cluster_ctarank());
+    const int pair = blockIdx.x / kCL;
     const int h = pair % H;
     int n = pair / H;
     int64_t t0, t1;
@@ -275,647 +1077,136 @@ kda_chunk_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         t0 = (int64_t)n * T;
         t1 = t0 + T;
     }
-    const int nchunks = static_cast<int>((t1 - t0 + kChunk - 1) / kChunk);
-    const int vcol0 = rank * kNV;
-    uint8_t *ws_cluster = workspace + (size_t)pair * CL * I::kStride;  // CL producer regions
 
     if (tid == 0) {
-        tc::mbar_init(&bar_m1, 1);
-        tc::mbar_init(&bar_m2, 1);
-        tc::mbar_init(&bar_m3, 1);
-        tc::mbar_init(&bar_m4, 1);
-        tc::mbar_init(&full1, 1);
-        tc::mbar_init(&full2, 1);
-        tc::mbar_init(&consumed, CL);
-        for (int p = 0; p < CL; ++p) tc::mbar_init(&pub[p], 1);
+        tc::mbar_init(&bars.full[0], 1);
+        tc::mbar_init(&bars.full[1], 1);
+        tc::mbar_init(&bars.slot_free[0], 1);
+        tc::mbar_init(&bars.slot_free[1], 1);
+        tc::mbar_init(&bars.mma1, 1);
+        tc::mbar_init(&bars.mma2, 1);
+        tc::mbar_init(&bars.mma3[0], 1);
+        tc::mbar_init(&bars.mma3[1], 1);
+        for (int p = 0; p < kNP; ++p) {
+            tc::mbar_init(&bars.pub[p][0], 1);
+            tc::mbar_init(&bars.pub[p][1], 1);
+        }
+        tc::mbar_init(&bars.m_ap, 1);
+        tc::mbar_init(&bars.m_wu, 1);
+        tc::mbar_init(&bars.consumed[0], 1);
+        tc::mbar_init(&bars.consumed[1], 1);
+        tc::mbar_init(&bars.staged, 1);
+        tc::mbar_init(&bars.staging_free, 1);
+        tc::mbar_init(&bars.raw_full, 1);
+        tc::mbar_init(&bars.raw_free, 1);
+        tc::mbar_init(&bars.fin, 1);
         tc::fence_mbar_init();
         abort_flag = 0;
     }
+    const uint32_t ncols = rank == 0 ? kTmChainCols : kTmPrepCols;
     if (warp == 0) {
-        tc::tmem_alloc(&tmem_base_sh, kTmCols);
+        tc::tmem_alloc(&tmem_base_sh, ncols);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::cluster_sync();  // every CTA's barriers are initialised before any remote arrive
     tc::tc_fence_after();
-    const uint32_t tmem = tmem_base_sh;
-    const uint32_t tl = tc::tmem_lane_base(warp);
 
-    if (warp < 4) {
-        // ===================================== chain role =====================================
-        const bool leader = tid == 0;
-        uint8_t *slot = sm + SM::kSlot;
-        const float *sGam = reinterpret_cast<const float *>(slot + I::kGamma);
-        const volatile int *sFlag = reinterpret_cast<const volatile int *>(slot + I::kFlag);
-        float S[kNV];  // fp32 master state: key row tid, this slice's value columns
-        const size_t state_base = ((size_t)n * H + h) * kDK * DV + (size_t)tid * DV + vcol0;
-#pragma unroll
-        for (int j = 0; j < kNV; ++j) S[j] = init_state ? init_state[state_base + j] : 0.f;
-        auto write_state_operand = [&]() {
-#pragma unroll
-            for (int j = 0; j < kNV / 8; ++j)
-                *reinterpret_cast<uint4 *>(sm + SM::kS + tile_chunk(tid, j, kDK, kNV)) = pack8_h(&S[8 * j]);
-            tc::fence_async_smem();
-        };
-        write_state_operand();
-
-        // V slice of a chunk: 64 rows x 4 chunks of 8 values, two per thread, prefetched a chunk ahead
-        uint4 rv[2];
-        auto load_v = [&](int c) {
-            const int64_t tok0 = t0 + (int64_t)c * kChunk;
-            const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = tid + e * kChainThreads, r = idx >> 2, j = idx & 3;
-                rv[e] = (r < L) ? *reinterpret_cast<const uint4 *>(v + ((tok0 + r) * H + h) * DV + vcol0 + j * 8)
-                                : make_uint4(0, 0, 0, 0);
-            }
-        };
-
-        // token-by-token fp32 evaluation of one chunk from the state in registers
-        auto exact_chunk = [&](int64_t tok0, int L) {
-            for (int r = 0; r < L; ++r) {
-                const int64_t row = (tok0 + r) * H + h;
-                const float a = expf(__bfloat162float(log_alpha[row * kDK + tid]));
-                const float kk = __bfloat162float(k[row * kDK + tid]);
-                const float qq = __bfloat162float(q[row * kDK + tid]);
-                float va[32], vb[32];
-#pragma unroll
-                for (int j = 0; j < kNV; ++j) {
-                    S[j] *= a;
-                    va[j] = S[j] * kk;
-                    vb[j] = S[j] * qq;
-                }
-                warp_transpose_sum32(va, lane);
-                warp_transpose_sum32(vb, lane);
-                float kq = kk * qq;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
-                sRed[warp * 64 + lane] = va[0];
-                sRed[warp * 64 + 32 + lane] = vb[0];
-                if (lane == 0) sRed[256 + warp] = kq;
-                tc::named_sync(kBarChain, kChainThreads);
-                if (warp == 0) {
-                    float aa = 0.f, bb = 0.f, kqs = 0.f;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        aa += sRed[w * 64 + lane];
-                        bb += sRed[w * 64 + 32 + lane];
-                        kqs += sRed[256 + w];
-                    }
-                    const float u = __bfloat162float(beta[row]) *
-                                    (__bfloat162float(v[row * DV + vcol0 + lane]) - aa);
-                    sRed[260 + lane] = u;
-                    out[row * DV + vcol0 + lane] = from_f32<TO>(fmaf(u, kqs, bb));
-                }
-                tc::named_sync(kBarChain, kChainThreads);
-#pragma unroll
-                for (int j = 0; j < kNV; ++j) S[j] = fmaf(kk, sRed[260 + j], S[j]);
-                tc::named_sync(kBarChain, kChainThreads);
-            }
-            write_state_operand();
-        };
-
-        // image loads (leader only): part 1 = Qg, W, Tb, gamma, flag; part 2 = Kd, P
-        auto region = [&](int c) -> const uint8_t * { return ws_cluster + (size_t)(c % CL) * I::kStride; };
-        auto issue_part1 = [&](int c) {
-            tc::mbar_arrive_expect_tx(&full1, I::kPart1Bytes);
-            tc::bulk_load(slot + I::kPart1, region(c) + I::kPart1, I::kPart1Bytes, &full1);
-        };
-        auto issue_part2 = [&](int c) {
-            tc::mbar_arrive_expect_tx(&full2, I::kPart2Bytes);
-            tc::bulk_load(slot, region(c), I::kPart2Bytes, &full2);
-        };
-        bool pre1 = false, pre2 = false;  // parts of the next chunk already issued (leader's view)
-
-        uint32_t ph_m3 = 0, ph_m4 = 0;
-        if (nchunks > 0) load_v(0);
-        tc::named_sync(kBarChain, kChainThreads);
-        for (int c = 0; c < nchunks; ++c) {
-            const int64_t tok0 = t0 + (int64_t)c * kChunk;
-            const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
-            const int prod = c % CL;
-            // ---- make sure this chunk's image loads are in flight ----
-            if (leader && !(pre1 && pre2)) {
-                bool ok = true;
-                if (!pre1) {
-                    ok = tc::mbar_wait_cluster(&pub[prod], (c / CL) & 1, &abort_flag);
-                    tc::fence_async_global();
-                    if (ok) issue_part1(c);
-                }
-                if (ok && !pre2) issue_part2(c);
-            }
-            pre1 = pre2 = false;
-            // V slice of this chunk (the previous chunk's U MMA has completed)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = tid + e * kChainThreads;
-                float f[8];
-                unpack8(rv[e], f);
-                *reinterpret_cast<uint4 *>(sm + SM::kV + tile_chunk(idx >> 2, idx & 3, kChunk, kNV)) = pack8_h(f);
-            }
-            tc::fence_async_smem();
-            if (c + 1 < nchunks) load_v(c + 1);
-            if (!role_wait(&full1, c & 1, leader, kBarChain, kChainThreads, &abort_flag)) break;
-            const bool exact = *sFlag != 0;
-            const float gam = sGam[tid];
-            bool bad = exact;
-            bool part2_done = false;
-            if (!exact) {
-                // ---- M3: U = Tb V;  U~ = U - W S;  O = Qg S ----
-                if (leader) {
-                    constexpr uint32_t idU = tc::make_idesc(64, kNV, tc::kF16, false, true);
-                    constexpr uint32_t idNeg = tc::make_idesc(64, kNV, tc::kF16, false, true, true);
-                    constexpr uint32_t idO = tc::make_idesc(64, kNV, tc::kF16, false, true);
-#pragma unroll
-                    for (int kk = 0; kk < kChunk / 16; ++kk)
-                        tc::mma_f16(tmem + kTmU, desc_kmajor(sbase + SM::kSlot + I::kTb, kChunk, kk),
-                                    desc_mnmajor(sbase + SM::kV, kChunk, kNV, kk), idU, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < kDK / 16; ++kk) {
-                        const uint64_t bdesc = desc_mnmajor(sbase + SM::kS, kDK, kNV, kk);
-                        tc::mma_f16(tmem + kTmU, desc_kmajor(sbase + SM::kSlot + I::kW, kChunk, kk), bdesc, idNeg,
-                                    true);
-                        tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + SM::kSlot + I::kQg, kChunk, kk), bdesc, idO,
-                                    kk > 0);
-                    }
-                    tc::mma_commit(&bar_m3);
-                }
-                if (!role_wait(&bar_m3, ph_m3, leader, kBarChain, kChainThreads, &abort_flag)) break;
-                ph_m3 ^= 1u;
-                // part 1 of the image has been read: start loading the next chunk's part 1
-                if (leader && c + 1 < nchunks &&
-                    tc::mbar_test_wait_cluster(&pub[(c + 1) % CL], ((c + 1) / CL) & 1)) {
-                    tc::fence_async_global();
-                    issue_part1(c + 1);
-                    pre1 = true;
-                }
-                // U~ -> fp16 B operand; a value outside the fp16 range sends the chunk to the exact path
-                {
-                    const int r = warp * 16 + lane;
-#pragma unroll
-                    for (int c16 = 0; c16 < kNV / 16; ++c16) {
-                        float u16[16];
-                        tc::tmem_ld16(tmem + tl + kTmU + c16 * 16, u16);
-                        tc::tmem_ld_wait();
-                        if (lane < 16) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) bad |= !(fabsf(u16[i]) <= 65000.f);
-                            *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16, kChunk, kNV)) =
-                                pack8_h(u16);
-                            *reinterpret_cast<uint4 *>(sm + SM::kUt + tile_chunk(r, 2 * c16 + 1, kChunk, kNV)) =
-                                pack8_h(u16 + 8);
-                        }
-                    }
-                    tc::fence_async_smem();
-                    tc::tc_fence_before();
-                }
-                bad = tc::named_sync_or(kBarChain, kChainThreads, bad);
-                if (!role_wait(&full2, c & 1, leader, kBarChain, kChainThreads, &abort_flag)) break;
-                part2_done = true;
-                if (leader) tc::mbar_arrive_cluster(tc::mapa(tc::smem_u32(&consumed), prod));
-                if (!bad) {
-                    // ---- M4: O += P U~,  Sn = Kd^T U~ ----
-                    if (leader) {
-                        constexpr uint32_t idO = tc::make_idesc(64, kNV, tc::kF16, false, true);
-                        constexpr uint32_t idS = tc::make_idesc(128, kNV, tc::kF16, true, true);
-#pragma unroll
-                        for (int kk = 0; kk < kChunk / 16; ++kk) {
-                            const uint64_t bdesc = desc_mnmajor(sbase + SM::kUt, kChunk, kNV, kk);
-                            tc::mma_f16(tmem + kTmO, desc_kmajor(sbase + SM::kSlot + I::kP, kChunk, kk), bdesc, idO,
-                                        true);
-                            tc::mma_f16(tmem + kTmSn, desc_mnmajor(sbase + SM::kSlot + I::kKd, kChunk, kDK, kk),
-                                        bdesc, idS, kk > 0);
-                        }
-                        tc::mma_commit(&bar_m4);
-                    }
-                    if (!role_wait(&bar_m4, ph_m4, leader, kBarChain, kChainThreads, &abort_flag)) break;
-                    ph_m4 ^= 1u;
-                    if (leader && pre1) {
-                        issue_part2(c + 1);
-                        pre2 = true;
-                    }
-                    // ---- epilogue: output rows, state update ----
-                    const int r = warp * 16 + lane;
-                    float o[kNV], sn[kNV];
-#pragma unroll
-                    for (int c16 = 0; c16 < kNV / 16; ++c16) {
-                        float x16[16];
-                        tc::tmem_ld16(tmem + tl + kTmSn + c16 * 16, x16);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) sn[c16 * 16 + i] = x16[i];
-                        tc::tmem_ld16(tmem + tl + kTmO + c16 * 16, x16);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) o[c16 * 16 + i] = x16[i];
-                    }
-                    bool obad = false;
-                    if (lane < 16)
-#pragma unroll
-                        for (int i = 0; i < kNV; ++i) obad |= !(fabsf(o[i]) <= 3.0e38f);
-                    tc::tc_fence_before();
-                    bad = tc::named_sync_or(kBarChain, kChainThreads, obad);
-                    if (!bad) {
-#pragma unroll
-                        for (int j = 0; j < kNV; ++j) S[j] = fmaf(gam, S[j], sn[j]);
-                        write_state_operand();
-                        if (lane < 16 && r < L) {
-                            TO *dst = out + ((tok0 + r) * H + h) * DV + vcol0;
-#pragma unroll
-                            for (int c16 = 0; c16 < kNV / 16; ++c16) store16<TO>(dst + c16 * 16, &o[c16 * 16]);
-                        }
-                        tc::named_sync(kBarChain, kChainThreads);
-                        continue;
-                    }
-                }
-            }
-            // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
-            if (!part2_done) {
-                if (!role_wait(&full2, c & 1, leader, kBarChain, kChainThreads, &abort_flag)) break;
-                if (leader) tc::mbar_arrive_cluster(tc::mapa(tc::smem_u32(&consumed), prod));
-            }
-            exact_chunk(tok0, L);
-            tc::tc_fence_before();
-            tc::named_sync(kBarChain, kChainThreads);
-        }
-        if (final_state && abort_flag == 0) {
-#pragma unroll
-            for (int j = 0; j < kNV; ++j) final_state[state_base + j] = S[j];
-        }
-    } else {
-        // ===================================== prep role ======================================
-        const int tp = tid - kChainThreads;      // 0..255
-        const bool leader = tp == 0;
-        const int cg = tp & 15, tg = tp >> 4;    // 8 channels [8cg, 8cg+8), 4 tokens [4tg, 4tg+4)
-        uint8_t *img = sm + SM::kImg;
-        uint4 rg[4], rk[4], rq[4];
-        float rb = 0.f;
-        auto load_raw = [&](int c) {
-            const int64_t tok0 = t0 + (int64_t)c * kChunk;
-            const int L = static_cast<int>((t1 - tok0) < kChunk ? (t1 - tok0) : kChunk);
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const int r = tg * 4 + rr;
-                if (r < L) {
-                    const int64_t off = ((tok0 + r) * H + h) * kDK + cg * 8;
-                    rg[rr] = *reinterpret_cast<const uint4 *>(log_alpha + off);
-                    rk[rr] = *reinterpret_cast<const uint4 *>(k + off);
-                    rq[rr] = *reinterpret_cast<const uint4 *>(q + off);
-                } else {
-                    rg[rr] = rk[rr] = rq[rr] = make_uint4(0, 0, 0, 0);
-                }
-            }
-            rb = (tp < kChunk && tp < L) ? __bfloat162float(beta[(tok0 + tp) * H + h]) : 0.f;
-        };
-        // store the finished image and announce it to every chain of the cluster
-        auto publish = [&](int c) -> bool {
-            bool ok = true;
-            if (leader) {
-                if (c >= CL) ok = tc::mbar_wait_cluster(&consumed, (c / CL - 1) & 1, &abort_flag);
-                if (ok) {
-                    tc::bulk_store_and_wait(ws_cluster + (size_t)rank * I::kStride, img, I::kBytes);
-                    tc::fence_async_global();
-                    for (int r = 0; r < CL; ++r) tc::mbar_arrive_cluster(tc::mapa(tc::smem_u32(&pub[rank]), r));
-                }
-            }
-            return !tc::named_sync_or(kBarPrep, kPrepThreads, !ok);
-        };
-        uint32_t ph_m1 = 0, ph_m2 = 0;
-        constexpr int ld = SM::kLd;
-        float *sA = reinterpret_cast<float *>(sm + SM::kA32);
-        float *sT = reinterpret_cast<float *>(sm + SM::kT32);
-        float *sX = reinterpret_cast<float *>(sm + SM::kX32);
-        int *img_flag = reinterpret_cast<int *>(img + I::kFlag);
-        float *img_gamma = reinterpret_cast<float *>(img + I::kGamma);
-        if (rank < nchunks) load_raw(rank);
-        for (int c = rank; c < nchunks; c += CL) {
-            // ---- decays (fp32 scan over the chunk, per channel) ----
-            float G[4][8];
-            {
-                float run[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) run[i] = 0.f;
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    float g8[8];
-                    unpack8(rg[rr], g8);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        run[i] += g8[i];
-                        G[rr][i] = run[i];
-                    }
-                }
-                // lanes 16-31 hold the odd token group of the warp's pair: add the even one's total
-                const int w4 = warp - 4;
-                float pair_tot[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float lower = __shfl_up_sync(0xffffffffu, run[i], 16);
-                    const float add = (lane >= 16) ? lower : 0.f;
-#pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) G[rr][i] += add;
-                    pair_tot[i] = run[i] + add;  // lanes 16-31: total of the warp's 8 tokens
-                }
-                if (lane >= 16) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) sTot[w4 * kDK + cg * 8 + i] = pair_tot[i];
-                }
-                if (tp < kChunk) sBeta[tp] = rb;
-                tc::named_sync(kBarPrep, kPrepThreads);
-                float off[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) off[i] = 0.f;
-                for (int pw = 0; pw < w4; ++pw)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) off[i] += sTot[pw * kDK + cg * 8 + i];
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) G[rr][i] += off[i];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (tg == 0) sG0[cg * 8 + i] = G[0][i];
-                    if (tg == 7) sGref[cg * 8 + i] = G[3][i];
-                    if (tg == 15) sGlast[cg * 8 + i] = G[3][i];
-                }
-            }
-            tc::named_sync(kBarPrep, kPrepThreads);
-            bool bad = false;
-            if (tp < kDK) {
-                const float g0 = sG0[tp], gr = sGref[tp], gl = sGlast[tp];
-                bad = !((g0 - gr <= kRangeLimit) && (gr - gl <= kRangeLimit));
-            }
-            if (tc::named_sync_or(kBarPrep, kPrepThreads, bad)) {
-                // decays too fast for the rebased products: every chain evaluates it exactly
-                if (c + CL < nchunks) load_raw(c + CL);
-                if (leader) *img_flag = 1;
-                tc::fence_async_smem();
-                tc::named_sync(kBarPrep, kPrepThreads);
-                if (!publish(c)) break;
-                continue;
-            }
-
-            // ---- rebased and decayed operands ----
-            {
-                float gref[8], erefabs[8], elast[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    gref[i] = sGref[cg * 8 + i];
-                    erefabs[i] = fast_exp(gref[i]);                       // exp(Gref)
-                    elast[i] = fast_exp(sGlast[cg * 8 + i] - gref[i]);   // exp(Glast - Gref)
-                }
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    const int r = tg * 4 + rr;
-                    float kf[8], qf[8];
-                    unpack8(rk[rr], kf);
-                    unpack8(rq[rr], qf);
-                    float kr[8], qr[8], kn[8], kg[8], qg[8], kd[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float dg = G[rr][i] - gref[i];
-                        const float e1 = fast_exp(dg), e2 = fast_exp(-dg);
-                        kr[i] = kf[i] * e1;
-                        qr[i] = qf[i] * e1;
-                        kn[i] = kf[i] * e2;
-                        kg[i] = kr[i] * erefabs[i];
-                        qg[i] = qr[i] * erefabs[i];
-                        kd[i] = kn[i] * elast[i];
-                    }
-                    const uint32_t off = tile_chunk(r, cg, kChunk, kDK);
-                    uint4 hi, lo;
-                    *reinterpret_cast<uint4 *>(sm + SM::kKr + off) = pack8_bf16(kr);
-                    split8_bf16(qr, hi, lo);
-                    *reinterpret_cast<uint4 *>(sm + SM::kQrHi + off) = hi;
-                    *reinterpret_cast<uint4 *>(sm + SM::kQrLo + off) = lo;
-                    split8_bf16(kn, hi, lo);
-                    *reinterpret_cast<uint4 *>(sm + SM::kKnHi + off) = hi;
-                    *reinterpret_cast<uint4 *>(sm + SM::kKnLo + off) = lo;
-                    *reinterpret_cast<uint4 *>(sm + SM::kKg + off) = pack8_h(kg);
-                    *reinterpret_cast<uint4 *>(img + I::kQg + off) = pack8_h(qg);
-                    *reinterpret_cast<uint4 *>(img + I::kKd + off) = pack8_h(kd);
-                }
-            }
-            // the raw registers are consumed: fetch this CTA's next chunk
-            if (c + CL < nchunks) load_raw(c + CL);
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_sync(kBarPrep, kPrepThreads);
-
-            // ---- M1: A_raw = Kr Kn^T,  P_raw = Qr Kn^T (two-term split); one commit, since the
-            //          UT scratch below reuses the operands of both ----
-            if (leader) {
-                tc::tc_fence_after();
-                constexpr uint32_t id = tc::make_idesc(64, 64, tc::kBF16, false, false);
-#pragma unroll
-                for (int kk = 0; kk < kDK / 16; ++kk) {
-                    const uint64_t bhi = desc_kmajor(sbase + SM::kKnHi, kChunk, kk);
-                    const uint64_t blo = desc_kmajor(sbase + SM::kKnLo, kChunk, kk);
-                    const uint64_t qhi = desc_kmajor(sbase + SM::kQrHi, kChunk, kk);
-                    tc::mma_f16(tmem + kTmA, desc_kmajor(sbase + SM::kKr, kChunk, kk), bhi, id, kk > 0);
-                    tc::mma_f16(tmem + kTmP, qhi, bhi, id, kk > 0);
-                    tc::mma_f16(tmem + kTmP, qhi, blo, id, true);
-                    tc::mma_f16(tmem + kTmP, desc_kmajor(sbase + SM::kQrLo, kChunk, kk), bhi, id, true);
-                }
-                tc::mma_commit(&bar_m1);
-            }
-            if (!role_wait(&bar_m1, ph_m1, leader, kBarPrep, kPrepThreads, &abort_flag)) break;
-            ph_m1 ^= 1u;
-
-            // ---- A (fp32, beta-scaled, strict lower) and tril(P) (fp16, into the image) ----
-            {
-                const int r = (warp & 3) * 16 + lane;
-                if (warp < 8) {
-                    const float br = (lane < 16) ? sBeta[r] : 0.f;
-#pragma unroll
-                    for (int c16 = 0; c16 < 4; ++c16) {
-                        float x16[16];
-                        tc::tmem_ld16(tmem + tl + kTmA + c16 * 16, x16);
-                        tc::tmem_ld_wait();
-                        if (lane < 16) {
-#pragma unroll
-                            for (int i = 0; i < 16; i += 4)
-                                *reinterpret_cast<float4 *>(&sA[r * ld + c16 * 16 + i]) =
-                                    make_float4((c16 * 16 + i < r) ? br * x16[i] : 0.f,
-                                                (c16 * 16 + i + 1 < r) ? br * x16[i + 1] : 0.f,
-                                                (c16 * 16 + i + 2 < r) ? br * x16[i + 2] : 0.f,
-                                                (c16 * 16 + i + 3 < r) ? br * x16[i + 3] : 0.f);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int c16 = 0; c16 < 4; ++c16) {
-                        float x16[16];
-                        tc::tmem_ld16(tmem + tl + kTmP + c16 * 16, x16);
-                        tc::tmem_ld_wait();
-                        if (lane < 16) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x16[i] = (c16 * 16 + i <= r) ? x16[i] : 0.f;
-                            *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, 2 * c16, kChunk, kChunk)) =
-                                pack8_h(x16);
-                            *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, 2 * c16 + 1, kChunk, kChunk)) =
-                                pack8_h(x16 + 8);
-                        }
-                    }
-                }
-            }
-            tc::tc_fence_before();
-            tc::named_sync(kBarPrep, kPrepThreads);
-
-            // ---- UT transform T = (I + A)^{-1} ----
-            // (a) 16x16 diagonal blocks: thread (bb, cc) solves column cc of (I + A_bb) x = e_cc by
-            //     forward substitution; the zeros above the diagonal are written too.
-            if (tp < 64) {
-                const int bb = tp >> 4, cc = tp & 15;
-                const float *arow = sA + (16 * bb) * ld + 16 * bb;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                    for (int s2 = 0; s2 < 15; ++s2)
-                        if (s2 < r) {
-                            const float term = arow[r * ld + s2] * ((s2 >= cc) ? x[s2] : 0.f);
-                            if (s2 & 1) acc1 += term; else acc0 += term;
-                        }
-                    x[r] = (r == cc) ? 1.f : ((r > cc) ? -(acc0 + acc1) : 0.f);
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) sT[(16 * bb + r) * ld + 16 * bb + cc] = x[r];
-            }
-            tc::named_sync(kBarPrep, kPrepThreads);
-            // (b) off-diagonal blocks by distance d = i - j: T_ij = -T_ii sum_{j<=m<i} A_im T_mj.
-            //     The 4 - d blocks of one distance are independent; 256 threads = one 16x16 block.
-#pragma unroll
-            for (int d = 1; d < 4; ++d) {
-                const int r = tp >> 4, cc = tp & 15;
-#pragma unroll
-                for (int blk = 0; blk < 4 - d; ++blk) {
-                    const int j = blk, i = blk + d;
-                    const float *arow = sA + (16 * i + r) * ld + 16 * j;
-                    const float *tcol = sT + (16 * j) * ld + 16 * j + cc;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int m = 0; m < 16 * d; m += 4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
-                        acc[0] = fmaf(a4.x, tcol[(m + 0) * ld], acc[0]);
-                        acc[1] = fmaf(a4.y, tcol[(m + 1) * ld], acc[1]);
-                        acc[2] = fmaf(a4.z, tcol[(m + 2) * ld], acc[2]);
-                        acc[3] = fmaf(a4.w, tcol[(m + 3) * ld], acc[3]);
-                    }
-                    sX[blk * 256 + r * 16 + cc] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                }
-                tc::named_sync(kBarPrep, kPrepThreads);
-#pragma unroll
-                for (int blk = 0; blk < 4 - d; ++blk) {
-                    const int j = blk, i = blk + d;
-                    const float *drow = sT + (16 * i + r) * ld + 16 * i;  // row r of T_ii (zero above the diagonal)
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int m = 0; m < 16; m += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
-                        acc[0] = fmaf(t4.x, sX[blk * 256 + (m + 0) * 16 + cc], acc[0]);
-                        acc[1] = fmaf(t4.y, sX[blk * 256 + (m + 1) * 16 + cc], acc[1]);
-                        acc[2] = fmaf(t4.z, sX[blk * 256 + (m + 2) * 16 + cc], acc[2]);
-                        acc[3] = fmaf(t4.w, sX[blk * 256 + (m + 3) * 16 + cc], acc[3]);
-                    }
-                    sT[(16 * i + r) * ld + 16 * j + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-                }
-                tc::named_sync(kBarPrep, kPrepThreads);
-            }
-            // T diag(beta) -> fp16 A operand [64 x 64] in the image: 2 chunks of 8 per thread; the
-            // strictly upper blocks of sT are never written, so the mask j*8 + i <= r is applied here
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = tp * 2 + e, r = idx >> 3, j = idx & 7;
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? sT[r * ld + j * 8 + i] * sBeta[j * 8 + i] : 0.f;
-                *reinterpret_cast<uint4 *>(img + I::kTb + tile_chunk(r, j, kChunk, kChunk)) = pack8_h(f);
-            }
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_sync(kBarPrep, kPrepThreads);
-
-            // ---- M2: W = (T b) Kg ----
-            if (leader) {
-                tc::tc_fence_after();
-                constexpr uint32_t idW = tc::make_idesc(64, kDK, tc::kF16, false, true);
-#pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk)
-                    tc::mma_f16(tmem + kTmW, desc_kmajor(sbase + SM::kImg + I::kTb, kChunk, kk),
-                                desc_mnmajor(sbase + SM::kKg, kChunk, kDK, kk), idW, kk > 0);
-                tc::mma_commit(&bar_m2);
-            }
-            if (!role_wait(&bar_m2, ph_m2, leader, kBarPrep, kPrepThreads, &abort_flag)) break;
-            ph_m2 ^= 1u;
-
-            // ---- W -> fp16 A operand [64 x 128] in the image; gamma; flag ----
-            {
-                const int w4 = warp - 4;
-                const int half = w4 >> 2;            // columns [64 half, 64 half + 64)
-                const int r = (warp & 3) * 16 + lane;
-#pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    float w16[16];
-                    tc::tmem_ld16(tmem + tl + kTmW + half * 64 + c16 * 16, w16);
-                    tc::tmem_ld_wait();
-                    if (lane < 16) {
-                        const int j = half * 8 + 2 * c16;
-                        *reinterpret_cast<uint4 *>(img + I::kW + tile_chunk(r, j, kChunk, kDK)) = pack8_h(w16);
-                        *reinterpret_cast<uint4 *>(img + I::kW + tile_chunk(r, j + 1, kChunk, kDK)) =
-                            pack8_h(w16 + 8);
-                    }
-                }
-            }
-            if (tp < kDK) img_gamma[tp] = fast_exp(sGlast[tp]);
-            if (leader) *img_flag = 0;
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::named_sync(kBarPrep, kPrepThreads);
-            if (!publish(c)) break;
-        }
-    }
+    ChunkCtx cx;
+    cx.n = n;
+    cx.h = h;
+    cx.H = H;
+    cx.t0 = t0;
+    cx.t1 = t1;
+    cx.nchunks = static_cast<int>((t1 - t0 + kChunk - 1) / kChunk);
+    cx.sm = sm;
+    cx.sbase = tc::smem_u32(sm);
+    cx.tmem = tmem_base_sh;
+    cx.ws_pair = workspace + (size_t)pair * kNP * 2 * Img<DV>::kStride;
+    cx.abort_flag = &abort_flag;
+    if (rank == 0)
+        chain_role<DV, TO>(cx, bars, maps, q, k, v, log_alpha, beta, init_state, out, final_state);
+    else
+        prep_role<DV>(cx, bars, rank - 1, maps, beta);
 
     tc::tc_fence_before();
     __syncthreads();
     tc::cluster_sync();  // no CTA leaves while a peer may still signal its barriers
-    if (warp == 0) tc::tmem_dealloc(tmem, kTmCols);
+    if (warp == 0) tc::tmem_dealloc(cx.tmem, ncols);
 }
 
-// Bytes of global workspace kda_chunk_fwd needs on the tensor-core path: one
-// chunk image per (sequence, head, value slice).
+// Bytes of global workspace kda_chunk_fwd needs on the tensor-core path: two chunk
+// image regions per (sequence, head) and prep CTA.
 inline size_t chunk_tc_workspace_bytes(int64_t pairs, int DV) {
-    return static_cast<size_t>(pairs) * (DV / kNV) * ChunkImage::kStride;
+    return static_cast<size_t>(pairs) * kNP * 2 * (DV == 64 ? Img<64>::kStride : Img<128>::kStride);
 }
 
-template <int CL, typename TO>
-cudaError_t launch_chunk_tc_cl(const void *q, const void *k, const void *v, const void *la, const void *beta,
-                               const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Map of a [tokens][H][d] tensor (bf16 or fp32) with boxes of 64 tokens x `box0` channels of one head.
+inline bool encode_row_map(CUtensorMap *m, const void *base, int d, int H, int64_t tokens, int box0 = 0,
+                           CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int esize = 2) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(H) * d * esize};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0 ? box0 : d), 1, kChunk};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DV, typename TO>
+cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, const void *la, const void *beta,
+                               const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H,
                                void *out, float *final_state, void *workspace, cudaStream_t stream) {
-    auto kern = kda_chunk_tc_kernel<CL, TO>;
-    const int smem = ChunkSmem::kBytes;
+    auto kern = kda_chunk_tc_kernel<DV, TO>;
+    const int smem = chunk_smem_bytes<DV>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int N = cu ? num_seqs : B;
+    RowMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    const int64_t tokens = (int64_t)B * T;
+    if (tokens > 0) {   // with no tokens no chunk is loaded and the maps stay unused
+        if (!encode_row_map(&maps.g, la, kDK, H, tokens) || !encode_row_map(&maps.k, k, kDK, H, tokens) ||
+            !encode_row_map(&maps.q, q, kDK, H, tokens) || !encode_row_map(&maps.v, v, DV, H, tokens) ||
+            !encode_row_map(&maps.o, out, DV, H, tokens, 64,
+                            sizeof(TO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            static_cast<int>(sizeof(TO))))
+            return cudaErrorInvalidValue;
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.x = kCL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(N) * H * CL);
+    cfg.gridDim = dim3(static_cast<unsigned>(N) * H * kCL);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
+    return cudaLaunchKernelEx(&cfg, kern, maps, static_cast<const __nv_bfloat16 *>(q),
                               static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
                               static_cast<const __nv_bfloat16 *>(la), static_cast<const __nv_bfloat16 *>(beta),
-                              init_state, cu, num_seqs, T, H, DV, static_cast<TO *>(out), final_state,
+                              init_state, cu, num_seqs, T, H, static_cast<TO *>(out), final_state,
                               static_cast<uint8_t *>(workspace));
 }
 
@@ -924,10 +1215,10 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
                             const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
                             void *out, float *final_state, void *workspace, cudaStream_t stream) {
     if (DV == 64)
-        return launch_chunk_tc_cl<2, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, DV, out, final_state,
-                                         workspace, stream);
-    return launch_chunk_tc_cl<4, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, DV, out, final_state,
-                                     workspace, stream);
+        return launch_chunk_tc_dv<64, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
+                                          workspace, stream);
+    return launch_chunk_tc_dv<128, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
+                                       workspace, stream);
 }
 
 }  // namespace kda

@@ -103,10 +103,11 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
 
 /*
  * Workspace kda_chunk_fwd needs, in bytes, for N sequences (B, or num_seqs with
- * cu_seqlens) of H heads: on the tensor-core path, one 65 KB chunk image per
- * (sequence, head, 32-column value slice), through which the CTAs of one head
- * hand each other the per-chunk operands (see kda_chunk_fwd); 0 on the fp32
- * path.  Pure host computation, never fails for valid sizes.
+ * cu_seqlens) of H heads: on the tensor-core path, six chunk images (73 KB each
+ * at d_v = 128, 65 KB at d_v = 64) per (sequence, head), through which the
+ * CTAs that prepare the chunk operands hand them to the CTA that runs the
+ * state recurrence (two regions per preparing CTA); 0 on the fp32 path.  Pure
+ * host computation, never fails for valid sizes.
  */
 kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v,
                                         kda_dtype dtype, size_t *bytes);
@@ -156,8 +157,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
  * d_v in {64, 128}.  It allocates nothing (no cudaMalloc, no library
  * allocator).  KDA_ERR_UNSUPPORTED if the problem needs more than
  * KDA_STATIC_WS_BYTES of handoff buffer, i.e. more than
- * KDA_STATIC_WS_BYTES / (65 KB * d_v / 32) (sequence, head) pairs: 63 at
- * d_v = 128, 126 at d_v = 64.
+ * KDA_STATIC_WS_BYTES / kda_chunk_fwd_workspace_size(1, 1, ...) (sequence,
+ * head) pairs: 37 at d_v = 128, 42 at d_v = 64.
  *
  * The first call on a device looks up that device's copy of the array (with
  * the device current), so make that first call before any stream capture.

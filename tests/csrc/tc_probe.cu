@@ -92,6 +92,81 @@ __global__ void __launch_bounds__(128) probe_kernel(const __nv_bfloat16 *A, cons
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// A operand in TMEM: thread m writes row m of A (K bf16, two per 32-bit column) with tcgen05.st,
+// B [N][K] (K-major) in shared memory; D = A * B^T read back as above.  M = 128.
+template <int N, int K>
+__global__ void __launch_bounds__(128) probe_tmem_a_kernel(const __nv_bfloat16 *A, const __nv_bfloat16 *B, float *D) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sB = smem;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tbase;
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x, warp = tid / 32;
+    constexpr int M = 128;
+    for (int i = tid; i < N * K; i += 128) {
+        int n = i / K, k = i % K;
+        *reinterpret_cast<__nv_bfloat16 *>(sB + tile_off(n, k, N, K)) = B[i];
+    }
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        abort_flag = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(&tbase, 512);
+        tmem_relinquish();
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tbase;
+    constexpr uint32_t kAcol = 256;   // A operand columns [256, 256 + K/2)
+    {
+        const uint32_t *arow = reinterpret_cast<const uint32_t *>(A + tid * K);  // row m = tid
+        for (int c0 = 0; c0 < K / 2; c0 += 16) {
+            uint32_t u[16];
+            for (int j = 0; j < 16; ++j) u[j] = arow[c0 + j];
+            tmem_st16(tmem + tmem_lane_base(warp) + kAcol + c0, u);
+        }
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        constexpr uint32_t idesc = make_idesc_bf16(M, N, false, false);
+        for (int kk = 0; kk < K / 16; ++kk) {
+            uint64_t bd = make_sdesc(smem_u32(sB) + (kk / 4) * (N * 128) + (kk % 4) * 32, 16, 1024, kSwz128);
+            mma_f16_ta(tmem, tmem + kAcol + kk * 8, bd, idesc, kk > 0);
+        }
+        mma_commit(&bar);
+    }
+    __syncwarp();
+    mbar_wait(&bar, 0, &abort_flag);
+    tc_fence_after();
+    const int row = warp * 32 + (tid % 32);
+    for (int c0 = 0; c0 < N; c0 += 16) {
+        float r[16];
+        tmem_ld16(tmem + tmem_lane_base(warp) + c0, r);
+        tmem_ld_wait();
+        for (int j = 0; j < 16; ++j) D[row * N + c0 + j] = r[j];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int N, int K>
+static int launch_tmem_a(const void *A, const void *B, void *D) {
+    size_t smem = N * K * 2 + 1024;
+    auto kern = probe_tmem_a_kernel<N, K>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return 1;
+    kern<<<1, 128, smem>>>((const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, (float *)D);
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
 template <int M, int N, int K, bool A_MN, bool B_MN>
 static int launch(const void *A, const void *B, void *D) {
     size_t smem = ((M * K * 2 + 1023) / 1024) * 1024 + N * K * 2 + 1024;
@@ -112,6 +187,8 @@ extern "C" int tc_probe_run(int case_id, const void *A, const void *B, void *D) 
         case 5: return launch<128, 32, 64, true, true>(A, B, D);     // NV = 32, SW64 B
         case 6: return launch<128, 128, 64, true, true>(A, B, D);    // NV = 128
         case 7: return launch<64, 128, 128, false, true>(A, B, D);   // NV = 128
+        case 8: return launch_tmem_a<64, 64>(A, B, D);               // A in TMEM, K-major B
+        case 9: return launch_tmem_a<128, 128>(A, B, D);
         default: return 3;
     }
 }

@@ -15,7 +15,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 # case id -> (M, N, K, A is MN-major, B is MN-major)
 CASES = {0: (64, 64, 128, False, False), 1: (64, 128, 64, False, True), 2: (128, 64, 64, True, True),
          3: (64, 64, 128, False, True), 4: (64, 32, 128, False, True), 5: (128, 32, 64, True, True),
-         6: (128, 128, 64, True, True), 7: (64, 128, 128, False, True)}
+         6: (128, 128, 64, True, True), 7: (64, 128, 128, False, True),
+         # A operand in TMEM (written with tcgen05.st), B K-major in shared memory
+         8: (128, 64, 64, False, False), 9: (128, 128, 128, False, False)}
 
 
 @pytest.fixture(scope="module")

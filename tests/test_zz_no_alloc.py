@@ -70,6 +70,6 @@ def test_two_calls_match_kda_chunk_fwd(cuda_lib):
 
 def test_refuses_problems_beyond_the_fixed_buffer(cuda_lib):
     fn = _static_ws(cuda_lib)
-    x = _case(T=64, H=70, dv=128, seed=13)   # 70 (sequence, head) pairs > 63 at d_v = 128
+    x = _case(T=64, H=70, dv=128, seed=13)   # 70 (sequence, head) pairs > 37 at d_v = 128
     st, _, _ = _call(fn, x)
     assert st == _lib.KDA_ERR_UNSUPPORTED
