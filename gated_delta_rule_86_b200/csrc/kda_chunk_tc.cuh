@@ -81,8 +81,9 @@ constexpr float kRangeLimit = 40.f;
 
 constexpr int kNP = 3;                // prep CTAs per cluster
 constexpr int kCL = kNP + 1;          // cluster: chain CTA (rank 0) + prep CTAs
-constexpr int kThreads = 384;         // 12 warps in every CTA of the cluster
-constexpr int kRoleThreads = 256;     // warps 0-7 run the role; warp 8 moves images
+constexpr int kRoleWarps = 16;                        // warps 0-15 run the role
+constexpr int kRoleThreads = kRoleWarps * 32;
+constexpr int kThreads = kRoleThreads + 64;           // + two helper warps that move data
 constexpr uint32_t kBarRole = 1, kBarU = 2, kBarOut = 3;  // named barriers: warps 0-7, U~ warps, output warps
 
 // ---- chunk image in the global workspace (fp16 tiles in their shared-memory layouts) ----------
@@ -111,10 +112,10 @@ template <int DV> struct ChainSmem {
     static constexpr int kFlag = kKd + (I::kFlag - I::kKd);
     static constexpr int kTailBytes = I::kBytes - I::kKd;
     static constexpr int kSlotBytes = (kKd + kTailBytes + 1023) / 1024 * 1024;
-    // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel half, k . q
+    // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel quarter, k . q
     static constexpr int kRedPk = 2 * kSlotBytes;
-    static constexpr int kRedPq = kRedPk + 2 * 128 * 4;
-    static constexpr int kRedKq = kRedPq + 2 * 128 * 4;
+    static constexpr int kRedPq = kRedPk + 4 * 128 * 4;
+    static constexpr int kRedKq = kRedPq + 4 * 128 * 4;
     // output staging of a full chunk: DV / 64 blocks of [64 tokens x 64 values] (fp32 or bf16),
     // written by a TMA tensor store per block
     static constexpr int kOut = (kRedKq + 16 + 1023) / 1024 * 1024;
@@ -153,8 +154,8 @@ template <int DV> struct PrepSmem {
     static constexpr int kTd32 = kX32 + 3 * 16 * 20 * 4;         // [4][16][20] diagonal blocks of T
     static_assert(kTd32 + 4 * 16 * 20 * 4 <= kKgV && kRawV + kChunk * DV * 2 <= kKgV, "A/P operand area");
     // scan scratch inside the K exp(G) | V operand (dead from [W | U] to the next rebase)
-    static constexpr int kTot = kKgV;                            // [8][128] per-warp totals
-    static constexpr int kPre = kTot + 8 * kDK * 4;              // [8][128] per-warp prefixes
+    static constexpr int kTot = kKgV;                            // [16][128] per-warp totals
+    static constexpr int kPre = kTot + 16 * kDK * 4;             // [16][128] per-warp prefixes
 };
 
 template <int DV> constexpr int chunk_smem_bytes() {
@@ -306,15 +307,16 @@ struct ChunkBars {
     int chain_ok;   // the chain leader's last MMA wait succeeded (read after a barrier)
 };
 
-// ================================== prep role (cluster ranks 1..kNP) ==================================
-// Producer p prepares chunks c = p, p + kNP, ... with warps 0-7.  Its k-th chunk is written straight
-// from registers into global region (p, k % 2) of the workspace, then announced to the chain CTA.
 // Tensor maps of the token tensors: [tokens][H][d] bf16, one box = 64 tokens x d channels of one
 // head; and of the output [tokens][H][d_v] (fp32 or bf16), one box = 64 tokens x 64 values.
 struct RowMaps {
     CUtensorMap g, k, q, v, o;
 };
 
+// ================================== prep role (cluster ranks 1..kNP) ==================================
+// Producer p prepares chunks c = p, p + kNP, ... with warps 0-15.  Lane 0 of warp 16 stores each
+// finished image to one of the producer's two global regions and announces it; lane 0 of warp 17
+// loads the raw input tiles of the next chunk.
 template <int DV>
 __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, int p, const RowMaps &maps,
                                           const __nv_bfloat16 *beta) {
@@ -325,10 +327,10 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     const uint32_t sbase = cx.sbase, tmem = cx.tmem;
     const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
     volatile int *abort_flag = cx.abort_flag;
-    if (warp == 8) {
-        // ---- publisher: staged image -> the chunk's global region (one bulk store), then announce the
-        //      region to the chain CTA ----
+    if (warp == kRoleWarps) {
         if (lane == 0) {
+            // ---- publisher: staged image -> the chunk's global region (one bulk store), then announce
+            //      the region to the chain CTA ----
             int kl = 0;
             for (int c = p; c < nchunks; c += kNP, ++kl) {
                 const int reg = kl & 1;
@@ -345,39 +347,37 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         }
         return;
     }
-    if (warp == 9) {
-        // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next chunk
-        //      (TMA; rows past the tensor end read as zero, rows past the sequence end are masked by the
-        //      readers), into the A/P operand area once the previous chunk's UT scratch is dead ----
-        int kl = 0, issued = -1;
-        for (int c = p; c < nchunks; c += kNP, ++kl) {
-            bool ok = true;
-            if (lane == 0 && kl >= 1) ok = tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-            const int64_t tok0 = cx.tok0(c);
-            if (lane == 0) {
+    if (warp == kRoleWarps + 1) {
+        if (lane == 0) {
+            // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next
+            //      chunk (TMA; rows past the tensor end read as zero, rows past the sequence end are
+            //      masked by the readers), into the A/P operand area once the previous chunk's UT
+            //      scratch is dead ----
+            int kl = 0, issued = -1;
+            for (int c = p; c < nchunks; c += kNP, ++kl) {
+                if (kl >= 1 && !tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag)) break;
+                const int t = static_cast<int>(cx.tok0(c));
                 tc::mbar_arrive_expect_tx(&bars.raw_full, SM::kRawBytes);
-                const int t = static_cast<int>(tok0);
                 tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
                 tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
                 tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
                 tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
+                issued = kl;
             }
-            issued = kl;
-        }
-        // no copy may still be in flight when the CTA leaves
-        if (lane == 0 && issued >= 0) {
-            int never = 0;
-            tc::mbar_wait(&bars.raw_full, issued & 1, &never);
+            // no copy may still be in flight when the CTA leaves
+            if (issued >= 0) {
+                int never = 0;
+                tc::mbar_wait(&bars.raw_full, issued & 1, &never);
+            }
         }
         return;
     }
-    if (warp > 9) return;
 
+    // ---- compute warps 0-15 ----
     const int tp = tid;
     const bool leader = tp == 0;
-    const int cg = tp & 15, tg = tp >> 4;   // channels [8cg, 8cg+8), tokens [4tg, 4tg+4)
-    const int sp = warp & 3, half = warp >> 2;
+    const int cg = tp & 15, tg = tp >> 4;   // channels [8cg, 8cg+8), tokens 2tg, 2tg + 1
+    const int sp = warp & 3, q4 = warp >> 2;
     const uint32_t tl = tc::tmem_lane_base(warp);
     float *sBeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *sG0 = reinterpret_cast<float *>(sm + SM::kG0);
@@ -424,14 +424,14 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         // the raw inputs of this chunk are in shared memory
         if (!role_wait(&bars.raw_full, kl & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
         // ---- decays: fp32 scan over the chunk, per channel ----
-        float G[4][8];
+        float G[2][8];
         {
             float run[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) run[i] = 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const int r = tg * 4 + rr;
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = tg * 2 + rr;
                 float g8[8];
                 const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
                                         : make_uint4(0, 0, 0, 0);
@@ -442,14 +442,14 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
                     G[rr][i] = run[i];
                 }
             }
-            // lanes 16-31 hold the odd token group of the warp's pair: add the even one's total
+            // lanes 16-31 hold the later token pair of the warp's four tokens: add the earlier total
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float lower = __shfl_up_sync(0xffffffffu, run[i], 16);
                 const float add = (lane >= 16) ? lower : 0.f;
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) G[rr][i] += add;
-                if (lane >= 16) sTot[warp * kDK + cg * 8 + i] = run[i] + add;   // the warp's 8 tokens
+                for (int rr = 0; rr < 2; ++rr) G[rr][i] += add;
+                if (lane >= 16) sTot[warp * kDK + cg * 8 + i] = run[i] + add;   // the warp's 4 tokens
             }
             if (tg == 0) {
 #pragma unroll
@@ -458,15 +458,15 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             if (tp < kChunk) sBeta[tp] = rb;
         }
         tc::named_sync(kBarRole, kRoleThreads);
-        // per channel: exclusive prefix over the 8 warps, G after tokens 31 and 63, range check
+        // per channel: exclusive prefix over the 16 warps, G after tokens 31 and 63, range check
         bool bad = false;
         if (tp < kDK) {
             float run = 0.f, gref = 0.f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
+            for (int w = 0; w < kRoleWarps; ++w) {
                 sPre[w * kDK + tp] = run;
                 run += sTot[w * kDK + tp];
-                if (w == 3) gref = run;
+                if (w == 7) gref = run;
             }
             sGref[tp] = gref;
             sGlast[tp] = run;
@@ -487,7 +487,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
 #pragma unroll
             for (int i = 0; i < 8; ++i) off[i] = sPre[warp * kDK + cg * 8 + i];
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
+            for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) G[rr][i] += off[i];
         }
@@ -498,10 +498,10 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             break;
         // ---- rebased and decayed operands; Q exp(G) and Kd into the staged image ----
         bool ovf = false;   // an fp16 operand or image value out of range
-        uint4 rk[4], rq[4], rv[4];
+        uint4 rk[2], rq[2], rv[2];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int r = tg * 4 + rr;
+        for (int rr = 0; rr < 2; ++rr) {
+            const int r = tg * 2 + rr;
             const bool in = r < L;
             rk[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawK + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
             rq[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawQ + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
@@ -519,8 +519,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
             const uint32_t okq = SM::kKQ + (cg >> 3) * SM::kKQBlk;
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const int r = tg * 4 + rr;
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = tg * 2 + rr;
                 float kf[8], qf[8];
                 unpack8(rk[rr], kf);
                 unpack8(rq[rr], qf);
@@ -581,57 +581,49 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         if (!role_wait(&bars.m_ap, ph_ap, leader, kBarRole, kRoleThreads, abort_flag)) break;
         ph_ap ^= 1u;
 
-        // ---- A (fp32, beta-scaled, strict lower) and tril(P) (fp16 A operand) ----
+        // ---- A (fp32, beta-scaled, strict lower) and tril(P) (fp16, into the image): warp (sp, q4)
+        //      reads accumulator rows 32 sp + lane, columns 16 q4 + [0, 16) ----
         {
-            const int m = sp * 32 + lane;   // accumulator row
-            const int c0 = half * 32;       // columns [c0, c0 + 32)
+            const int m = sp * 32 + lane;
+            const int cb = q4 * 16;
+            float x16[16];
+            tc::tmem_ld16(tmem + tl + kTmA + cb, x16);
             if (sp < 2) {
+                tc::tmem_ld_wait();
                 const int r = m;
                 const float br = sBeta[r];
 #pragma unroll
-                for (int c16 = 0; c16 < 2; ++c16) {
-                    float x16[16];
-                    tc::tmem_ld16(tmem + tl + kTmA + c0 + c16 * 16, x16);
-                    tc::tmem_ld_wait();
-                    const int cb = c0 + c16 * 16;
-#pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4 *>(&sA[r * ld + cb + i]) =
-                            make_float4((cb + i < r) ? br * x16[i] : 0.f, (cb + i + 1 < r) ? br * x16[i + 1] : 0.f,
-                                        (cb + i + 2 < r) ? br * x16[i + 2] : 0.f,
-                                        (cb + i + 3 < r) ? br * x16[i + 3] : 0.f);
-                }
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4 *>(&sA[r * ld + cb + i]) =
+                        make_float4((cb + i < r) ? br * x16[i] : 0.f, (cb + i + 1 < r) ? br * x16[i + 1] : 0.f,
+                                    (cb + i + 2 < r) ? br * x16[i + 2] : 0.f,
+                                    (cb + i + 3 < r) ? br * x16[i + 3] : 0.f);
             } else {
+                float y16[16];
+                tc::tmem_ld16(tmem + tl + kTmP2 + cb, y16);
+                tc::tmem_ld_wait();
                 const int r = m - 64;
 #pragma unroll
-                for (int c16 = 0; c16 < 2; ++c16) {
-                    float x16[16], y16[16];
-                    tc::tmem_ld16(tmem + tl + kTmA + c0 + c16 * 16, x16);
-                    tc::tmem_ld16(tmem + tl + kTmP2 + c0 + c16 * 16, y16);
-                    tc::tmem_ld_wait();
-                    const int cb = c0 + c16 * 16;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) x16[i] = (cb + i <= r) ? x16[i] + y16[i] : 0.f;
-                    *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8, kChunk)) = pack8_h(x16);
-                    *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8 + 1, kChunk)) = pack8_h(x16 + 8);
-                }
+                for (int i = 0; i < 16; ++i) x16[i] = (cb + i <= r) ? x16[i] + y16[i] : 0.f;
+                *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8, kChunk)) = pack8_h(x16);
+                *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8 + 1, kChunk)) = pack8_h(x16 + 8);
             }
         }
         tc::tc_fence_before();
         tc::named_sync(kBarRole, kRoleThreads);
 
-        // ---- UT transform T = (I + A)^{-1} ----
-        // (a) 16x16 diagonal blocks: four threads (p = tp % 4) solve column cc of (I + A_bb) x = e_cc by
-        //     right-looking substitution: thread p keeps rows r = p + 4 k in registers, the owner of
-        //     row s finalises x_s and shuffles it to the other three, which update their later rows.
-        //     The zeros above the diagonal are written too.
+        // ---- UT transform T = (I + A)^{-1}, stored transposed (sT row c = column c of T) ----
+        // (a) 16x16 diagonal blocks: eight threads (pp = tp % 8) solve column cc of (I + A_bb) x = e_cc
+        //     by right-looking substitution: thread pp keeps rows pp and pp + 8 in registers, the
+        //     owner of row s finalises x_s and shuffles it to the others, which update their later
+        //     rows.  The zeros above the diagonal are written too.
         {
-            const int col = tp >> 2, pp = tp & 3;
+            const int col = tp >> 3, pp = tp & 7;
             const int bb = col >> 4, cc = col & 15;
-            float a[4][16], part[4], x[4];
+            float a[2][16], part[2], x[2];
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-                const float *arow = sA + (16 * bb + pp + 4 * kq) * ld + 16 * bb;
+            for (int kq = 0; kq < 2; ++kq) {
+                const float *arow = sA + (16 * bb + pp + 8 * kq) * ld + 16 * bb;
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4) {
                     const float4 v4 = *reinterpret_cast<const float4 *>(arow + 4 * s4);
@@ -644,70 +636,70 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
 #pragma unroll
             for (int s2 = 0; s2 < 16; ++s2) {
-                float xs = (s2 == cc) ? 1.f : ((s2 < cc) ? 0.f : -part[s2 >> 2]);
-                xs = __shfl_sync(0xffffffffu, xs, (lane & ~3) | (s2 & 3));
-                if (pp == (s2 & 3)) x[s2 >> 2] = xs;
+                float xs = (s2 == cc) ? 1.f : ((s2 < cc) ? 0.f : -part[s2 >> 3]);
+                xs = __shfl_sync(0xffffffffu, xs, (lane & ~7) | (s2 & 7));
+                if (pp == (s2 & 7)) x[s2 >> 3] = xs;
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq)
-                    if (pp + 4 * kq > s2) part[kq] = fmaf(a[kq][s2], xs, part[kq]);
+                for (int kq = 0; kq < 2; ++kq)
+                    if (pp + 8 * kq > s2) part[kq] = fmaf(a[kq][s2], xs, part[kq]);
             }
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-                sT[(16 * bb + cc) * ld + 16 * bb + pp + 4 * kq] = x[kq];   // T^T
-                sTd[(bb * 16 + pp + 4 * kq) * 20 + cc] = x[kq];            // T_bb, row-major
+            for (int kq = 0; kq < 2; ++kq) {
+                sT[(16 * bb + cc) * ld + 16 * bb + pp + 8 * kq] = x[kq];   // T^T
+                sTd[(bb * 16 + pp + 8 * kq) * 20 + cc] = x[kq];            // T_bb, row-major
             }
         }
         tc::named_sync(kBarRole, kRoleThreads);
         // (b) off-diagonal blocks by distance d = i - j: T_ij = -T_ii sum_{j<=m<i} A_im T_mj.
-        //     The 4 - d blocks of one distance are independent; 256 threads = one 16x16 block.  With T
-        //     stored transposed, both factors of every dot product are contiguous (float4 reads).
-        {
-            const int r = tp >> 4, cc = tp & 15;
+        //     The 4 - d blocks of one distance are independent: entry e = blk * 256 + r * 16 + cc,
+        //     threads take e = tp and tp + 512.  With T stored transposed, both factors of every dot
+        //     product are contiguous (float4 reads).
 #pragma unroll 1
-            for (int d = 1; d < 4; ++d) {
+        for (int d = 1; d < 4; ++d) {
+            const int ne = (4 - d) * 256;
 #pragma unroll 1
-                for (int blk = 0; blk < 4 - d; ++blk) {
-                    const int j = blk, i = blk + d;
-                    const float *arow = sA + (16 * i + r) * ld + 16 * j;     // A[16i + r][16j + m]
-                    const float *tcol = sT + (16 * j + cc) * ld + 16 * j;    // T[16j + m][16j + cc]
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int e = tp; e < ne; e += kRoleThreads) {
+                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int j = blk, i = blk + d;
+                const float *arow = sA + (16 * i + r) * ld + 16 * j;     // A[16i + r][16j + m]
+                const float *tcol = sT + (16 * j + cc) * ld + 16 * j;    // T[16j + m][16j + cc]
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-                    for (int m = 0; m < 16 * d; m += 4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
-                        const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m);
-                        acc[0] = fmaf(a4.x, t4.x, acc[0]);
-                        acc[1] = fmaf(a4.y, t4.y, acc[1]);
-                        acc[2] = fmaf(a4.z, t4.z, acc[2]);
-                        acc[3] = fmaf(a4.w, t4.w, acc[3]);
-                    }
-                    sX[(blk * 16 + cc) * 20 + r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // X^T
+                for (int m = 0; m < 16 * d; m += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
+                    const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m);
+                    acc[0] = fmaf(a4.x, t4.x, acc[0]);
+                    acc[1] = fmaf(a4.y, t4.y, acc[1]);
+                    acc[2] = fmaf(a4.z, t4.z, acc[2]);
+                    acc[3] = fmaf(a4.w, t4.w, acc[3]);
                 }
-                tc::named_sync(kBarRole, kRoleThreads);
-#pragma unroll 1
-                for (int blk = 0; blk < 4 - d; ++blk) {
-                    const int j = blk, i = blk + d;
-                    const float *drow = sTd + (i * 16 + r) * 20;   // T_ii[r][m] (zero above the diagonal)
-                    const float *xcol = sX + (blk * 16 + cc) * 20;  // X[m][cc]
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int m = 0; m < 16; m += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
-                        const float4 x4 = *reinterpret_cast<const float4 *>(xcol + m);
-                        acc[0] = fmaf(t4.x, x4.x, acc[0]);
-                        acc[1] = fmaf(t4.y, x4.y, acc[1]);
-                        acc[2] = fmaf(t4.z, x4.z, acc[2]);
-                        acc[3] = fmaf(t4.w, x4.w, acc[3]);
-                    }
-                    sT[(16 * j + cc) * ld + 16 * i + r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));   // T^T
-                }
-                tc::named_sync(kBarRole, kRoleThreads);
+                sX[(blk * 16 + cc) * 20 + r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // X^T
             }
-        }
-        // T diag(beta) -> fp16 A operand [64 x 64]: 2 chunks of 8 per thread; the strictly upper
-        // blocks of sT are never written, so the mask j*8 + i <= r is applied here
+            tc::named_sync(kBarRole, kRoleThreads);
+#pragma unroll 1
+            for (int e = tp; e < ne; e += kRoleThreads) {
+                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int j = blk, i = blk + d;
+                const float *drow = sTd + (i * 16 + r) * 20;   // T_ii[r][m] (zero above the diagonal)
+                const float *xcol = sX + (blk * 16 + cc) * 20;  // X[m][cc]
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int idx = tp * 2 + e, r = idx >> 3, j = idx & 7;
+                for (int m = 0; m < 16; m += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
+                    const float4 x4 = *reinterpret_cast<const float4 *>(xcol + m);
+                    acc[0] = fmaf(t4.x, x4.x, acc[0]);
+                    acc[1] = fmaf(t4.y, x4.y, acc[1]);
+                    acc[2] = fmaf(t4.z, x4.z, acc[2]);
+                    acc[3] = fmaf(t4.w, x4.w, acc[3]);
+                }
+                sT[(16 * j + cc) * ld + 16 * i + r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));   // T^T
+            }
+            tc::named_sync(kBarRole, kRoleThreads);
+        }
+        // T diag(beta) -> fp16 A operand [64 x 64], one chunk of 8 per thread; the strictly upper
+        // blocks of T are never written, so the mask s <= r is applied here
+        {
+            const int r = tp >> 3, j = tp & 7;
             float f[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? sT[(j * 8 + i) * ld + r] * sBeta[j * 8 + i] : 0.f;
@@ -734,36 +726,34 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
             tc::mma_commit(&bars.m_wu);
         }
+        if (tp < kDK) reinterpret_cast<float *>(img + I::kGam)[tp] = fast_exp(sGlast[tp]);
         if (!role_wait(&bars.m_wu, ph_wu, leader, kBarRole, kRoleThreads, abort_flag)) break;
         ph_wu ^= 1u;
-        // -W (rows 0-63, duplicated in 64-127: warp (sp, half) takes rows 32 (sp % 2) + lane, columns
-        // 32 (2 (sp / 2) + half) + [0, 32)) and U^T (value row j = 32 sp + lane, tokens 32 half + [0, 32))
+        // -W (rows 0-63, duplicated in 64-127: warp (sp, q4) takes rows 32 (sp % 2) + lane, columns
+        // 64 (sp / 2) + 16 q4 + [0, 16)) and U^T (value row j = 32 sp + lane, tokens 16 q4 + [0, 16))
         // -> fp16 in the staged image
         {
-            float x[32];
-            const int r = (sp & 1) * 32 + lane, qd = (sp >> 1) * 2 + half;
-            tc::tmem_ld32(tmem + tl + kTmW + qd * 32, x);
+            float x[16];
+            const int r = (sp & 1) * 32 + lane, cw = (sp >> 1) * 64 + q4 * 16;
+            tc::tmem_ld16(tmem + tl + kTmW + cw, x);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
                 x[i] = -x[i];
                 ovf |= !(fabsf(x[i]) <= 65000.f);
             }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, 4 * qd + q4, kChunk)) = pack8_h(x + 8 * q4);
+            *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, cw / 8, kChunk)) = pack8_h(x);
+            *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, cw / 8 + 1, kChunk)) = pack8_h(x + 8);
             const int j = sp * 32 + lane;
-            tc::tmem_ld32(tmem + tl + kTmUT + half * 32, x);
+            tc::tmem_ld16(tmem + tl + kTmUT + q4 * 16, x);
             tc::tmem_ld_wait();
             if (j < DV) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ovf |= !(fabsf(x[i]) <= 65000.f);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(img + I::kUT + tile_chunk(j, 4 * half + q4, DV)) = pack8_h(x + 8 * q4);
+                for (int i = 0; i < 16; ++i) ovf |= !(fabsf(x[i]) <= 65000.f);
+                *reinterpret_cast<uint4 *>(img + I::kUT + tile_chunk(j, 2 * q4, DV)) = pack8_h(x);
+                *reinterpret_cast<uint4 *>(img + I::kUT + tile_chunk(j, 2 * q4 + 1, DV)) = pack8_h(x + 8);
             }
         }
-        if (tp < kDK) reinterpret_cast<float *>(img + I::kGam)[tp] = fast_exp(sGlast[tp]);
         tc::tc_fence_before();
         stage_done(ovf);
     }
@@ -776,8 +766,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
 //   D1^T = S^T [-W ; Qg]^T        (columns 0-63: (U~ - U)^T, columns 64-127: (Qg S)^T)
 //   D2^T = U~^T Kd                 (the state increment, transposed)
 //   D1^T[:, 64:128] += U~^T P^T    (so that columns 64-127 become O^T)
-// Warps 0-7 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
-// channels [64 (w / 4), 64 (w / 4) + 64) of S^T.  Lane 0 of warp 8 loads the chunk images.
+// Warps 0-15 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
+// channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Lane 0 of warp 16 loads the chunk images.
 template <int DV, typename TO>
 __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const RowMaps &maps,
                                            const __nv_bfloat16 *q,
@@ -792,9 +782,9 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
     volatile int *abort_flag = cx.abort_flag;
 
-    if (warp == 8) {
+    if (warp >= kRoleWarps) {
         // ---- loader: producer region -> image slot c % 2, once the slot is free and the image published ----
-        if (lane == 0) {
+        if (warp == kRoleWarps && lane == 0) {
             int last = -1;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
@@ -827,35 +817,32 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         }
         return;
     }
-    if (warp > 8) return;
 
     const bool leader = tid == 0;
-    const int sp = warp & 3, half = warp >> 2;
+    const int sp = warp & 3, qd = warp >> 2;
     const int j = sp * 32 + lane;            // value column (TMEM lane)
     const bool jv = j < DV;
-    const int c0 = half * 64;                // key channels [c0, c0 + 64)
+    const int c0 = qd * 32;                  // key channels [c0, c0 + 32)
     const uint32_t tl = tc::tmem_lane_base(warp);
     float *redPk = reinterpret_cast<float *>(sm + SM::kRedPk);
     float *redPq = reinterpret_cast<float *>(sm + SM::kRedPq);
     float *redKq = reinterpret_cast<float *>(sm + SM::kRedKq);
 
-    float S[64];  // fp32 master state: S^T[j][c0 + i]
+    float S[32];  // fp32 master state: S^T[j][c0 + i]
     const size_t state_base = ((size_t)cx.n * H + h) * kDK * DV + (size_t)c0 * DV + j;
 #pragma unroll
-    for (int i = 0; i < 64; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
-    // S^T -> fp16 A operand in TMEM (lane j, channels c0..c0+63 in 32 columns); returns whether some
+    for (int i = 0; i < 32; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
+    // S^T -> fp16 A operand in TMEM (lane j, channels c0..c0+31 in 16 columns); returns whether some
     // entry left the fp16 range
     auto write_state_operand = [&]() -> bool {
         bool big = false;
+        uint32_t u[16];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) big |= !(fabsf(S[i]) <= 65000.f);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            uint32_t u[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) u[i] = pack_h(S[32 * g + 2 * i], S[32 * g + 2 * i + 1]);
-            tc::tmem_st16(tmem + tl + kTmS + half * 32 + g * 16, u);
+        for (int i = 0; i < 16; ++i) {
+            big |= !(fabsf(S[2 * i]) <= 65000.f) || !(fabsf(S[2 * i + 1]) <= 65000.f);
+            u[i] = pack_h(S[2 * i], S[2 * i + 1]);
         }
+        tc::tmem_st16(tmem + tl + kTmS + qd * 16, u);
         tc::tmem_st_wait();
         return big;
     };
@@ -870,7 +857,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                                 *qr = q + trow * kDK + c0;
             float pk = 0.f, pq = 0.f, kq = 0.f;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int i = 0; i < 32; ++i) {
                 const float a = expf(__bfloat162float(gr[i])), kk = __bfloat162float(kr[i]),
                             qq = __bfloat162float(qr[i]);
                 S[i] *= a;
@@ -878,24 +865,24 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 pq = fmaf(S[i], qq, pq);
                 kq = fmaf(kk, qq, kq);
             }
-            redPk[half * 128 + j] = pk;
-            redPq[half * 128 + j] = pq;
-            if (sp == 0 && lane == 0) redKq[half] = kq;
+            redPk[qd * 128 + j] = pk;
+            redPq[qd * 128 + j] = pq;
+            if (sp == 0 && lane == 0) redKq[qd] = kq;
             tc::named_sync(kBarRole, kRoleThreads);
-            const float u = jv ? __bfloat162float(beta[trow]) *
-                                     (__bfloat162float(v[trow * DV + j]) - (redPk[j] + redPk[128 + j]))
-                               : 0.f;
-            if (half == 0 && jv)
-                out[trow * DV + j] = from_f32<TO>(fmaf(u, redKq[0] + redKq[1], redPq[j] + redPq[128 + j]));
+            const float skq = (redKq[0] + redKq[1]) + (redKq[2] + redKq[3]);
+            const float spk = (redPk[j] + redPk[128 + j]) + (redPk[256 + j] + redPk[384 + j]);
+            const float spq = (redPq[j] + redPq[128 + j]) + (redPq[256 + j] + redPq[384 + j]);
+            const float u = jv ? __bfloat162float(beta[trow]) * (__bfloat162float(v[trow * DV + j]) - spk) : 0.f;
+            if (qd == 0 && jv) out[trow * DV + j] = from_f32<TO>(fmaf(u, skq, spq));
 #pragma unroll
-            for (int i = 0; i < 64; ++i) S[i] = fmaf(__bfloat162float(kr[i]), u, S[i]);
+            for (int i = 0; i < 32; ++i) S[i] = fmaf(__bfloat162float(kr[i]), u, S[i]);
             tc::named_sync(kBarRole, kRoleThreads);
         }
         return write_state_operand();
     };
 
     // output of a tensor-path chunk: columns 64-127 of D1^T[b] hold O^T once [. ; P] U~ completed;
-    // thread (j, half) has tokens 32 half + [0, 32) of value column j.  A full chunk is staged in
+    // thread (j, qd) has tokens 16 qd + [0, 16) of value column j.  A full chunk is staged in
     // shared memory (a warp writes 32 consecutive values of one token: no bank conflicts) and written
     // by TMA tensor stores; a partial last chunk is stored directly.
     uint32_t ph_m3[2] = {0, 0};
@@ -904,8 +891,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         if (leader) tc::bulk_wait_read_all();   // the previous chunk's stores have read the staging
         if (!role_wait(&bars.mma3[bp], ph_m3[bp], leader, kBarRole, kRoleThreads, abort_flag)) return false;
         ph_m3[bp] ^= 1u;
-        float o[32];
-        tc::tmem_ld32(tmem + tl + kTmD1 + bp * 128 + 64 + half * 32, o);
+        float o[16];
+        tc::tmem_ld16(tmem + tl + kTmD1 + bp * 128 + 64 + qd * 16, o);
         tc::tmem_ld_wait();
         const int64_t tok0 = cx.tok0(cp);
         const int L = cx.len(cp);
@@ -913,7 +900,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             if (jv) {
                 TO *col = stage + (j >> 6) * (kChunk * 64) + (j & 63);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) col[(half * 32 + i) * 64] = from_f32<TO>(o[i]);
+                for (int i = 0; i < 16; ++i) col[(qd * 16 + i) * 64] = from_f32<TO>(o[i]);
             }
             tc::fence_async_smem();
             tc::named_sync(kBarRole, kRoleThreads);
@@ -925,8 +912,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             }
         } else if (jv) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = half * 32 + i;
+            for (int i = 0; i < 16; ++i) {
+                const int r = qd * 16 + i;
                 if (r < L) out[((tok0 + r) * H + h) * DV + j] = from_f32<TO>(o[i]);
             }
         }
@@ -959,31 +946,31 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         if (!flagged) {
             if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) break;
             ph1 ^= 1u;
-            // ---- U~^T = U^T + (-W S)^T (tokens 32 half + [0, 32)) -> fp16 A operand in TMEM ----
+            // ---- U~^T = U^T + (-W S)^T (tokens 16 qd + [0, 16)) -> fp16 A operand in TMEM ----
             bool mybad = force_exact;
             {
-                float x[32];
-                tc::tmem_ld32(tmem + tl + kTmD1 + b * 128 + half * 32, x);
+                float x[16];
+                tc::tmem_ld16(tmem + tl + kTmD1 + b * 128 + qd * 16, x);
                 tc::tmem_ld_wait();
-                uint32_t u[16];
+                uint32_t u[8];
                 if (jv) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
+                    for (int h2 = 0; h2 < 2; ++h2) {
                         float u8[8];
-                        unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 4 * half + q4, DV)),
+                        unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 2 * qd + h2, DV)),
                                   u8);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) x[8 * q4 + i] += u8[i];
+                        for (int i = 0; i < 8; ++i) x[8 * h2 + i] += u8[i];
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mybad |= !(fabsf(x[i]) <= 65000.f);
+                    for (int i = 0; i < 16; ++i) mybad |= !(fabsf(x[i]) <= 65000.f);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) u[i] = pack_h(x[2 * i], x[2 * i + 1]);
+                    for (int i = 0; i < 8; ++i) u[i] = pack_h(x[2 * i], x[2 * i + 1]);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) u[i] = 0u;
+                    for (int i = 0; i < 8; ++i) u[i] = 0u;
                 }
-                tc::tmem_st16(tmem + tl + kTmUt + half * 16, u);
+                tc::tmem_st8(tmem + tl + kTmUt + qd * 8, u);
                 tc::tmem_st_wait();
             }
             tc::tc_fence_before();
@@ -1009,19 +996,18 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             if (!bad) {
                 // ---- S^T = S^T Diag(gamma) + D2^T ----
                 const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
+                {
                     float d[32];
-                    tc::tmem_ld32(tmem + tl + kTmD2 + c0 + g * 32, d);
+                    tc::tmem_ld32(tmem + tl + kTmD2 + c0, d);
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int i4 = 0; i4 < 8; ++i4) {
-                        const float4 gg = gam4[g * 8 + i4];
-                        const int i = 32 * g + 4 * i4;
-                        S[i] = fmaf(gg.x, S[i], d[4 * i4]);
-                        S[i + 1] = fmaf(gg.y, S[i + 1], d[4 * i4 + 1]);
-                        S[i + 2] = fmaf(gg.z, S[i + 2], d[4 * i4 + 2]);
-                        S[i + 3] = fmaf(gg.w, S[i + 3], d[4 * i4 + 3]);
+                        const float4 gg = gam4[i4];
+                        const int i = 4 * i4;
+                        S[i] = fmaf(gg.x, S[i], d[i]);
+                        S[i + 1] = fmaf(gg.y, S[i + 1], d[i + 1]);
+                        S[i + 2] = fmaf(gg.z, S[i + 2], d[i + 2]);
+                        S[i + 3] = fmaf(gg.w, S[i + 3], d[i + 3]);
                     }
                 }
                 const bool big = write_state_operand();
@@ -1043,7 +1029,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     if (leader) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
     if (final_state && *abort_flag == 0 && jv) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) final_state[state_base + (size_t)i * DV] = S[i];
+        for (int i = 0; i < 32; ++i) final_state[state_base + (size_t)i * DV] = S[i];
     }
     if (leader) drain_mma(&bars.fin, 0);
 }
