@@ -37,8 +37,8 @@
 // Precision (fp32 accumulation in TMEM, fp32 master state in registers, fp32
 // decays and substitution, fp32 or bf16 output):
 //   * A and P need the rebased factors below, whose range exceeds fp16: they are
-//     bf16 operands, and P (which feeds the output directly) uses a two-term
-//     bf16 split of both operands (hi*hi + hi*lo + lo*hi), ~16-bit accuracy.
+//     one tf32 product (fp32 operands read with an 11-bit significand and the fp32
+//     exponent range), [Kr ; Qr] Kn^T; the UT transform then runs in fp32.
 //   * Every other product has operands bounded by the inputs and runs on fp16
 //     operands (11-bit significand, same tensor rate as bf16).  A value outside
 //     the fp16 range turns U~ or O non-finite; that is detected and the chunk is
@@ -83,8 +83,8 @@ constexpr int kNP = 3;                // prep CTAs per cluster
 constexpr int kCL = kNP + 1;          // cluster: chain CTA (rank 0) + prep CTAs
 constexpr int kRoleWarps = 16;                        // warps 0-15 run the role
 constexpr int kRoleThreads = kRoleWarps * 32;
-constexpr int kThreads = kRoleThreads + 64;           // + two helper warps that move data
-constexpr uint32_t kBarRole = 1, kBarU = 2, kBarOut = 3;  // named barriers: warps 0-7, U~ warps, output warps
+constexpr int kThreads = kRoleThreads + 128;          // + four helper warps that move data
+constexpr uint32_t kBarRole = 1, kBarOut = 2;          // named barriers: role warps, helper warps
 
 // ---- chunk image in the global workspace (fp16 tiles in their shared-memory layouts) ----------
 template <int DV> struct Img {
@@ -116,23 +116,25 @@ template <int DV> struct ChainSmem {
     static constexpr int kRedPk = 2 * kSlotBytes;
     static constexpr int kRedPq = kRedPk + 4 * 128 * 4;
     static constexpr int kRedKq = kRedPq + 4 * 128 * 4;
-    // output staging of a full chunk: DV / 64 blocks of [64 tokens x 64 values] (fp32 or bf16),
-    // written by a TMA tensor store per block
+    // output staging of a full chunk, double-buffered: DV / 64 blocks of [64 tokens x 64 values]
+    // (fp32 or bf16), written by a TMA tensor store per block
     static constexpr int kOut = (kRedKq + 16 + 1023) / 1024 * 1024;
-    static constexpr int kBytes = kOut + kChunk * DV * 4;
+    static constexpr int kOutBytes = kChunk * DV * 4;   // two buffers
+    static constexpr int kBytes = kOut + 2 * kOutBytes;
 };
 
 // ---- prep CTA shared memory -------------------------------------------------------------------
 template <int DV> struct PrepSmem {
     using I = Img<DV>;
     static constexpr int kTile = kChunk * kDK * 2;         // [64 x 128] 16-bit tile
-    // A operands of the A/P products, per 64-channel block b: [Kr_b | Qh_b | Ql_b]
-    // (8 KB each), so that [Kr ; Qh] and [Qh ; Ql] are 128-row operands
-    static constexpr int kKQBlk = 3 * kChunk * 128;
+    // fp32 (tf32) operands of the A/P product, K-major SW128 in 32-channel blocks of 128-byte rows:
+    // A = [Kr ; Qr] (per block b: rows 0-63 K exp(G - Gref), rows 64-127 Q exp(G - Gref); 16 KB),
+    // B = Kn = K exp(Gref - G) (per block: 64 rows, 8 KB)
+    static constexpr int kKQBlk = 2 * kChunk * 128;
+    static constexpr int kKnBlk = kChunk * 128;
     static constexpr int kKQ = 0;
-    static constexpr int kKh = 2 * kKQBlk;                 // K exp(Gref - G), hi  [64 x 128] (B)
-    static constexpr int kKl = kKh + kTile;                //                  lo
-    static constexpr int kKgV = kKl + kTile;               // [K exp(G) | V] [64 x 256], V zero past DV
+    static constexpr int kKn = 4 * kKQBlk;
+    static constexpr int kKgV = kKn + 4 * kKnBlk;          // [K exp(G) | V] [64 x 256], V zero past DV
     // [Tb | Tb]: the A operand of W (both row halves give the same rows, so all warps can read
     // them); the first Tb is also the B operand of U^T = V^T Tb^T
     static constexpr int kTbP = kKgV + kChunk * 2 * kDK * 2;
@@ -141,18 +143,20 @@ template <int DV> struct PrepSmem {
     static constexpr int kG0 = kBeta + kChunk * 4;               // fp32 [128] decay after token 0
     static constexpr int kGref = kG0 + kDK * 4;                  //            after token 31
     static constexpr int kGlast = kGref + kDK * 4;               //            after token 63
-    static constexpr int kBytes = kGlast + kDK * 4;
+    static constexpr int kEref = kGlast + kDK * 4;               // exp(Gref)
+    static constexpr int kElast = kEref + kDK * 4;               // exp(Glast - Gref)
+    static constexpr int kBytes = kElast + kDK * 4;
     // The A/P operand area also holds, in turn: the raw bf16 inputs of the chunk (bulk-loaded
     // rows of log_alpha, k, q, v; read into registers before the operands are written) and the
     // fp32 scratch of the UT transform (once the A/P products complete).
     static constexpr int kRawG = 0, kRawK = kChunk * 256, kRawQ = 2 * kChunk * 256, kRawV = 3 * kChunk * 256;
     static constexpr int kRawBytes = kChunk * (3 * kDK * 2 + DV * 2);   // one TMA box per tensor
-    static constexpr int kLd = 68;                               // row stride of A and T^T
+    static constexpr int kLd = 68;                               // row stride of A and T
     static constexpr int kA32 = 0;                               // A [64][68]
-    static constexpr int kT32 = kA32 + kChunk * kLd * 4;         // T^T [64][68] (row c = column c of T)
-    static constexpr int kX32 = kT32 + kChunk * kLd * 4;         // [3][16][20] block products, transposed
-    static constexpr int kTd32 = kX32 + 3 * 16 * 20 * 4;         // [4][16][20] diagonal blocks of T
-    static_assert(kTd32 + 4 * 16 * 20 * 4 <= kKgV && kRawV + kChunk * DV * 2 <= kKgV, "A/P operand area");
+    static constexpr int kT32 = kA32 + kChunk * kLd * 4;         // T [64][68]
+    static constexpr int kScr32 = kT32 + kChunk * kLd * 4;       // per-warp product tiles (warps 0-3)
+    static constexpr int kScrFloats = 16 * 24;                   // [16][24] or [32][8]
+    static_assert(kScr32 + 4 * kScrFloats * 4 <= kKgV && kRawV + kChunk * DV * 2 <= kKgV, "A/P operand area");
     // scan scratch inside the K exp(G) | V operand (dead from [W | U] to the next rebase)
     static constexpr int kTot = kKgV;                            // [16][128] per-warp totals
     static constexpr int kPre = kTot + 16 * kDK * 4;             // [16][128] per-warp prefixes
@@ -166,7 +170,7 @@ static_assert(chunk_smem_bytes<128>() <= 232448, "shared memory plan exceeds 227
 // TMEM columns (fp32 accumulators, M = 128 layout: row m -> lane m).
 // chain: D1^T double-buffered (0, 128), D2^T, the S^T operand (64 columns) and the U~^T operand (32)
 constexpr uint32_t kTmD1 = 0, kTmD2 = 256, kTmS = 384, kTmUt = 448, kTmChainCols = 512;
-constexpr uint32_t kTmA = 0, kTmP2 = 64, kTmW = 256, kTmUT = 384, kTmPrepCols = 512;  // prep
+constexpr uint32_t kTmA = 0, kTmW = 256, kTmUT = 384, kTmPrepCols = 512;  // prep
 
 // Descriptor of k-step `kk` (16 elements along K) of a K-major SW128 operand with `rows` rows.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int kk) {
@@ -212,22 +216,14 @@ __device__ __forceinline__ void unpack8_h(const uint4 &u, float *f) {
 __device__ __forceinline__ uint4 pack8_bf16(const float *f) {
     return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
 }
+// Finite fp32 -> nearest tf32 value (ties away from zero: add half a unit of the 10-bit significand,
+// then clear the 13 low bits), still as an fp32 bit pattern
+__device__ __forceinline__ float round_tf32(float x) {
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+}
 __device__ __forceinline__ uint4 pack8_h(const float *f) {
     return make_uint4(pack_h(f[0], f[1]), pack_h(f[2], f[3]), pack_h(f[4], f[5]), pack_h(f[6], f[7]));
 }
-// Two-term bf16 split x ~= hi + lo: hi is x truncated to bf16 (exact in fp32),
-// lo the bf16 rounding of the exact remainder; |x - hi - lo| <= 2^-15 |x|.
-__device__ __forceinline__ void split8_bf16(const float *f, uint4 &hi, uint4 &lo) {
-    float r[8];
-    uint32_t h[4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) r[i] = f[i] - __uint_as_float(__float_as_uint(f[i]) & 0xffff0000u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __byte_perm(__float_as_uint(f[2 * i]), __float_as_uint(f[2 * i + 1]), 0x7632);
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = pack8_bf16(r);
-}
-
 template <typename TO> __device__ __forceinline__ void store16(TO *dst, const float *f);
 template <> __device__ __forceinline__ void store16<float>(float *dst, const float *f) {
 #pragma unroll
@@ -301,6 +297,9 @@ struct ChunkCtx {
 struct ChunkBars {
     // chain: image slot full / free, MMA completions, producer publications (per producer region)
     uint64_t full[2], slot_free[2], mma1, mma2, mma3[2], pub[kNP][2];
+    // chain: chunk evaluation mode handed to the output warps, TMEM accumulator read by them
+    uint64_t outq[2], d1_free[2];
+    int outmode[2];   // 0: no MMAs issued, 1: MMAs issued but evaluated exactly, 2: tensor output
     // prep: MMA completions, global region consumed by the chain (per region)
     uint64_t m_ap, m_wu, consumed[2], staged, staging_free, raw_full, raw_free;
     uint64_t fin;
@@ -347,6 +346,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         }
         return;
     }
+    if (warp >= kRoleWarps + 2) return;   // warps 18, 19 serve the chain CTA only
     if (warp == kRoleWarps + 1) {
         if (lane == 0) {
             // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next
@@ -388,8 +388,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     constexpr int ld = SM::kLd;
     float *sA = reinterpret_cast<float *>(sm + SM::kA32);
     float *sT = reinterpret_cast<float *>(sm + SM::kT32);
-    float *sX = reinterpret_cast<float *>(sm + SM::kX32);
-    float *sTd = reinterpret_cast<float *>(sm + SM::kTd32);
+    float *sS = reinterpret_cast<float *>(sm + SM::kScr32);
 
     // beta of the next chunk, prefetched into registers (one value per thread of warps 0-1)
     float rb = 0.f;
@@ -470,6 +469,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
             sGref[tp] = gref;
             sGlast[tp] = run;
+            reinterpret_cast<float *>(sm + SM::kEref)[tp] = fast_exp(gref);
+            reinterpret_cast<float *>(sm + SM::kElast)[tp] = fast_exp(run - gref);
             bad = !((sG0[tp] - gref <= kRangeLimit) && (gref - run <= kRangeLimit));
         }
         if (tc::named_sync_or(kBarRole, kRoleThreads, bad)) {
@@ -510,20 +511,39 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         }
         tc::named_sync(kBarRole, kRoleThreads);   // the operands below overwrite the raw rows
         {
-            float gref[8], elast[8], erefabs[8];
+            // fp32 operand rows: channels 8 cg .. 8 cg + 7 are 16-byte chunks 2 (cg % 4) and 2 (cg % 4) + 1
+            // of 32-channel block cg / 4; lanes of odd blocks store the second chunk first, so that
+            // each group of eight lanes covers all eight chunk positions of a row (no bank conflicts)
+            const int c16 = 2 * (cg & 3);
+            const bool swap = (cg >> 2) & 1;
+            const uint32_t okq = SM::kKQ + (cg >> 2) * SM::kKQBlk, okn = SM::kKn + (cg >> 2) * SM::kKnBlk;
+            // values are rounded to tf32 here (to nearest): the tensor cores would otherwise drop the
+            // low mantissa bits, a bias that adds up coherently over the 128 channels of a product
+            auto st_f32x8 = [&](uint32_t base, int row, const float *f) {
+                float t[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                gref[i] = sGref[cg * 8 + i];
-                erefabs[i] = fast_exp(gref[i]);                       // exp(Gref)
-                elast[i] = fast_exp(sGlast[cg * 8 + i] - gref[i]);   // exp(Glast - Gref)
-            }
-            const uint32_t okq = SM::kKQ + (cg >> 3) * SM::kKQBlk;
+                for (int i = 0; i < 8; ++i) t[i] = round_tf32(f[i]);
+                const float4 lo = make_float4(t[0], t[1], t[2], t[3]), hi = make_float4(t[4], t[5], t[6], t[7]);
+                const uint32_t olo = base + tc::sw128(row, c16), ohi = base + tc::sw128(row, c16 + 1);
+                *reinterpret_cast<float4 *>(sm + (swap ? ohi : olo)) = swap ? hi : lo;
+                *reinterpret_cast<float4 *>(sm + (swap ? olo : ohi)) = swap ? lo : hi;
+            };
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = tg * 2 + rr;
                 float kf[8], qf[8];
                 unpack8(rk[rr], kf);
                 unpack8(rq[rr], qf);
+                // per-channel constants, re-read from shared memory for each token (fewer live registers)
+                float gref[8], eref[8], elast[8];
+                const float *sEref = reinterpret_cast<const float *>(sm + SM::kEref) + cg * 8;
+                const float *sElast = reinterpret_cast<const float *>(sm + SM::kElast) + cg * 8;
+#pragma unroll
+                for (int i4 = 0; i4 < 8; i4 += 4) {
+                    *reinterpret_cast<float4 *>(gref + i4) = *reinterpret_cast<const float4 *>(sGref + cg * 8 + i4);
+                    *reinterpret_cast<float4 *>(eref + i4) = *reinterpret_cast<const float4 *>(sEref + i4);
+                    *reinterpret_cast<float4 *>(elast + i4) = *reinterpret_cast<const float4 *>(sElast + i4);
+                }
                 float kr[8], qr[8], kn[8], kd[8], kg[8], qg[8], vf[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -533,8 +553,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
                     qr[i] = qf[i] * e1;
                     kn[i] = kf[i] * e2;
                     kd[i] = kn[i] * elast[i];
-                    kg[i] = kr[i] * erefabs[i];
-                    qg[i] = qr[i] * erefabs[i];
+                    kg[i] = kr[i] * eref[i];
+                    qg[i] = qr[i] * eref[i];
                 }
                 const uint32_t o128 = tile_chunk(r, cg, kChunk);   // [64 x 128] tiles
                 *reinterpret_cast<uint4 *>(sm + SM::kKgV + o128) = pack8_h(kg);
@@ -543,15 +563,9 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ovf |= !(fabsf(vf[i]) <= 65000.f);
                 *reinterpret_cast<uint4 *>(sm + SM::kKgV + tile_chunk(r, 16 + cg, kChunk)) = pack8_h(vf);
-                const uint32_t okr = okq + tc::sw128(r, cg & 7);   // [Kr | Qh | Ql] blocks
-                uint4 hi, lo;
-                *reinterpret_cast<uint4 *>(sm + okr) = pack8_bf16(kr);
-                split8_bf16(qr, hi, lo);
-                *reinterpret_cast<uint4 *>(sm + okr + 8192) = hi;
-                *reinterpret_cast<uint4 *>(sm + okr + 16384) = lo;
-                split8_bf16(kn, hi, lo);
-                *reinterpret_cast<uint4 *>(sm + SM::kKh + o128) = hi;
-                *reinterpret_cast<uint4 *>(sm + SM::kKl + o128) = lo;
+                st_f32x8(okq, r, kr);
+                st_f32x8(okq, 64 + r, qr);
+                st_f32x8(okn, r, kn);
                 *reinterpret_cast<uint4 *>(img + I::kKd + o128) = pack8_h(kd);
             }
         }
@@ -559,21 +573,17 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         tc::tc_fence_before();
         tc::named_sync(kBarRole, kRoleThreads);
 
-        // ---- A/P products: D_A = [Kr ; Qh] Kh^T (rows 0-63 A_raw, rows 64-127 Qh Kh^T),
-        //      D_P2 = [Kr ; Qh] Kl^T + [Qh ; Ql] Kh^T (rows 64-127 Qh Kl^T + Ql Kh^T) ----
+        // ---- A/P product (tf32): D = [Kr ; Qr] Kn^T: rows 0-63 A_raw, rows 64-127 P ----
         if (leader) {
             tc::tc_fence_after();
-            constexpr uint32_t id = tc::make_idesc(128, 64, tc::kBF16, false, false);
+            constexpr uint32_t id = tc::make_idesc(128, 64, tc::kTF32, false, false);
 #pragma unroll
-            for (int kk = 0; kk < kDK / 16; ++kk) {
-                const uint32_t a0 = sbase + SM::kKQ + (kk >> 2) * SM::kKQBlk + (kk & 3) * 32;
-                const uint64_t akq = tc::make_sdesc(a0, 16, 1024, tc::kSwz128);
-                const uint64_t aqq = tc::make_sdesc(a0 + 8192, 16, 1024, tc::kSwz128);
-                const uint64_t bh = desc_kmajor(sbase + SM::kKh, kChunk, kk);
-                const uint64_t bl = desc_kmajor(sbase + SM::kKl, kChunk, kk);
-                tc::mma_f16(tmem + kTmA, akq, bh, id, kk > 0);
-                tc::mma_f16(tmem + kTmP2, akq, bl, id, kk > 0);
-                tc::mma_f16(tmem + kTmP2, aqq, bh, id, true);
+            for (int kk = 0; kk < kDK / 8; ++kk) {
+                const uint64_t a = tc::make_sdesc(sbase + SM::kKQ + (kk >> 2) * SM::kKQBlk + (kk & 3) * 32, 16, 1024,
+                                                  tc::kSwz128);
+                const uint64_t bd = tc::make_sdesc(sbase + SM::kKn + (kk >> 2) * SM::kKnBlk + (kk & 3) * 32, 16, 1024,
+                                                   tc::kSwz128);
+                tc::mma_tf32(tmem + kTmA, a, bd, id, kk > 0);
             }
             tc::mma_commit(&bars.m_ap);
         }
@@ -599,12 +609,10 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
                                     (cb + i + 2 < r) ? br * x16[i + 2] : 0.f,
                                     (cb + i + 3 < r) ? br * x16[i + 3] : 0.f);
             } else {
-                float y16[16];
-                tc::tmem_ld16(tmem + tl + kTmP2 + cb, y16);
                 tc::tmem_ld_wait();
                 const int r = m - 64;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x16[i] = (cb + i <= r) ? x16[i] + y16[i] : 0.f;
+                for (int i = 0; i < 16; ++i) x16[i] = (cb + i <= r) ? x16[i] : 0.f;
                 *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8, kChunk)) = pack8_h(x16);
                 *reinterpret_cast<uint4 *>(img + I::kP + tile_chunk(r, cb / 8 + 1, kChunk)) = pack8_h(x16 + 8);
             }
@@ -612,7 +620,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         tc::tc_fence_before();
         tc::named_sync(kBarRole, kRoleThreads);
 
-        // ---- UT transform T = (I + A)^{-1}, stored transposed (sT row c = column c of T) ----
+        // ---- UT transform T = (I + A)^{-1} (row-major in sT; blocks above the diagonal never written) ----
         // (a) 16x16 diagonal blocks: eight threads (pp = tp % 8) solve column cc of (I + A_bb) x = e_cc
         //     by right-looking substitution: thread pp keeps rows pp and pp + 8 in registers, the
         //     owner of row s finalises x_s and shuffles it to the others, which update their later
@@ -645,54 +653,84 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
 #pragma unroll
             for (int kq = 0; kq < 2; ++kq) {
-                sT[(16 * bb + cc) * ld + 16 * bb + pp + 8 * kq] = x[kq];   // T^T
-                sTd[(bb * 16 + pp + 8 * kq) * 20 + cc] = x[kq];            // T_bb, row-major
+                sT[(16 * bb + pp + 8 * kq) * ld + 16 * bb + cc] = x[kq];
+                // the upper blocks (0, 1) and (2, 3) are zero: the block products below read them
+                if ((bb & 1) == 0) sT[(16 * bb + pp + 8 * kq) * ld + 16 * bb + 16 + cc] = 0.f;
             }
         }
         tc::named_sync(kBarRole, kRoleThreads);
-        // (b) off-diagonal blocks by distance d = i - j: T_ij = -T_ii sum_{j<=m<i} A_im T_mj.
-        //     The 4 - d blocks of one distance are independent: entry e = blk * 256 + r * 16 + cc,
-        //     threads take e = tp and tp + 512.  With T stored transposed, both factors of every dot
-        //     product are contiguous (float4 reads).
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            const int ne = (4 - d) * 256;
-#pragma unroll 1
-            for (int e = tp; e < ne; e += kRoleThreads) {
-                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int j = blk, i = blk + d;
-                const float *arow = sA + (16 * i + r) * ld + 16 * j;     // A[16i + r][16j + m]
-                const float *tcol = sT + (16 * j + cc) * ld + 16 * j;    // T[16j + m][16j + cc]
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-                for (int m = 0; m < 16 * d; m += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + m);
-                    const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m);
-                    acc[0] = fmaf(a4.x, t4.x, acc[0]);
-                    acc[1] = fmaf(a4.y, t4.y, acc[1]);
-                    acc[2] = fmaf(a4.z, t4.z, acc[2]);
-                    acc[3] = fmaf(a4.w, t4.w, acc[3]);
+        // (b) the blocks below the diagonal, as two levels of the 2x2 block inverse
+        //     [[Ta, 0], [Lba, Tb']]^{-1} = [[Ta, 0], [-Tb' Lba Ta, Tb']], fp32 on CUDA cores.
+        //     Level 1 (16-row blocks): T10 and T32; level 2 (32-row blocks): the lower-left 32x32
+        //     block.  Each product goes through the scratch tile X; a thread reads a row of the left
+        //     factor as float4 (shared by the 16 lanes of that row) and the right factor's values
+        //     for its own columns (consecutive over the lanes).
+        {
+            float *sXs = sS;   // level 1: [2][16][16];  level 2: [32][32]
+            {
+                const int blk = tp >> 8, r = (tp >> 4) & 15, n = tp & 15;
+                const int j = 2 * blk, i = j + 1;
+                const float *arow = sA + (16 * i + r) * ld + 16 * j;
+                float acc = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                    const float *tk = sT + (16 * j + 4 * k4) * ld + 16 * j + n;
+                    acc = fmaf(a4.x, tk[0], acc);
+                    acc = fmaf(a4.y, tk[ld], acc);
+                    acc = fmaf(a4.z, tk[2 * ld], acc);
+                    acc = fmaf(a4.w, tk[3 * ld], acc);
                 }
-                sX[(blk * 16 + cc) * 20 + r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);   // X^T
+                sXs[blk * 256 + r * 16 + n] = acc;                       // X = A_ij T_jj
+                tc::named_sync(kBarRole, kRoleThreads);
+                const float *trow = sT + (16 * i + r) * ld + 16 * i;
+                const float *xk = sXs + blk * 256 + n;
+                acc = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(trow + 4 * k4);
+                    acc = fmaf(t4.x, xk[(4 * k4) * 16], acc);
+                    acc = fmaf(t4.y, xk[(4 * k4 + 1) * 16], acc);
+                    acc = fmaf(t4.z, xk[(4 * k4 + 2) * 16], acc);
+                    acc = fmaf(t4.w, xk[(4 * k4 + 3) * 16], acc);
+                }
+                sT[(16 * i + r) * ld + 16 * j + n] = -acc;               // T_ij = -T_ii X
             }
             tc::named_sync(kBarRole, kRoleThreads);
-#pragma unroll 1
-            for (int e = tp; e < ne; e += kRoleThreads) {
-                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int j = blk, i = blk + d;
-                const float *drow = sTd + (i * 16 + r) * 20;   // T_ii[r][m] (zero above the diagonal)
-                const float *xcol = sX + (blk * 16 + cc) * 20;  // X[m][cc]
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                const int r = tp >> 4, n = 2 * (tp & 15);
+                const float *arow = sA + (32 + r) * ld;
+                float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; m += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4 *>(drow + m);
-                    const float4 x4 = *reinterpret_cast<const float4 *>(xcol + m);
-                    acc[0] = fmaf(t4.x, x4.x, acc[0]);
-                    acc[1] = fmaf(t4.y, x4.y, acc[1]);
-                    acc[2] = fmaf(t4.z, x4.z, acc[2]);
-                    acc[3] = fmaf(t4.w, x4.w, acc[3]);
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 t2 = *reinterpret_cast<const float2 *>(sT + (4 * k4 + e) * ld + n);
+                        y0 = fmaf(av[e], t2.x, y0);
+                        y1 = fmaf(av[e], t2.y, y1);
+                    }
                 }
-                sT[(16 * j + cc) * ld + 16 * i + r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));   // T^T
+                *reinterpret_cast<float2 *>(sXs + r * 32 + n) = make_float2(y0, y1);   // Y = Lba Ta
+                tc::named_sync(kBarRole, kRoleThreads);
+                const float *trow = sT + (32 + r) * ld + 32;
+                const int k4n = (r >> 4) * 4 + 4;   // Tb'[r][k] = 0 for k > r: whole 16-blocks skipped
+                y0 = 0.f;
+                y1 = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    if (k4 >= k4n) break;
+                    const float4 t4 = *reinterpret_cast<const float4 *>(trow + 4 * k4);
+                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x2 = *reinterpret_cast<const float2 *>(sXs + (4 * k4 + e) * 32 + n);
+                        y0 = fmaf(tv[e], x2.x, y0);
+                        y1 = fmaf(tv[e], x2.y, y1);
+                    }
+                }
+                *reinterpret_cast<float2 *>(sT + (32 + r) * ld + n) = make_float2(-y0, -y1);   // Tba = -Tb' Y
             }
             tc::named_sync(kBarRole, kRoleThreads);
         }
@@ -700,9 +738,12 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         // blocks of T are never written, so the mask s <= r is applied here
         {
             const int r = tp >> 3, j = tp & 7;
+            const float4 t0 = *reinterpret_cast<const float4 *>(sT + r * ld + 8 * j);
+            const float4 t1 = *reinterpret_cast<const float4 *>(sT + r * ld + 8 * j + 4);
+            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
             float f[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? sT[(j * 8 + i) * ld + r] * sBeta[j * 8 + i] : 0.f;
+            for (int i = 0; i < 8; ++i) f[i] = (j * 8 + i <= r) ? tv[i] * sBeta[j * 8 + i] : 0.f;
             const uint4 t8 = pack8_h(f);
             *reinterpret_cast<uint4 *>(sm + SM::kTbP + tile_chunk(r, j, kChunk)) = t8;
             *reinterpret_cast<uint4 *>(sm + SM::kTbP + 8192 + tile_chunk(r, j, kChunk)) = t8;
@@ -767,7 +808,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
 //   D2^T = U~^T Kd                 (the state increment, transposed)
 //   D1^T[:, 64:128] += U~^T P^T    (so that columns 64-127 become O^T)
 // Warps 0-15 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
-// channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Lane 0 of warp 16 loads the chunk images.
+// channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Warps 16-19 store the outputs; lane 0 of warp 16
+// also loads the chunk images.
 template <int DV, typename TO>
 __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const RowMaps &maps,
                                            const __nv_bfloat16 *q,
@@ -783,36 +825,121 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     volatile int *abort_flag = cx.abort_flag;
 
     if (warp >= kRoleWarps) {
-        // ---- loader: producer region -> image slot c % 2, once the slot is free and the image published ----
-        if (warp == kRoleWarps && lane == 0) {
-            int last = -1;
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                if (c >= 2) {
-                    if (!tc::mbar_wait(&bars.slot_free[s], ((c >> 1) - 1) & 1, abort_flag)) break;
-                    // chunk c - 2 has long been loaded: its producer may rewrite that region
-                    const int pc = c - 2;
-                    tc::mbar_arrive_cluster_relaxed(
-                        tc::mapa(tc::smem_u32(&bars.consumed[(pc / kNP) & 1]), 1 + pc % kNP));
-                }
-                const int p = c % kNP, kq = c / kNP, reg = kq & 1;
-                if (!tc::mbar_wait_cluster(&bars.pub[p][reg], (kq >> 1) & 1, abort_flag)) break;
-                tc::fence_async_global();
-                const uint8_t *src = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
-                uint8_t *slot = sm + s * SM::kSlotBytes;
-                uint64_t *fb = &bars.full[s];
-                tc::mbar_arrive_expect_tx(fb, I::kBytes);
-                tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
-                tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
-                tc::bulk_load(slot + SM::kA1 + 8192, src + I::kQt, 8192, fb);
-                tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
-                tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
-                tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
-                last = c;
+        // ---- output and image warps 16-19: warp 16 + w reads TMEM lanes 32 w .. 32 w + 31, i.e. value
+        //      columns j = 32 w + lane of O^T (columns 64-127 of D1^T[b]) once [. ; P] U~ completed,
+        //      and stages them for TMA tensor stores (double-buffered); lane 0 of warp 16 also moves
+        //      the chunk images from the producers' global regions into the two slots ----
+        const int jo = (warp & 3) * 32 + lane;
+        const bool jov = jo < DV;
+        const bool lead = warp == kRoleWarps && lane == 0;
+        const uint32_t tlo = tc::tmem_lane_base(warp);
+        constexpr uint32_t kOutThreads = kThreads - kRoleThreads;
+        int last_load = -1;
+        auto load_image = [&](int c) -> bool {   // lane 0 of warp 16
+            const int p = c % kNP, kq = c / kNP, reg = kq & 1;
+            if (!tc::mbar_wait_cluster(&bars.pub[p][reg], (kq >> 1) & 1, abort_flag)) return false;
+            tc::fence_async_global();
+            const uint8_t *src = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
+            uint8_t *slot = sm + (c & 1) * SM::kSlotBytes;
+            uint64_t *fb = &bars.full[c & 1];
+            tc::mbar_arrive_expect_tx(fb, I::kBytes);
+            tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
+            tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
+            tc::bulk_load(slot + SM::kA1 + 8192, src + I::kQt, 8192, fb);
+            tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
+            tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
+            tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
+            last_load = c;
+            return true;
+        };
+        if (lead)
+            for (int c = 0; c < 2 && c < nchunks; ++c)
+                if (!load_image(c)) break;
+        // a wait by lane 0 of warp 16, whose outcome all four warps share (they leave together)
+        auto out_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            bool ok = true;
+            if (lead) ok = tc::mbar_wait(bar, parity, abort_flag);
+            const bool failed = tc::named_sync_or(kBarOut, kOutThreads, !ok);
+            tc::tc_fence_after();
+            return !failed;
+        };
+        uint32_t ph_q[2] = {0, 0}, ph3[2] = {0, 0};
+        int nstore = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            // the state warps have chosen how chunk c is evaluated (outmode) ...
+            if (!out_wait(&bars.outq[b], ph_q[b])) break;
+            ph_q[b] ^= 1u;
+            const int mode = *reinterpret_cast<volatile int *>(&bars.outmode[b]);
+            // ... and, when its MMAs were issued, they have completed
+            if (mode >= 1) {
+                if (!out_wait(&bars.mma3[b], ph3[b])) break;
+                ph3[b] ^= 1u;
             }
-            // no copy may still be in flight when the CTA leaves
+            if (mode == 2) {
+                const int64_t tok0 = cx.tok0(c);
+                const int L = cx.len(c);
+                const bool full = L == kChunk;
+                TO *stage = reinterpret_cast<TO *>(sm + SM::kOut + (nstore & 1) * SM::kOutBytes);
+                if (full) {
+                    // the stores issued from this buffer two chunks ago have read it
+                    if (lead) tc::bulk_wait_read_1();
+                    tc::named_sync(kBarOut, kOutThreads);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
+                    float o[32];
+                    tc::tmem_ld32(tmem + tlo + kTmD1 + b * 128 + 64 + 32 * half, o);
+                    tc::tmem_ld_wait();
+                    if (half == 1) {
+                        // D1^T[b] may be overwritten by the MMAs of chunk c + 2
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
+                    }
+                    if (!jov) continue;
+                    if (full) {
+                        TO *col = stage + (jo >> 6) * (kChunk * 64) + (jo & 63) + 32 * half * 64;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) col[i * 64] = from_f32<TO>(o[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (32 * half + i < L) out[((tok0 + 32 * half + i) * H + h) * DV + jo] = from_f32<TO>(o[i]);
+                    }
+                }
+                if (full) {
+                    tc::fence_async_smem();
+                    tc::named_sync(kBarOut, kOutThreads);
+                    if (lead) {
+#pragma unroll
+                        for (int blk = 0; blk < DV / 64; ++blk)
+                            tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0), stage + blk * (kChunk * 64));
+                        tc::bulk_commit();
+                    }
+                    ++nstore;
+                }
+            } else {
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
+            }
+            // the image of chunk c + 2 goes into slot b once the state warps are done with chunk c;
+            // chunk c's own copy out of its producer region completed long ago: the region is free
+            bool lok = true;
+            if (lead && c + 2 < nchunks) {
+                int never = 0;
+                tc::mbar_wait(&bars.full[b], (c >> 1) & 1, &never);
+                tc::mbar_arrive_cluster_relaxed(tc::mapa(tc::smem_u32(&bars.consumed[(c / kNP) & 1]), 1 + c % kNP));
+                lok = tc::mbar_wait(&bars.slot_free[b], (c >> 1) & 1, abort_flag) && load_image(c + 2);
+            }
+            if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) break;
+        }
+        if (lead) {
+            tc::bulk_wait_all();   // every output store has completed before the CTA leaves
+            // no image copy may still be in flight either
             int never = 0;
-            for (int c = (last >= 1 ? last - 1 : 0); c <= last; ++c)
+            for (int c = (last_load >= 1 ? last_load - 1 : 0); c <= last_load; ++c)
                 tc::mbar_wait(&bars.full[c & 1], (c >> 1) & 1, &never);
         }
         return;
@@ -881,47 +1008,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         return write_state_operand();
     };
 
-    // output of a tensor-path chunk: columns 64-127 of D1^T[b] hold O^T once [. ; P] U~ completed;
-    // thread (j, qd) has tokens 16 qd + [0, 16) of value column j.  A full chunk is staged in
-    // shared memory (a warp writes 32 consecutive values of one token: no bank conflicts) and written
-    // by TMA tensor stores; a partial last chunk is stored directly.
-    uint32_t ph_m3[2] = {0, 0};
-    TO *const stage = reinterpret_cast<TO *>(sm + SM::kOut);
-    auto store_output = [&](int cp, int bp) -> bool {
-        if (leader) tc::bulk_wait_read_all();   // the previous chunk's stores have read the staging
-        if (!role_wait(&bars.mma3[bp], ph_m3[bp], leader, kBarRole, kRoleThreads, abort_flag)) return false;
-        ph_m3[bp] ^= 1u;
-        float o[16];
-        tc::tmem_ld16(tmem + tl + kTmD1 + bp * 128 + 64 + qd * 16, o);
-        tc::tmem_ld_wait();
-        const int64_t tok0 = cx.tok0(cp);
-        const int L = cx.len(cp);
-        if (L == kChunk) {
-            if (jv) {
-                TO *col = stage + (j >> 6) * (kChunk * 64) + (j & 63);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) col[(qd * 16 + i) * 64] = from_f32<TO>(o[i]);
-            }
-            tc::fence_async_smem();
-            tc::named_sync(kBarRole, kRoleThreads);
-            if (leader) {
-#pragma unroll
-                for (int blk = 0; blk < DV / 64; ++blk)
-                    tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0), stage + blk * (kChunk * 64));
-                tc::bulk_commit();
-            }
-        } else if (jv) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = qd * 16 + i;
-                if (r < L) out[((tok0 + r) * H + h) * DV + j] = from_f32<TO>(o[i]);
-            }
-        }
-        return true;
-    };
-
     uint32_t ph1 = 0, ph2 = 0;
-    bool prev_tensor = false;   // chunk c - 1 went through the tensor path: its output is pending
     for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, b = c & 1;
         const int64_t tok0 = cx.tok0(c);
@@ -930,19 +1017,24 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         const uint32_t sslot = sbase + s * SM::kSlotBytes;
         if (!role_wait(&bars.full[s], (c >> 1) & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
         const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
-        if (!flagged && leader) {
-            // ---- D1^T[b] = S^T [-W ; Qg]^T ----
-            constexpr uint32_t id1 = tc::make_idesc(128, 128, tc::kF16, false, false);
+        if (leader) {
+            // the output warps have read D1^T[b] of chunk c - 2
+            bool ok = c < 2 || tc::mbar_wait(&bars.d1_free[b], ((c >> 1) - 1) & 1, abort_flag);
+            if (ok && !flagged) {
+                tc::tc_fence_after();
+                // ---- D1^T[b] = S^T [-W ; Qg]^T ----
+                constexpr uint32_t id1 = tc::make_idesc(128, 128, tc::kF16, false, false);
 #pragma unroll
-            for (int kk = 0; kk < kDK / 16; ++kk)
-                tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8, desc_kmajor(sslot + SM::kA1, 128, kk),
-                               id1, kk > 0);
-            tc::mma_commit(&bars.mma1);
+                for (int kk = 0; kk < kDK / 16; ++kk)
+                    tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8,
+                                   desc_kmajor(sslot + SM::kA1, 128, kk), id1, kk > 0);
+                tc::mma_commit(&bars.mma1);
+            }
+            if (flagged) {
+                bars.outmode[b] = 0;   // no MMAs, no tensor output
+                tc::mbar_arrive(&bars.outq[b]);
+            }
         }
-        // the previous chunk's output, while D1^T[b] is computed; then its slot is free
-        if (prev_tensor && !store_output(c - 1, b ^ 1)) break;
-        if (c >= 1 && leader) tc::mbar_arrive(&bars.slot_free[s ^ 1]);
-        prev_tensor = false;
         if (!flagged) {
             if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) break;
             ph1 ^= 1u;
@@ -990,6 +1082,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     tc::mma_f16_ta(tmem + kTmD1 + b * 128 + 64, tmem + kTmUt + kk * 8,
                                    desc_kmajor(sslot + SM::kP, kChunk, kk), id3, true);
                 tc::mma_commit(&bars.mma3[b]);
+                bars.outmode[b] = bad ? 1 : 2;   // MMAs issued; O^T is the output unless evaluated exactly
+                tc::mbar_arrive(&bars.outq[b]);
             }
             if (!role_wait(&bars.mma2, ph2, leader, kBarRole, kRoleThreads, abort_flag)) break;
             ph2 ^= 1u;
@@ -1013,20 +1107,16 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 const bool big = write_state_operand();
                 tc::tc_fence_before();
                 force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
-                prev_tensor = true;
+                if (leader) tc::mbar_arrive(&bars.slot_free[s]);   // done with the slot
                 continue;
             }
-            // this chunk is evaluated exactly: its pending [. ; P] U~ must still complete
-            if (!role_wait(&bars.mma3[b], ph_m3[b], leader, kBarRole, kRoleThreads, abort_flag)) break;
-            ph_m3[b] ^= 1u;
         }
         // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
         const bool big = exact_chunk(tok0, L);
         tc::tc_fence_before();
         force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+        if (leader) tc::mbar_arrive(&bars.slot_free[s]);
     }
-    if (prev_tensor && nchunks > 0) store_output(nchunks - 1, (nchunks - 1) & 1);
-    if (leader) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
     if (final_state && *abort_flag == 0 && jv) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) final_state[state_base + (size_t)i * DV] = S[i];
@@ -1073,6 +1163,10 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __nv_bfloat16 *_
         tc::mbar_init(&bars.mma2, 1);
         tc::mbar_init(&bars.mma3[0], 1);
         tc::mbar_init(&bars.mma3[1], 1);
+        tc::mbar_init(&bars.outq[0], 1);
+        tc::mbar_init(&bars.outq[1], 1);
+        tc::mbar_init(&bars.d1_free[0], kThreads / 32 - kRoleWarps);
+        tc::mbar_init(&bars.d1_free[1], kThreads / 32 - kRoleWarps);
         for (int p = 0; p < kNP; ++p) {
             tc::mbar_init(&bars.pub[p][0], 1);
             tc::mbar_init(&bars.pub[p][1], 1);

@@ -303,10 +303,11 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_byte
     return d;
 }
 
-// Instruction descriptor for kind::f16 with an fp32 accumulator.  `fmt`
-// selects the operand type of both A and B (kF16 or kBF16: one tcgen05.mma
-// never mixes them); a_mn / b_mn select MN-major operands; neg_a negates A.
-enum OpFmt : uint32_t { kF16 = 0, kBF16 = 1 };
+// Instruction descriptor for kind::f16 or kind::tf32 with an fp32 accumulator.
+// `fmt` selects the operand type of both A and B (kF16 or kBF16 for kind::f16:
+// one tcgen05.mma never mixes them; kTF32 for kind::tf32); a_mn / b_mn select
+// MN-major operands; neg_a negates A.
+enum OpFmt : uint32_t { kF16 = 0, kBF16 = 1, kTF32 = 2 };
 __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t fmt, bool a_mn, bool b_mn,
                                                   bool neg_a = false) {
     return (1u << 4)                       // D format: f32
@@ -328,6 +329,18 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem] (kind::tf32: fp32 operands, read as tf32; K = 8 per
+// instruction, i.e. the same 32 bytes of an operand row as a kind::f16 k-step); one thread.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
         : "memory");
 }
