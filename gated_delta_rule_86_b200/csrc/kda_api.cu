@@ -175,9 +175,10 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
     if (out_dtype == KDA_F32)
         return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
-                                                     T, H, d_v, out, final_state, workspace, st));
+                                                     T, H, d_v, out, final_state, workspace, workspace_bytes, st));
     return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                                         B, T, H, d_v, out, final_state, workspace, st));
+                                                         B, T, H, d_v, out, final_state, workspace, workspace_bytes,
+                                                         st));
 }
 
 kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, const void *log_alpha,
@@ -191,17 +192,21 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
     if (chunk < 1) return KDA_ERR_INVALID_ARG;
     if (chunk != 64 || dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
     if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
-    const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
-    if (need > KDA_STATIC_WS_BYTES) return KDA_ERR_UNSUPPORTED;
+    // the schedule tables and rings of at least kMinRing images for each chain always fit
+    const int64_t pairs = (int64_t)(cu_seqlens ? num_seqs : B) * H;
+    const int64_t chains = pairs < kda::kMaxChains ? pairs : kda::kMaxChains;
+    if (kda::flags_region_bytes() + (size_t)chains * kda::kMinRing * kda::img_stride(d_v) > KDA_STATIC_WS_BYTES)
+        return KDA_ERR_UNSUPPORTED;
     void *ws = nullptr;
     s = static_ws_address(&ws);
     if (s != KDA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (out_dtype == KDA_F32)
         return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
-                                                     T, H, d_v, out, final_state, ws, st));
+                                                     T, H, d_v, out, final_state, ws, KDA_STATIC_WS_BYTES, st));
     return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                                         B, T, H, d_v, out, final_state, ws, st));
+                                                         B, T, H, d_v, out, final_state, ws, KDA_STATIC_WS_BYTES,
+                                                         st));
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,

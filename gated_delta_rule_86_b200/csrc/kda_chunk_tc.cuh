@@ -17,19 +17,24 @@
 // which equals the token recurrence exactly in exact arithmetic.
 //
 // Work split.  Only U~ and the state update sit on the sequential chain; every
-// other quantity depends on the chunk's own inputs alone.  One cluster of
-// 1 + kNP CTAs handles one (sequence, head):
-//   * prep CTAs (ranks 1..kNP): CTA 1 + p prepares chunks c = p mod kNP: decays,
-//     rebased operands, A and P, the UT transform, then W and U on the tensor
-//     cores.  The finished chunk image (-W, U, Qg = Q exp(G), Kd = K exp(G_last - G),
-//     P, gamma = exp(G_last) and a flag) is bulk-stored to this producer's region
-//     of a global workspace (it stays in L2) and announced to the chain CTA
-//     through a remote mbarrier arrive;
-//   * the chain CTA (rank 0) bulk-loads each image into a two-deep shared-memory
-//     ring and runs, per chunk, one MMA group [-W ; Qg] S (rows 0-63 give
-//     U~ - U, rows 64-127 give Qg S), the U~ epilogue, the MMAs Kd^T U~ and
-//     [. ; P] U~ (adding P U~ to rows 64-127) and the fp32 state update, while
-//     dedicated warps store the output rows.
+// other quantity depends on the chunk's own inputs alone.  One grid, every CTA
+// resident at once (cooperative launch), one CTA per SM:
+//   * chain CTAs (one per (sequence, head) pair in flight; a chain runs its
+//     pairs one after another) copy each chunk image from the chain's ring in a
+//     global workspace (it stays in L2) into a two-deep shared-memory ring and
+//     run, per chunk, one MMA group [-W ; Qg] S (rows 0-63 give U~ - U, rows
+//     64-127 give Qg S), the U~ epilogue, the MMAs Kd^T U~ and [. ; P] U~ (adding
+//     P U~ to rows 64-127) and the fp32 state update, while dedicated warps store
+//     the output rows;
+//   * producer CTAs (all other SMs, shared by all chains) prepare the chunks in
+//     the order the chains need them: decays, rebased operands, A and P, the UT
+//     transform, then W and U on the tensor cores.  The finished chunk image (-W,
+//     U, Qg = Q exp(G), Kd = K exp(G_last - G), P, gamma = exp(G_last) and a
+//     flag) is bulk-stored into its ring slot and announced through a flag in
+//     global memory (release / acquire at GPU scope); the chain announces in turn
+//     which slots it has copied out.
+// Every producer serves every chain, so the preparation throughput per pair is
+// (SMs - chains) / chains producer CTAs rather than a fixed cluster share.
 // The chain CTA computes all d_v columns of S at once: a tcgen05.mma costs about
 // the same for N = 32 and N = 128 value columns, so slicing d_v across CTAs would
 // multiply the tensor-core time of the chain without shortening it.
@@ -79,8 +84,6 @@ constexpr int kDK = 128;
 // and bf16 overflow threshold exp(88.7).
 constexpr float kRangeLimit = 40.f;
 
-constexpr int kNP = 3;                // prep CTAs per cluster
-constexpr int kCL = kNP + 1;          // cluster: chain CTA (rank 0) + prep CTAs
 constexpr int kRoleWarps = 16;                        // warps 0-15 run the role
 constexpr int kRoleThreads = kRoleWarps * 32;
 constexpr int kThreads = kRoleThreads + 128;          // + four helper warps that move data
@@ -260,16 +263,6 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, bool l
     tc::tc_fence_after();
     return !failed;
 }
-// Same with a phase completed by other CTAs of the cluster.
-__device__ __forceinline__ bool role_wait_cluster(uint64_t *bar, uint32_t parity, bool leader, uint32_t bar_id,
-                                                  uint32_t nthreads, volatile int *abort_flag) {
-    bool ok = true;
-    if (leader) ok = tc::mbar_wait_cluster(bar, parity, abort_flag);
-    const bool failed = tc::named_sync_or(bar_id, nthreads, !ok);
-    tc::tc_fence_after();
-    return !failed;
-}
-
 // Wait (bounded, ignoring the abort flag) for all tcgen05 operations this thread issued.
 __device__ __forceinline__ void drain_mma(uint64_t *bar, uint32_t parity) {
     int never = 0;
@@ -277,14 +270,25 @@ __device__ __forceinline__ void drain_mma(uint64_t *bar, uint32_t parity) {
     tc::mbar_wait(bar, parity, &never);
 }
 
-// Per-CTA bookkeeping shared by both roles.
-struct ChunkCtx {
-    int n, h, H, nchunks;
+// Launch-wide schedule (computed on the host by launch_chunk_tc_dv) and its workspace tables.
+// The grid has nchain chain CTAs and nprod producer CTAs, all resident at once (cooperative
+// launch).  Chain k runs the (sequence, head) pairs k, k + nchain, ... one after another; its
+// chunks, counted across those pairs, are numbered t = 0, 1, ...  Producer j prepares the items
+// i = j, j + nprod, ..., item i being chunk t = i / nchain of chain k = i % nchain, and stores
+// its image into slot t % ring of chain k's ring in the workspace.
+struct ChunkSched {
+    int npairs, nchain, nprod, ring, H, T;
+    const int32_t *cu;      // cu_seqlens, or null for [B, T] inputs
+    const int32_t *order;   // sequences longest-first (packed inputs), or null for the identity
+    int *ready;             // [nchain][ring]: 1 + number of the chunk whose image the slot holds
+    int *consumed;          // [nchain]: chunks the chain has copied out of its ring
+    uint8_t *rings;         // [nchain][ring] chunk images (Img layout, Img::kStride apart)
+};
+
+// One (sequence, head) pair.
+struct PairInfo {
+    int n, h, nchunks;
     int64_t t0, t1;
-    uint32_t sbase, tmem;
-    uint8_t *sm;
-    uint8_t *ws_pair;        // this (sequence, head)'s kNP producer regions
-    volatile int *abort_flag;
     // chunk c: first token and valid length
     __device__ __forceinline__ int64_t tok0(int c) const { return t0 + (int64_t)c * kChunk; }
     __device__ __forceinline__ int len(int c) const {
@@ -292,18 +296,72 @@ struct ChunkCtx {
         return static_cast<int>(r < kChunk ? r : kChunk);
     }
 };
+__device__ __forceinline__ PairInfo pair_info(const ChunkSched &s, int p) {
+    PairInfo r;
+    r.h = p % s.H;
+    const int rank = p / s.H;
+    if (s.cu) {
+        r.n = s.order ? s.order[rank] : rank;
+        r.t0 = s.cu[r.n];
+        r.t1 = s.cu[r.n + 1];
+    } else {
+        r.n = rank;
+        r.t0 = (int64_t)rank * s.T;
+        r.t1 = r.t0 + s.T;
+    }
+    r.nchunks = static_cast<int>((r.t1 - r.t0 + kChunk - 1) / kChunk);
+    return r;
+}
+// Chunk t of chain k: its pair and chunk index there; false if the chain has fewer chunks.
+__device__ __forceinline__ bool chain_chunk(const ChunkSched &s, int k, int t, PairInfo &pi, int &c) {
+    if (!s.cu) {   // equal lengths: direct
+        pi = pair_info(s, k);
+        if (pi.nchunks == 0) return false;
+        const int q = t / pi.nchunks, p = k + q * s.nchain;
+        if (p >= s.npairs) return false;
+        pi = pair_info(s, p);
+        c = t - q * pi.nchunks;
+        return true;
+    }
+    for (int p = k; p < s.npairs; p += s.nchain) {
+        pi = pair_info(s, p);
+        if (t < pi.nchunks) {
+            c = t;
+            return true;
+        }
+        t -= pi.nchunks;
+    }
+    return false;
+}
+// Largest number of chunks any chain runs.
+__device__ __forceinline__ int chain_tmax(const ChunkSched &s) {
+    int tmax = 0;
+    for (int k = 0; k < s.nchain; ++k) {
+        int tot = 0;
+        for (int p = k; p < s.npairs; p += s.nchain) tot += pair_info(s, p).nchunks;
+        tmax = tot > tmax ? tot : tmax;
+        if (!s.cu) break;   // equal lengths: chain 0 runs the most pairs
+    }
+    return tmax;
+}
+
+// Per-CTA bookkeeping shared by both roles.
+struct ChunkCtx {
+    uint32_t sbase, tmem;
+    uint8_t *sm;
+    volatile int *abort_flag;
+};
 
 // Mbarriers of one CTA (each role uses its own subset).
 struct ChunkBars {
-    // chain: image slot full / free, MMA completions, producer publications (per producer region)
-    uint64_t full[2], slot_free[2], mma1, mma2, mma3[2], pub[kNP][2];
+    // chain: image slot full / free, MMA completions
+    uint64_t full[2], slot_free[2], mma1, mma2, mma3[2];
     // chain: chunk evaluation mode handed to the output warps, TMEM accumulator read by them
     uint64_t outq[2], d1_free[2];
     int outmode[2];   // 0: no MMAs issued, 1: MMAs issued but evaluated exactly, 2: tensor output
-    // prep: MMA completions, global region consumed by the chain (per region)
-    uint64_t m_ap, m_wu, consumed[2], staged, staging_free, raw_full, raw_free;
+    // prep: MMA completions, staging image and raw input tiles
+    uint64_t m_ap, m_wu, staged, staging_free, raw_full, raw_free;
     uint64_t fin;
-    int chain_ok;   // the chain leader's last MMA wait succeeded (read after a barrier)
 };
 
 // Tensor maps of the token tensors: [tokens][H][d] bf16, one box = 64 tokens x d channels of one
@@ -312,36 +370,64 @@ struct RowMaps {
     CUtensorMap g, k, q, v, o;
 };
 
-// ================================== prep role (cluster ranks 1..kNP) ==================================
-// Producer p prepares chunks c = p, p + kNP, ... with warps 0-15.  Lane 0 of warp 16 stores each
-// finished image to one of the producer's two global regions and announces it; lane 0 of warp 17
-// loads the raw input tiles of the next chunk.
+// ======================================== producer role ==========================================
+// Producer j prepares its items (see ChunkSched) with warps 0-15.  Lane 0 of warp 16 stores each
+// finished image into its ring slot once the chain has copied out the slot's previous image, and
+// publishes it; lane 0 of warp 17 loads the raw input tiles of the next item.
+
+// The producer's current item: chunk t of chain k, i.e. chunk c of pair pi.
+struct ProdItem {
+    int i, k, t, c;
+    PairInfo pi;
+};
+// Advance `it` to the producer's next item (it.i + nprod, ...), skipping chunks past a chain's end;
+// false once no chain has chunk t any more.
+__device__ __forceinline__ bool next_item(const ChunkSched &s, int tmax, ProdItem &it) {
+    for (int i = it.i + s.nprod;; i += s.nprod) {
+        const int t = i / s.nchain, k = i - t * s.nchain;
+        if (t >= tmax) return false;
+        if (chain_chunk(s, k, t, it.pi, it.c)) {
+            it.i = i;
+            it.k = k;
+            it.t = t;
+            return true;
+        }
+    }
+}
+__device__ __forceinline__ bool first_item(const ChunkSched &s, int tmax, int j, ProdItem &it) {
+    it.i = j - s.nprod;
+    return next_item(s, tmax, it);
+}
+
 template <int DV>
-__device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, int p, const RowMaps &maps,
-                                          const __nv_bfloat16 *beta) {
+__device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, const ChunkSched &sched, int j,
+                                          int tmax, const RowMaps &maps, const __nv_bfloat16 *beta) {
     using SM = PrepSmem<DV>;
     using I = Img<DV>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t *const sm = cx.sm;
     const uint32_t sbase = cx.sbase, tmem = cx.tmem;
-    const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
+    const int H = sched.H;
     volatile int *abort_flag = cx.abort_flag;
     if (warp == kRoleWarps) {
         if (lane == 0) {
-            // ---- publisher: staged image -> the chunk's global region (one bulk store), then announce
-            //      the region to the chain CTA ----
-            int kl = 0;
-            for (int c = p; c < nchunks; c += kNP, ++kl) {
-                const int reg = kl & 1;
-                uint8_t *gimg = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
+            // ---- publisher: staged image -> its ring slot (one bulk store), then announce it ----
+            ProdItem it;
+            bool have = first_item(sched, tmax, j, it);
+            for (int kl = 0; have; ++kl, have = next_item(sched, tmax, it)) {
+                const int slot = it.t % sched.ring;
+                uint8_t *gimg = sched.rings + ((size_t)it.k * sched.ring + slot) * I::kStride;
                 if (!tc::mbar_wait(&bars.staged, kl & 1, abort_flag)) break;
+                // the chain has copied out the slot's previous image (chunk t - ring)
+                if (!tc::flag_wait_ge(sched.consumed + it.k, it.t - sched.ring + 1, abort_flag)) break;
+                tc::fence_async_global();
                 tc::bulk_store_nc(gimg, sm + SM::kImg, I::kBytes);
                 tc::bulk_commit();
                 tc::bulk_wait_read_all();
                 tc::mbar_arrive(&bars.staging_free);
                 tc::bulk_wait_all();
                 tc::fence_async_global();
-                tc::mbar_arrive_cluster(tc::mapa(tc::smem_u32(&bars.pub[p][reg]), 0));
+                tc::st_release_gpu(sched.ready + it.k * sched.ring + slot, it.t + 1);
             }
         }
         return;
@@ -350,13 +436,15 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     if (warp == kRoleWarps + 1) {
         if (lane == 0) {
             // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next
-            //      chunk (TMA; rows past the tensor end read as zero, rows past the sequence end are
-            //      masked by the readers), into the A/P operand area once the previous chunk's UT
+            //      item (TMA; rows past the tensor end read as zero, rows past the sequence end are
+            //      masked by the readers), into the A/P operand area once the previous item's UT
             //      scratch is dead ----
-            int kl = 0, issued = -1;
-            for (int c = p; c < nchunks; c += kNP, ++kl) {
+            int issued = -1;
+            ProdItem it;
+            bool have = first_item(sched, tmax, j, it);
+            for (int kl = 0; have; ++kl, have = next_item(sched, tmax, it)) {
                 if (kl >= 1 && !tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag)) break;
-                const int t = static_cast<int>(cx.tok0(c));
+                const int t = static_cast<int>(it.pi.tok0(it.c)), h = it.pi.h;
                 tc::mbar_arrive_expect_tx(&bars.raw_full, SM::kRawBytes);
                 tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
                 tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
@@ -390,11 +478,11 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     float *sT = reinterpret_cast<float *>(sm + SM::kT32);
     float *sS = reinterpret_cast<float *>(sm + SM::kScr32);
 
-    // beta of the next chunk, prefetched into registers (one value per thread of warps 0-1)
+    // beta of the next item, prefetched into registers (one value per thread of warps 0-1)
     float rb = 0.f;
-    auto load_beta = [&](int c) {
-        const int64_t tok0 = cx.tok0(c);
-        rb = (tp < kChunk && tp < cx.len(c)) ? __bfloat162float(beta[(tok0 + tp) * H + h]) : 0.f;
+    auto load_beta = [&](const ProdItem &x) {
+        const int64_t tok0 = x.pi.tok0(x.c);
+        rb = (tp < kChunk && tp < x.pi.len(x.c)) ? __bfloat162float(beta[(tok0 + tp) * H + x.pi.h]) : 0.f;
     };
     // the staged chunk image is complete: set its flag (1: some value left the fp16 range, or the
     // decays the rebasing range; the chain then evaluates the chunk exactly) and hand it to the
@@ -411,15 +499,13 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     };
 
     uint32_t ph_ap = 0, ph_wu = 0;
-    if (p < nchunks) load_beta(p);
-    int kl = 0;
-    for (int c = p; c < nchunks; c += kNP, ++kl) {
-        const int reg = kl & 1;
-        // region `reg` last held this producer's chunk kl - 2: the chain must have loaded it
-        if (kl >= 2 &&
-            !role_wait_cluster(&bars.consumed[reg], ((kl >> 1) - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
-            break;
-        const int L = cx.len(c);
+    ProdItem cur, nxt;
+    bool have = first_item(sched, tmax, j, cur), have_next = false;
+    if (have) load_beta(cur);
+    for (int kl = 0; have; ++kl, cur = nxt, have = have_next) {
+        nxt = cur;
+        have_next = next_item(sched, tmax, nxt);
+        const int L = cur.pi.len(cur.c);
         // the raw inputs of this chunk are in shared memory
         if (!role_wait(&bars.raw_full, kl & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
         // ---- decays: fp32 scan over the chunk, per channel ----
@@ -475,7 +561,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
         }
         if (tc::named_sync_or(kBarRole, kRoleThreads, bad)) {
             // decays too fast for the rebased products: the chain evaluates this chunk exactly
-            if (c + kNP < nchunks) load_beta(c + kNP);
+            if (have_next) load_beta(nxt);
             if (leader) tc::mbar_arrive(&bars.raw_free);
             if (kl >= 1 &&
                 !role_wait(&bars.staging_free, (kl - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
@@ -587,7 +673,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
             }
             tc::mma_commit(&bars.m_ap);
         }
-        if (c + kNP < nchunks) load_beta(c + kNP);
+        if (have_next) load_beta(nxt);
         if (!role_wait(&bars.m_ap, ph_ap, leader, kBarRole, kRoleThreads, abort_flag)) break;
         ph_ap ^= 1u;
 
@@ -801,7 +887,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
     if (leader) drain_mma(&bars.fin, 0);
 }
 
-// ================================== chain role (cluster rank 0) =====================================
+// ========================================== chain role ===========================================
 // The chain works on transposed tiles so that the state and U~ are the A operands of its MMAs,
 // held in TMEM:
 //   D1^T = S^T [-W ; Qg]^T        (columns 0-63: (U~ - U)^T, columns 64-127: (Qg S)^T)
@@ -809,10 +895,11 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, i
 //   D1^T[:, 64:128] += U~^T P^T    (so that columns 64-127 become O^T)
 // Warps 0-15 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
 // channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Warps 16-19 store the outputs; lane 0 of warp 16
-// also loads the chunk images.
+// also copies the chunk images out of the chain's ring.  Chain kc runs the pairs kc, kc + nchain, ...;
+// its chunks are numbered t across them (image slots, barrier phases and ring slots follow t).
 template <int DV, typename TO>
-__device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const RowMaps &maps,
-                                           const __nv_bfloat16 *q,
+__device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const ChunkSched &sched, int kc,
+                                           const RowMaps &maps, const __nv_bfloat16 *q,
                                            const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                                            const __nv_bfloat16 *log_alpha, const __nv_bfloat16 *beta,
                                            const float *init_state, TO *out, float *final_state) {
@@ -821,27 +908,29 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t *const sm = cx.sm;
     const uint32_t sbase = cx.sbase, tmem = cx.tmem;
-    const int H = cx.H, h = cx.h, nchunks = cx.nchunks;
+    const int H = sched.H;
     volatile int *abort_flag = cx.abort_flag;
+    int ttot = 0;   // chunks of this chain
+    for (int p = kc; p < sched.npairs; p += sched.nchain) ttot += pair_info(sched, p).nchunks;
 
     if (warp >= kRoleWarps) {
         // ---- output and image warps 16-19: warp 16 + w reads TMEM lanes 32 w .. 32 w + 31, i.e. value
         //      columns j = 32 w + lane of O^T (columns 64-127 of D1^T[b]) once [. ; P] U~ completed,
-        //      and stages them for TMA tensor stores (double-buffered); lane 0 of warp 16 also moves
-        //      the chunk images from the producers' global regions into the two slots ----
+        //      and stages them for TMA tensor stores (double-buffered); lane 0 of warp 16 also copies
+        //      the chunk images from the chain's ring in global memory into the two slots ----
         const int jo = (warp & 3) * 32 + lane;
         const bool jov = jo < DV;
         const bool lead = warp == kRoleWarps && lane == 0;
         const uint32_t tlo = tc::tmem_lane_base(warp);
         constexpr uint32_t kOutThreads = kThreads - kRoleThreads;
         int last_load = -1;
-        auto load_image = [&](int c) -> bool {   // lane 0 of warp 16
-            const int p = c % kNP, kq = c / kNP, reg = kq & 1;
-            if (!tc::mbar_wait_cluster(&bars.pub[p][reg], (kq >> 1) & 1, abort_flag)) return false;
+        auto load_image = [&](int t) -> bool {   // lane 0 of warp 16
+            const int rs = kc * sched.ring + t % sched.ring;
+            if (!tc::flag_wait_ge(sched.ready + rs, t + 1, abort_flag)) return false;
             tc::fence_async_global();
-            const uint8_t *src = cx.ws_pair + (size_t)(p * 2 + reg) * I::kStride;
-            uint8_t *slot = sm + (c & 1) * SM::kSlotBytes;
-            uint64_t *fb = &bars.full[c & 1];
+            const uint8_t *src = sched.rings + (size_t)rs * I::kStride;
+            uint8_t *slot = sm + (t & 1) * SM::kSlotBytes;
+            uint64_t *fb = &bars.full[t & 1];
             tc::mbar_arrive_expect_tx(fb, I::kBytes);
             tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
             tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
@@ -849,12 +938,12 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
             tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
             tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
-            last_load = c;
+            last_load = t;
             return true;
         };
         if (lead)
-            for (int c = 0; c < 2 && c < nchunks; ++c)
-                if (!load_image(c)) break;
+            for (int t = 0; t < 2 && t < ttot; ++t)
+                if (!load_image(t)) break;
         // a wait by lane 0 of warp 16, whose outcome all four warps share (they leave together)
         auto out_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
             bool ok = true;
@@ -864,83 +953,100 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             return !failed;
         };
         uint32_t ph_q[2] = {0, 0}, ph3[2] = {0, 0};
-        int nstore = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1;
-            // the state warps have chosen how chunk c is evaluated (outmode) ...
-            if (!out_wait(&bars.outq[b], ph_q[b])) break;
-            ph_q[b] ^= 1u;
-            const int mode = *reinterpret_cast<volatile int *>(&bars.outmode[b]);
-            // ... and, when its MMAs were issued, they have completed
-            if (mode >= 1) {
-                if (!out_wait(&bars.mma3[b], ph3[b])) break;
-                ph3[b] ^= 1u;
-            }
-            if (mode == 2) {
-                const int64_t tok0 = cx.tok0(c);
-                const int L = cx.len(c);
-                const bool full = L == kChunk;
-                TO *stage = reinterpret_cast<TO *>(sm + SM::kOut + (nstore & 1) * SM::kOutBytes);
-                if (full) {
-                    // the stores issued from this buffer two chunks ago have read it
-                    if (lead) tc::bulk_wait_read_1();
-                    tc::named_sync(kBarOut, kOutThreads);
+        int nstore = 0, t = 0;
+        bool stop = false;
+        for (int pr = kc; pr < sched.npairs && !stop; pr += sched.nchain) {
+            const PairInfo pi = pair_info(sched, pr);
+            const int h = pi.h;
+            for (int c = 0; c < pi.nchunks; ++c, ++t) {
+                const int b = t & 1;
+                // the state warps have chosen how chunk t is evaluated (outmode) ...
+                if (!out_wait(&bars.outq[b], ph_q[b])) {
+                    stop = true;
+                    break;
                 }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
-                    float o[32];
-                    tc::tmem_ld32(tmem + tlo + kTmD1 + b * 128 + 64 + 32 * half, o);
-                    tc::tmem_ld_wait();
-                    if (half == 1) {
-                        // D1^T[b] may be overwritten by the MMAs of chunk c + 2
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
+                ph_q[b] ^= 1u;
+                const int mode = *reinterpret_cast<volatile int *>(&bars.outmode[b]);
+                // ... and, when its MMAs were issued, they have completed
+                if (mode >= 1) {
+                    if (!out_wait(&bars.mma3[b], ph3[b])) {
+                        stop = true;
+                        break;
                     }
-                    if (!jov) continue;
+                    ph3[b] ^= 1u;
+                }
+                if (mode == 2) {
+                    const int64_t tok0 = pi.tok0(c);
+                    const int L = pi.len(c);
+                    const bool full = L == kChunk;
+                    TO *stage = reinterpret_cast<TO *>(sm + SM::kOut + (nstore & 1) * SM::kOutBytes);
                     if (full) {
-                        TO *col = stage + (jo >> 6) * (kChunk * 64) + (jo & 63) + 32 * half * 64;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) col[i * 64] = from_f32<TO>(o[i]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (32 * half + i < L) out[((tok0 + 32 * half + i) * H + h) * DV + jo] = from_f32<TO>(o[i]);
+                        // the stores issued from this buffer two chunks ago have read it
+                        if (lead) tc::bulk_wait_read_1();
+                        tc::named_sync(kBarOut, kOutThreads);
                     }
-                }
-                if (full) {
-                    tc::fence_async_smem();
-                    tc::named_sync(kBarOut, kOutThreads);
-                    if (lead) {
 #pragma unroll
-                        for (int blk = 0; blk < DV / 64; ++blk)
-                            tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0), stage + blk * (kChunk * 64));
-                        tc::bulk_commit();
+                    for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
+                        float o[32];
+                        tc::tmem_ld32(tmem + tlo + kTmD1 + b * 128 + 64 + 32 * half, o);
+                        tc::tmem_ld_wait();
+                        if (half == 1) {
+                            // D1^T[b] may be overwritten by the MMAs of chunk t + 2
+                            tc::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
+                        }
+                        if (!jov) continue;
+                        if (full) {
+                            TO *col = stage + (jo >> 6) * (kChunk * 64) + (jo & 63) + 32 * half * 64;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) col[i * 64] = from_f32<TO>(o[i]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (32 * half + i < L)
+                                    out[((tok0 + 32 * half + i) * H + h) * DV + jo] = from_f32<TO>(o[i]);
+                        }
                     }
-                    ++nstore;
+                    if (full) {
+                        tc::fence_async_smem();
+                        tc::named_sync(kBarOut, kOutThreads);
+                        if (lead) {
+#pragma unroll
+                            for (int blk = 0; blk < DV / 64; ++blk)
+                                tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0),
+                                                 stage + blk * (kChunk * 64));
+                            tc::bulk_commit();
+                        }
+                        ++nstore;
+                    }
+                } else {
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
                 }
-            } else {
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
+                // chunk t's copy out of the ring completed long ago (the state warps are past it): its
+                // ring slot may be rewritten; the image of chunk t + 2 goes into slot b once the state
+                // warps are done with chunk t
+                bool lok = true;
+                if (lead && t + 2 < ttot) {
+                    int never = 0;
+                    tc::mbar_wait(&bars.full[b], (t >> 1) & 1, &never);
+                    tc::st_release_gpu(sched.consumed + kc, t + 1);
+                    lok = tc::mbar_wait(&bars.slot_free[b], (t >> 1) & 1, abort_flag) && load_image(t + 2);
+                }
+                if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) {
+                    stop = true;
+                    break;
+                }
             }
-            // the image of chunk c + 2 goes into slot b once the state warps are done with chunk c;
-            // chunk c's own copy out of its producer region completed long ago: the region is free
-            bool lok = true;
-            if (lead && c + 2 < nchunks) {
-                int never = 0;
-                tc::mbar_wait(&bars.full[b], (c >> 1) & 1, &never);
-                tc::mbar_arrive_cluster_relaxed(tc::mapa(tc::smem_u32(&bars.consumed[(c / kNP) & 1]), 1 + c % kNP));
-                lok = tc::mbar_wait(&bars.slot_free[b], (c >> 1) & 1, abort_flag) && load_image(c + 2);
-            }
-            if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) break;
         }
         if (lead) {
             tc::bulk_wait_all();   // every output store has completed before the CTA leaves
             // no image copy may still be in flight either
             int never = 0;
-            for (int c = (last_load >= 1 ? last_load - 1 : 0); c <= last_load; ++c)
-                tc::mbar_wait(&bars.full[c & 1], (c >> 1) & 1, &never);
+            for (int tt = (last_load >= 1 ? last_load - 1 : 0); tt <= last_load; ++tt)
+                tc::mbar_wait(&bars.full[tt & 1], (tt >> 1) & 1, &never);
         }
         return;
     }
@@ -955,10 +1061,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     float *redPq = reinterpret_cast<float *>(sm + SM::kRedPq);
     float *redKq = reinterpret_cast<float *>(sm + SM::kRedKq);
 
-    float S[32];  // fp32 master state: S^T[j][c0 + i]
-    const size_t state_base = ((size_t)cx.n * H + h) * kDK * DV + (size_t)c0 * DV + j;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
+    float S[32];  // fp32 master state: S^T[j][c0 + i] of the current pair
+    int h = 0;    // the current pair's head
     // S^T -> fp16 A operand in TMEM (lane j, channels c0..c0+31 in 16 columns); returns whether some
     // entry left the fp16 range
     auto write_state_operand = [&]() -> bool {
@@ -973,9 +1077,6 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         tc::tmem_st_wait();
         return big;
     };
-    tc::tc_fence_before();
-    bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
-
     // token-by-token fp32 evaluation of one chunk from the state in registers
     auto exact_chunk = [&](int64_t tok0, int L) -> bool {
         for (int r = 0; r < L; ++r) {
@@ -1009,117 +1110,137 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     };
 
     uint32_t ph1 = 0, ph2 = 0;
-    for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1, b = c & 1;
-        const int64_t tok0 = cx.tok0(c);
-        const int L = cx.len(c);
-        const uint8_t *slot = sm + s * SM::kSlotBytes;
-        const uint32_t sslot = sbase + s * SM::kSlotBytes;
-        if (!role_wait(&bars.full[s], (c >> 1) & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
-        const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
-        if (leader) {
-            // the output warps have read D1^T[b] of chunk c - 2
-            bool ok = c < 2 || tc::mbar_wait(&bars.d1_free[b], ((c >> 1) - 1) & 1, abort_flag);
-            if (ok && !flagged) {
-                tc::tc_fence_after();
-                // ---- D1^T[b] = S^T [-W ; Qg]^T ----
-                constexpr uint32_t id1 = tc::make_idesc(128, 128, tc::kF16, false, false);
+    int t = 0;   // chunk number within this chain
+    bool stop = false;
+    for (int pr = kc; pr < sched.npairs && !stop; pr += sched.nchain) {
+        const PairInfo pi = pair_info(sched, pr);
+        h = pi.h;
+        const size_t state_base = ((size_t)pi.n * H + h) * kDK * DV + (size_t)c0 * DV + j;
 #pragma unroll
-                for (int kk = 0; kk < kDK / 16; ++kk)
-                    tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8,
-                                   desc_kmajor(sslot + SM::kA1, 128, kk), id1, kk > 0);
-                tc::mma_commit(&bars.mma1);
-            }
-            if (flagged) {
-                bars.outmode[b] = 0;   // no MMAs, no tensor output
-                tc::mbar_arrive(&bars.outq[b]);
-            }
-        }
-        if (!flagged) {
-            if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) break;
-            ph1 ^= 1u;
-            // ---- U~^T = U^T + (-W S)^T (tokens 16 qd + [0, 16)) -> fp16 A operand in TMEM ----
-            bool mybad = force_exact;
-            {
-                float x[16];
-                tc::tmem_ld16(tmem + tl + kTmD1 + b * 128 + qd * 16, x);
-                tc::tmem_ld_wait();
-                uint32_t u[8];
-                if (jv) {
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        float u8[8];
-                        unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 2 * qd + h2, DV)),
-                                  u8);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) x[8 * h2 + i] += u8[i];
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) mybad |= !(fabsf(x[i]) <= 65000.f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[i] = pack_h(x[2 * i], x[2 * i + 1]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[i] = 0u;
-                }
-                tc::tmem_st8(tmem + tl + kTmUt + qd * 8, u);
-                tc::tmem_st_wait();
-            }
-            tc::tc_fence_before();
-            const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
-            if (leader) {
-                tc::tc_fence_after();
-                // ---- D2^T = U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
-                constexpr uint32_t id2 = tc::make_idesc(128, 128, tc::kF16, false, true);
-                constexpr uint32_t id3 = tc::make_idesc(128, kChunk, tc::kF16, false, false);
-#pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk)
-                    tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + SM::kKd, kChunk, kk),
-                                   id2, kk > 0);
-                tc::mma_commit(&bars.mma2);
-#pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk)
-                    tc::mma_f16_ta(tmem + kTmD1 + b * 128 + 64, tmem + kTmUt + kk * 8,
-                                   desc_kmajor(sslot + SM::kP, kChunk, kk), id3, true);
-                tc::mma_commit(&bars.mma3[b]);
-                bars.outmode[b] = bad ? 1 : 2;   // MMAs issued; O^T is the output unless evaluated exactly
-                tc::mbar_arrive(&bars.outq[b]);
-            }
-            if (!role_wait(&bars.mma2, ph2, leader, kBarRole, kRoleThreads, abort_flag)) break;
-            ph2 ^= 1u;
-            if (!bad) {
-                // ---- S^T = S^T Diag(gamma) + D2^T ----
-                const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
-                {
-                    float d[32];
-                    tc::tmem_ld32(tmem + tl + kTmD2 + c0, d);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                        const float4 gg = gam4[i4];
-                        const int i = 4 * i4;
-                        S[i] = fmaf(gg.x, S[i], d[i]);
-                        S[i + 1] = fmaf(gg.y, S[i + 1], d[i + 1]);
-                        S[i + 2] = fmaf(gg.z, S[i + 2], d[i + 2]);
-                        S[i + 3] = fmaf(gg.w, S[i + 3], d[i + 3]);
-                    }
-                }
-                const bool big = write_state_operand();
-                tc::tc_fence_before();
-                force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
-                if (leader) tc::mbar_arrive(&bars.slot_free[s]);   // done with the slot
-                continue;
-            }
-        }
-        // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
-        const bool big = exact_chunk(tok0, L);
+        for (int i = 0; i < 32; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
         tc::tc_fence_before();
-        force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
-        if (leader) tc::mbar_arrive(&bars.slot_free[s]);
-    }
-    if (final_state && *abort_flag == 0 && jv) {
+        bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
+        for (int c = 0; c < pi.nchunks; ++c, ++t) {
+            const int s = t & 1, b = t & 1;
+            const int64_t tok0 = pi.tok0(c);
+            const int L = pi.len(c);
+            const uint8_t *slot = sm + s * SM::kSlotBytes;
+            const uint32_t sslot = sbase + s * SM::kSlotBytes;
+            if (!role_wait(&bars.full[s], (t >> 1) & 1, leader, kBarRole, kRoleThreads, abort_flag)) {
+                stop = true;
+                break;
+            }
+            const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
+            if (leader) {
+                // the output warps have read D1^T[b] of chunk t - 2
+                bool ok = t < 2 || tc::mbar_wait(&bars.d1_free[b], ((t >> 1) - 1) & 1, abort_flag);
+                if (ok && !flagged) {
+                    tc::tc_fence_after();
+                    // ---- D1^T[b] = S^T [-W ; Qg]^T ----
+                    constexpr uint32_t id1 = tc::make_idesc(128, 128, tc::kF16, false, false);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) final_state[state_base + (size_t)i * DV] = S[i];
+                    for (int kk = 0; kk < kDK / 16; ++kk)
+                        tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8,
+                                       desc_kmajor(sslot + SM::kA1, 128, kk), id1, kk > 0);
+                    tc::mma_commit(&bars.mma1);
+                }
+                if (flagged) {
+                    bars.outmode[b] = 0;   // no MMAs, no tensor output
+                    tc::mbar_arrive(&bars.outq[b]);
+                }
+            }
+            if (!flagged) {
+                if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                ph1 ^= 1u;
+                // ---- U~^T = U^T + (-W S)^T (tokens 16 qd + [0, 16)) -> fp16 A operand in TMEM ----
+                bool mybad = force_exact;
+                {
+                    float x[16];
+                    tc::tmem_ld16(tmem + tl + kTmD1 + b * 128 + qd * 16, x);
+                    tc::tmem_ld_wait();
+                    uint32_t u[8];
+                    if (jv) {
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            float u8[8];
+                            unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 2 * qd + h2, DV)),
+                                      u8);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) x[8 * h2 + i] += u8[i];
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) mybad |= !(fabsf(x[i]) <= 65000.f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) u[i] = pack_h(x[2 * i], x[2 * i + 1]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) u[i] = 0u;
+                    }
+                    tc::tmem_st8(tmem + tl + kTmUt + qd * 8, u);
+                    tc::tmem_st_wait();
+                }
+                tc::tc_fence_before();
+                const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
+                if (leader) {
+                    tc::tc_fence_after();
+                    // ---- D2^T = U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
+                    constexpr uint32_t id2 = tc::make_idesc(128, 128, tc::kF16, false, true);
+                    constexpr uint32_t id3 = tc::make_idesc(128, kChunk, tc::kF16, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < kChunk / 16; ++kk)
+                        tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + SM::kKd, kChunk, kk),
+                                       id2, kk > 0);
+                    tc::mma_commit(&bars.mma2);
+#pragma unroll
+                    for (int kk = 0; kk < kChunk / 16; ++kk)
+                        tc::mma_f16_ta(tmem + kTmD1 + b * 128 + 64, tmem + kTmUt + kk * 8,
+                                       desc_kmajor(sslot + SM::kP, kChunk, kk), id3, true);
+                    tc::mma_commit(&bars.mma3[b]);
+                    bars.outmode[b] = bad ? 1 : 2;   // MMAs issued; O^T is the output unless evaluated exactly
+                    tc::mbar_arrive(&bars.outq[b]);
+                }
+                if (!role_wait(&bars.mma2, ph2, leader, kBarRole, kRoleThreads, abort_flag)) {
+                    stop = true;
+                    break;
+                }
+                ph2 ^= 1u;
+                if (!bad) {
+                    // ---- S^T = S^T Diag(gamma) + D2^T ----
+                    const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
+                    {
+                        float d[32];
+                        tc::tmem_ld32(tmem + tl + kTmD2 + c0, d);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 gg = gam4[i4];
+                            const int i = 4 * i4;
+                            S[i] = fmaf(gg.x, S[i], d[i]);
+                            S[i + 1] = fmaf(gg.y, S[i + 1], d[i + 1]);
+                            S[i + 2] = fmaf(gg.z, S[i + 2], d[i + 2]);
+                            S[i + 3] = fmaf(gg.w, S[i + 3], d[i + 3]);
+                        }
+                    }
+                    const bool big = write_state_operand();
+                    tc::tc_fence_before();
+                    force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+                    if (leader) tc::mbar_arrive(&bars.slot_free[s]);   // done with the slot
+                    continue;
+                }
+            }
+            // exact path: the chunk's decays exceed the rebasing range, or an fp16 value overflowed
+            const bool big = exact_chunk(tok0, L);
+            tc::tc_fence_before();
+            force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+            if (leader) tc::mbar_arrive(&bars.slot_free[s]);
+        }
+        if (!stop && final_state && *abort_flag == 0 && jv) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) final_state[state_base + (size_t)i * DV] = S[i];
+        }
     }
     if (leader) drain_mma(&bars.fin, 0);
 }
@@ -1127,34 +1248,22 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
 // ====================================== kernel and launch ==========================================
 template <int DV, typename TO>
 __global__ void __launch_bounds__(kThreads, 1)
-kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __nv_bfloat16 *__restrict__ q,
-                    const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-                    const __nv_bfloat16 *__restrict__ log_alpha, const __nv_bfloat16 *__restrict__ beta,
-                    const float *init_state, const int32_t *__restrict__ cu_seqlens, int num_seqs, int T, int H,
-                    TO *__restrict__ out, float *final_state, uint8_t *__restrict__ workspace) {
+kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant__ ChunkSched sched,
+                    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                    const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ log_alpha,
+                    const __nv_bfloat16 *__restrict__ beta, const float *init_state, TO *__restrict__ out,
+                    float *final_state) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ ChunkBars bars;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ int s_slot;
+    __shared__ int s_tmax;
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int rank = static_cast<int>(tc::cluster_ctarank());
-    const int pair = blockIdx.x / kCL;
-    const int h = pair % H;
-    int n = pair / H;
-    int64_t t0, t1;
-    if (cu_seqlens) {
-        if (num_seqs <= kLongestFirstMaxSeqs) n = longest_first_seq(cu_seqlens, num_seqs, n, &s_slot);
-        t0 = cu_seqlens[n];
-        t1 = cu_seqlens[n + 1];
-    } else {
-        t0 = (int64_t)n * T;
-        t1 = t0 + T;
-    }
-
+    const bool is_chain = static_cast<int>(blockIdx.x) < sched.nchain;
     if (tid == 0) {
+        if (!is_chain) s_tmax = chain_tmax(sched);
         tc::mbar_init(&bars.full[0], 1);
         tc::mbar_init(&bars.full[1], 1);
         tc::mbar_init(&bars.slot_free[0], 1);
@@ -1167,14 +1276,8 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __nv_bfloat16 *_
         tc::mbar_init(&bars.outq[1], 1);
         tc::mbar_init(&bars.d1_free[0], kThreads / 32 - kRoleWarps);
         tc::mbar_init(&bars.d1_free[1], kThreads / 32 - kRoleWarps);
-        for (int p = 0; p < kNP; ++p) {
-            tc::mbar_init(&bars.pub[p][0], 1);
-            tc::mbar_init(&bars.pub[p][1], 1);
-        }
         tc::mbar_init(&bars.m_ap, 1);
         tc::mbar_init(&bars.m_wu, 1);
-        tc::mbar_init(&bars.consumed[0], 1);
-        tc::mbar_init(&bars.consumed[1], 1);
         tc::mbar_init(&bars.staged, 1);
         tc::mbar_init(&bars.staging_free, 1);
         tc::mbar_init(&bars.raw_full, 1);
@@ -1183,43 +1286,75 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __nv_bfloat16 *_
         tc::fence_mbar_init();
         abort_flag = 0;
     }
-    const uint32_t ncols = rank == 0 ? kTmChainCols : kTmPrepCols;
+    const uint32_t ncols = is_chain ? kTmChainCols : kTmPrepCols;
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base_sh, ncols);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
     __syncthreads();
-    tc::cluster_sync();  // every CTA's barriers are initialised before any remote arrive
     tc::tc_fence_after();
 
     ChunkCtx cx;
-    cx.n = n;
-    cx.h = h;
-    cx.H = H;
-    cx.t0 = t0;
-    cx.t1 = t1;
-    cx.nchunks = static_cast<int>((t1 - t0 + kChunk - 1) / kChunk);
     cx.sm = sm;
     cx.sbase = tc::smem_u32(sm);
     cx.tmem = tmem_base_sh;
-    cx.ws_pair = workspace + (size_t)pair * kNP * 2 * Img<DV>::kStride;
     cx.abort_flag = &abort_flag;
-    if (rank == 0)
-        chain_role<DV, TO>(cx, bars, maps, q, k, v, log_alpha, beta, init_state, out, final_state);
+    if (is_chain)
+        chain_role<DV, TO>(cx, bars, sched, blockIdx.x, maps, q, k, v, log_alpha, beta, init_state, out,
+                           final_state);
     else
-        prep_role<DV>(cx, bars, rank - 1, maps, beta);
+        prep_role<DV>(cx, bars, sched, blockIdx.x - sched.nchain, s_tmax, maps, beta);
 
     tc::tc_fence_before();
     __syncthreads();
-    tc::cluster_sync();  // no CTA leaves while a peer may still signal its barriers
     if (warp == 0) tc::tmem_dealloc(cx.tmem, ncols);
 }
 
-// Bytes of global workspace kda_chunk_fwd needs on the tensor-core path: two chunk
-// image regions per (sequence, head) and prep CTA.
+// Workspace tables of the schedule: zeroes the ring flags and, for packed sequences, writes the
+// longest-first order of the sequences (ties by index), so that long sequences start first.
+__global__ void __launch_bounds__(256) kda_chunk_sched_kernel(const int32_t *__restrict__ cu, int num_seqs,
+                                                              int32_t *order, int *flags, int nflags) {
+    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0;
+    if (!order) return;
+    for (int n = threadIdx.x; n < num_seqs; n += blockDim.x) {
+        const int ln = cu[n + 1] - cu[n];
+        int rank = 0;
+        for (int m = 0; m < num_seqs; ++m) {
+            const int lm = cu[m + 1] - cu[m];
+            rank += (lm > ln) || (lm == ln && m < n);
+        }
+        order[rank] = n;
+    }
+}
+
+// Grid split for npairs (sequence, head) pairs on nsm SMs: at most a quarter of the SMs (and 64)
+// run chains, a pair each per wave; the rest produce chunk images.
+struct ChunkGrid {
+    int nchain, nprod;
+};
+inline ChunkGrid chunk_grid(int64_t npairs, int nsm) {
+    ChunkGrid g;
+    int cap = nsm / 4;
+    cap = cap < 1 ? 1 : (cap > 64 ? 64 : cap);
+    const int64_t waves = (npairs + cap - 1) / cap;
+    g.nchain = static_cast<int>((npairs + waves - 1) / waves);
+    g.nprod = nsm - g.nchain;
+    return g;
+}
+constexpr int kRing = 8;                 // ring slots per chain (workspace variant)
+constexpr int kMinRing = 3;
+constexpr int kMaxChains = 64;
+constexpr size_t kFlagsBytes = 4096 + (size_t)(kMaxChains * kRing + kMaxChains) * 4;   // order + flags
+template <int DV> constexpr size_t ring_stride() { return Img<DV>::kStride; }
+inline size_t img_stride(int DV) { return DV == 64 ? Img<64>::kStride : Img<128>::kStride; }
+inline size_t flags_region_bytes() { return (kFlagsBytes + 1023) / 1024 * 1024; }
+
+// Bytes of global workspace kda_chunk_fwd needs on the tensor-core path: the schedule tables and a
+// ring of kRing chunk images for each chain (at most kMaxChains chains, whatever the SM count).
 inline size_t chunk_tc_workspace_bytes(int64_t pairs, int DV) {
-    return static_cast<size_t>(pairs) * kNP * 2 * (DV == 64 ? Img<64>::kStride : Img<128>::kStride);
+    const int64_t chains = pairs < kMaxChains ? pairs : kMaxChains;
+    return flags_region_bytes() + static_cast<size_t>(chains) * kRing * img_stride(DV);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
@@ -1251,15 +1386,43 @@ inline bool encode_row_map(CUtensorMap *m, const void *base, int d, int H, int64
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SM count of the current device (cached per device).
+inline int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static int cache[64] = {};
+    if (dev < 0 || dev >= 64) return 0;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Launches the schedule-table kernel and the chunk kernel.  `ws_bytes` bounds the ring depth: the
+// workspace holds the schedule tables and nchain rings of `ring` images (kMinRing <= ring <= kRing).
 template <int DV, typename TO>
 cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, const void *la, const void *beta,
                                const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H,
-                               void *out, float *final_state, void *workspace, cudaStream_t stream) {
+                               void *out, float *final_state, void *workspace, size_t ws_bytes,
+                               cudaStream_t stream) {
     auto kern = kda_chunk_tc_kernel<DV, TO>;
     const int smem = chunk_smem_bytes<DV>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int N = cu ? num_seqs : B;
+    const int64_t npairs = (int64_t)N * H;
+    if (npairs <= 0) return cudaSuccess;
+    const int nsm = device_sm_count();
+    if (nsm < 2) return cudaErrorInvalidDevice;
+    const ChunkGrid grid = chunk_grid(npairs, nsm);
+    const size_t flags = flags_region_bytes();
+    if (ws_bytes < flags) return cudaErrorInvalidValue;
+    int64_t ring = static_cast<int64_t>((ws_bytes - flags) / ((size_t)grid.nchain * Img<DV>::kStride));
+    if (ring > kRing) ring = kRing;
+    if (ring < kMinRing) return cudaErrorInvalidValue;
+
     RowMaps maps;
     memset(&maps, 0, sizeof(maps));
     const int64_t tokens = (int64_t)B * T;
@@ -1271,34 +1434,52 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
                             static_cast<int>(sizeof(TO))))
             return cudaErrorInvalidValue;
     }
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    ChunkSched sched;
+    sched.npairs = static_cast<int>(npairs);
+    sched.nchain = grid.nchain;
+    sched.nprod = grid.nprod;
+    sched.ring = static_cast<int>(ring);
+    sched.H = H;
+    sched.T = T;
+    sched.cu = cu;
+    const bool sorted = cu && num_seqs <= kLongestFirstMaxSeqs;
+    sched.order = sorted ? reinterpret_cast<const int32_t *>(ws) : nullptr;
+    sched.ready = reinterpret_cast<int *>(ws + 4096);
+    sched.consumed = sched.ready + grid.nchain * sched.ring;
+    sched.rings = ws + flags;
+    const int nflags = grid.nchain * sched.ring + grid.nchain;
+    kda_chunk_sched_kernel<<<1, 256, 0, stream>>>(cu, num_seqs, sorted ? reinterpret_cast<int32_t *>(ws) : nullptr,
+                                                  sched.ready, nflags);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // every CTA must be resident at once (chains and producers wait on one another)
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(N) * H * kCL);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid.nchain + grid.nprod));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, kern, maps, static_cast<const __nv_bfloat16 *>(q),
+    return cudaLaunchKernelEx(&cfg, kern, maps, sched, static_cast<const __nv_bfloat16 *>(q),
                               static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
                               static_cast<const __nv_bfloat16 *>(la), static_cast<const __nv_bfloat16 *>(beta),
-                              init_state, cu, num_seqs, T, H, static_cast<TO *>(out), final_state,
-                              static_cast<uint8_t *>(workspace));
+                              init_state, static_cast<TO *>(out), final_state);
 }
 
 template <typename TO>
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *la, const void *beta,
                             const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
-                            void *out, float *final_state, void *workspace, cudaStream_t stream) {
+                            void *out, float *final_state, void *workspace, size_t ws_bytes, cudaStream_t stream) {
     if (DV == 64)
         return launch_chunk_tc_dv<64, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
-                                          workspace, stream);
+                                          workspace, ws_bytes, stream);
     return launch_chunk_tc_dv<128, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
-                                       workspace, stream);
+                                       workspace, ws_bytes, stream);
 }
 
 }  // namespace kda

@@ -156,6 +156,38 @@ __device__ __forceinline__ void cluster_sync() {
 }
 __device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
+// ---- flags in global memory (progress signals between CTAs of one grid) -----------------------
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Longest wait on a global flag before the kernel gives up (a healthy grid waits microseconds).
+constexpr uint64_t kFlagWaitNs = 2000000000ull;
+// Wait until *p >= v (acquire, GPU scope), bounded by kFlagWaitNs; same contract as mbar_wait.
+__device__ __forceinline__ bool flag_wait_ge(const int *p, int v, volatile int *abort) {
+    if (ld_acquire_gpu(p) >= v) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(p) >= v) return true;
+        if (*abort) return false;
+        if ((i & 255u) == 255u && global_ns() - t0 > kFlagWaitNs) break;
+    }
+    record_device_error(kDevErrTimeout);
+    *abort = 1;
+    return false;
+}
+
 // Bulk copy global -> this CTA's shared memory; completes `bytes` of transaction on `bar`.
 __device__ __forceinline__ void bulk_load(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

@@ -93,6 +93,10 @@ typedef enum {
  * Supported: d_k == 128 and d_v in {64, 128} for bf16 (tensor-core path);
  * d_k, d_v in {64, 128} for fp32 (fp32 CUDA-core path, fp32 accuracy).
  * T == 0 is valid (final_state = init_state or zeros).
+ * The tensor-core path launches one CTA per SM of the device as a cooperative
+ * grid (its CTAs wait on one another, so all must be resident at once); the
+ * launch fails (KDA_ERR_CUDA) rather than start when the GPU cannot hold them
+ * all, e.g. while another kernel occupies some SMs.
  */
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
                          const void *beta, const float *init_state, const int32_t *cu_seqlens,
@@ -103,11 +107,12 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
 
 /*
  * Workspace kda_chunk_fwd needs, in bytes, for N sequences (B, or num_seqs with
- * cu_seqlens) of H heads: on the tensor-core path, six chunk images (73 KB each
- * at d_v = 128, 65 KB at d_v = 64) per (sequence, head), through which the
- * CTAs that prepare the chunk operands hand them to the CTA that runs the
- * state recurrence (two regions per preparing CTA); 0 on the fp32 path.  Pure
- * host computation, never fails for valid sizes.
+ * cu_seqlens) of H heads: on the tensor-core path, about 7 KB of schedule
+ * tables (ring flags, sequence order) and, for each of up to min(N * H, 64)
+ * chains, a ring of 8 chunk images (73 KB each at d_v = 128, 65 KB at
+ * d_v = 64) through which the CTAs that prepare the chunk operands hand them
+ * to the CTA that runs the state recurrence; 0 on the fp32 path.  Pure host
+ * computation, never fails for valid sizes.
  */
 kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v,
                                         kda_dtype dtype, size_t *bytes);
@@ -155,10 +160,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
  * Same arguments, layouts and results as kda_chunk_fwd, without workspace /
  * workspace_bytes.  Only the tensor-core path: dtype KDA_BF16, d_k == 128,
  * d_v in {64, 128}.  It allocates nothing (no cudaMalloc, no library
- * allocator).  KDA_ERR_UNSUPPORTED if the problem needs more than
- * KDA_STATIC_WS_BYTES of handoff buffer, i.e. more than
- * KDA_STATIC_WS_BYTES / kda_chunk_fwd_workspace_size(1, 1, ...) (sequence,
- * head) pairs: 37 at d_v = 128, 42 at d_v = 64.
+ * allocator).  Any number of (sequence, head) pairs fits: the chains' rings
+ * are made shallower (down to 3 images) when the array cannot hold 8 each.
  *
  * The first call on a device looks up that device's copy of the array (with
  * the device current), so make that first call before any stream capture.

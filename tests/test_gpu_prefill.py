@@ -45,7 +45,7 @@ def test_tiny_fp32_recurrent(cuda_lib):
 # ---- small ragged bf16 cases -------------------------------------------------------------------
 
 @pytest.mark.parametrize("T", [1, 17, 64, 65, 200, 333])
-@pytest.mark.parametrize("H", [2, 80])   # 2 pairs -> 32-wide d_v slices, 80 pairs -> 64-wide
+@pytest.mark.parametrize("H", [2, 80])   # 80 (sequence, head) pairs: chains run several pairs in turn
 def test_chunk_bf16_ragged(cuda_lib, T, H):
     x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=T, H=H, init_state=True)
     run_and_check(kda_chunk_fwd, x, BF16_TOL, heads=[0, H - 1] if H > 2 else None)

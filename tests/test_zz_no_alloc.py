@@ -7,7 +7,7 @@ buffer from a fixed array inside the library instead.  This file checks,
 through the C ABI, that two calls in a row give the same results as
 kda_chunk_fwd (within the parity tolerance of the other tests; the array
 keeps the previous call's contents, which must not leak into the next call),
-and that a problem larger than the array is refused without a launch.
+also for more (sequence, head) pairs than the GPU runs chains at once.
 
 Collected last on purpose (file name), and self-contained: it passes both
 alone in a fresh process and after every other test.
@@ -68,8 +68,14 @@ def test_two_calls_match_kda_chunk_fwd(cuda_lib):
         assert rel_err(fs, ref_s.double().cpu().numpy()) <= BF16_TOL
 
 
-def test_refuses_problems_beyond_the_fixed_buffer(cuda_lib):
+def test_more_pairs_than_chains(cuda_lib):
+    # 70 (sequence, head) pairs: more than one wave of chains (at most a quarter of the SMs), so
+    # chains run several pairs and the fixed array holds shallower rings
     fn = _static_ws(cuda_lib)
-    x = _case(T=64, H=70, dv=128, seed=13)   # 70 (sequence, head) pairs > 37 at d_v = 128
-    st, _, _ = _call(fn, x)
-    assert st == _lib.KDA_ERR_UNSUPPORTED
+    x = _case(T=130, H=70, dv=128, seed=13)
+    ref_o, ref_s = kda_chunk_fwd(*(x[n] for n in NAMES), initial_state=x["init_state"])
+    st, out, fs = _call(fn, x)
+    torch.cuda.synchronize()
+    assert st == _lib.KDA_OK, _lib.status_string(st)
+    assert rel_err(out, ref_o.double().cpu().numpy()) <= BF16_TOL
+    assert rel_err(fs, ref_s.double().cpu().numpy()) <= BF16_TOL
