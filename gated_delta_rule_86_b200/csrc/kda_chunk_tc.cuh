@@ -142,13 +142,14 @@ template <int DV> struct PrepSmem {
     // them); the first Tb is also the B operand of U^T = V^T Tb^T
     static constexpr int kTbP = kKgV + kChunk * 2 * kDK * 2;
     static constexpr int kImg = kTbP + 2 * kChunk * kChunk * 2;  // staging image (Img layout)
-    static constexpr int kBeta = kImg + I::kStride;              // fp32 [64]
-    static constexpr int kG0 = kBeta + kChunk * 4;               // fp32 [128] decay after token 0
+    static constexpr int kG0 = kImg + I::kStride;                // fp32 [128] decay after token 0
     static constexpr int kGref = kG0 + kDK * 4;                  //            after token 31
     static constexpr int kGlast = kGref + kDK * 4;               //            after token 63
     static constexpr int kEref = kGlast + kDK * 4;               // exp(Gref)
     static constexpr int kElast = kEref + kDK * 4;               // exp(Glast - Gref)
-    static constexpr int kBytes = kElast + kDK * 4;
+    static constexpr int kBetaIn = kElast + kDK * 4;              // fp32 [2][64] beta of items kl, kl + 1
+    static constexpr int kLenIn = kBetaIn + 2 * kChunk * 4;       // int [2] valid tokens (-1: no item)
+    static constexpr int kBytes = kLenIn + 16;
     // The A/P operand area also holds, in turn: the raw bf16 inputs of the chunk (bulk-loaded
     // rows of log_alpha, k, q, v; read into registers before the operands are written) and the
     // fp32 scratch of the UT transform (once the A/P products complete).
@@ -417,9 +418,9 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             for (int kl = 0; have; ++kl, have = next_item(sched, tmax, it)) {
                 const int slot = it.t % sched.ring;
                 uint8_t *gimg = sched.rings + ((size_t)it.k * sched.ring + slot) * I::kStride;
-                if (!tc::mbar_wait(&bars.staged, kl & 1, abort_flag)) break;
                 // the chain has copied out the slot's previous image (chunk t - ring)
                 if (!tc::flag_wait_ge(sched.consumed + it.k, it.t - sched.ring + 1, abort_flag)) break;
+                if (!tc::mbar_wait(&bars.staged, kl & 1, abort_flag)) break;
                 tc::fence_async_global();
                 tc::bulk_store_nc(gimg, sm + SM::kImg, I::kBytes);
                 tc::bulk_commit();
@@ -434,29 +435,47 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     }
     if (warp >= kRoleWarps + 2) return;   // warps 18, 19 serve the chain CTA only
     if (warp == kRoleWarps + 1) {
-        if (lane == 0) {
-            // ---- raw input loader: the 64-token tiles of log_alpha, k, q, v of this producer's next
-            //      item (TMA; rows past the tensor end read as zero, rows past the sequence end are
-            //      masked by the readers), into the A/P operand area once the previous item's UT
-            //      scratch is dead ----
-            int issued = -1;
-            ProdItem it;
-            bool have = first_item(sched, tmax, j, it);
-            for (int kl = 0; have; ++kl, have = next_item(sched, tmax, it)) {
-                if (kl >= 1 && !tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag)) break;
-                const int t = static_cast<int>(it.pi.tok0(it.c)), h = it.pi.h;
-                tc::mbar_arrive_expect_tx(&bars.raw_full, SM::kRawBytes);
-                tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
-                tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
-                tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
-                tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
-                issued = kl;
+        // ---- item loader: for each item, lane 0 issues the 64-token TMA tiles of log_alpha, k, q,
+        //      v (rows past the tensor end read as zero, rows past the sequence end are masked by the
+        //      readers) into the A/P operand area once the previous item's UT scratch is dead; the
+        //      warp then stores the item's beta and length into shared memory.  raw_full completes
+        //      with both arrivals and the tile bytes.  After the last item a length of -1 (no tiles)
+        //      tells the compute warps to stop ----
+        float *sBetaIn = reinterpret_cast<float *>(sm + SM::kBetaIn);
+        int *sLenIn = reinterpret_cast<int *>(sm + SM::kLenIn);
+        int last = -1;   // last raw_full phase this warp arrived on
+        ProdItem it;
+        bool have = first_item(sched, tmax, j, it);
+        for (int kl = 0;; ++kl) {
+            bool ok = true;
+            if (lane == 0 && kl >= 1) ok = tc::mbar_wait(&bars.raw_free, (kl - 1) & 1, abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int64_t tok0 = have ? it.pi.tok0(it.c) : 0;
+            const int L = have ? it.pi.len(it.c) : -1, h = it.pi.h;
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&bars.raw_full, have ? SM::kRawBytes : 0);
+                if (have) {
+                    const int t = static_cast<int>(tok0);
+                    tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
+                    tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
+                    tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
+                    tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
+                }
             }
-            // no copy may still be in flight when the CTA leaves
-            if (issued >= 0) {
-                int never = 0;
-                tc::mbar_wait(&bars.raw_full, issued & 1, &never);
-            }
+            float *bdst = sBetaIn + (kl & 1) * kChunk;
+            bdst[lane] = (lane < L) ? __bfloat162float(beta[(tok0 + lane) * H + h]) : 0.f;
+            bdst[32 + lane] = (32 + lane < L) ? __bfloat162float(beta[(tok0 + 32 + lane) * H + h]) : 0.f;
+            if (lane == 0) sLenIn[kl & 1] = L;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars.raw_full);
+            last = kl;
+            if (!have) break;
+            have = next_item(sched, tmax, it);
+        }
+        // no copy may still be in flight when the CTA leaves (phases complete in order)
+        if (lane == 0 && last >= 0) {
+            int never = 0;
+            tc::mbar_wait(&bars.raw_full, last & 1, &never);
         }
         return;
     }
@@ -467,7 +486,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     const int cg = tp & 15, tg = tp >> 4;   // channels [8cg, 8cg+8), tokens 2tg, 2tg + 1
     const int sp = warp & 3, q4 = warp >> 2;
     const uint32_t tl = tc::tmem_lane_base(warp);
-    float *sBeta = reinterpret_cast<float *>(sm + SM::kBeta);
+    const int *sLenIn = reinterpret_cast<const int *>(sm + SM::kLenIn);
     float *sG0 = reinterpret_cast<float *>(sm + SM::kG0);
     float *sGref = reinterpret_cast<float *>(sm + SM::kGref);
     float *sGlast = reinterpret_cast<float *>(sm + SM::kGlast);
@@ -478,12 +497,6 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     float *sT = reinterpret_cast<float *>(sm + SM::kT32);
     float *sS = reinterpret_cast<float *>(sm + SM::kScr32);
 
-    // beta of the next item, prefetched into registers (one value per thread of warps 0-1)
-    float rb = 0.f;
-    auto load_beta = [&](const ProdItem &x) {
-        const int64_t tok0 = x.pi.tok0(x.c);
-        rb = (tp < kChunk && tp < x.pi.len(x.c)) ? __bfloat162float(beta[(tok0 + tp) * H + x.pi.h]) : 0.f;
-    };
     // the staged chunk image is complete: set its flag (1: some value left the fp16 range, or the
     // decays the rebasing range; the chain then evaluates the chunk exactly) and hand it to the
     // publisher
@@ -499,15 +512,12 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     };
 
     uint32_t ph_ap = 0, ph_wu = 0;
-    ProdItem cur, nxt;
-    bool have = first_item(sched, tmax, j, cur), have_next = false;
-    if (have) load_beta(cur);
-    for (int kl = 0; have; ++kl, cur = nxt, have = have_next) {
-        nxt = cur;
-        have_next = next_item(sched, tmax, nxt);
-        const int L = cur.pi.len(cur.c);
-        // the raw inputs of this chunk are in shared memory
+    for (int kl = 0;; ++kl) {
+        // the raw inputs, beta and length of the item are in shared memory
         if (!role_wait(&bars.raw_full, kl & 1, leader, kBarRole, kRoleThreads, abort_flag)) break;
+        const int L = sLenIn[kl & 1];
+        if (L < 0) break;   // no more items
+        const float *sBeta = reinterpret_cast<const float *>(sm + SM::kBetaIn) + (kl & 1) * kChunk;
         // ---- decays: fp32 scan over the chunk, per channel ----
         float G[2][8];
         {
@@ -540,7 +550,6 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
 #pragma unroll
                 for (int i = 0; i < 8; ++i) sG0[cg * 8 + i] = G[0][i];             // token 0: no prefix
             }
-            if (tp < kChunk) sBeta[tp] = rb;
         }
         tc::named_sync(kBarRole, kRoleThreads);
         // per channel: exclusive prefix over the 16 warps, G after tokens 31 and 63, range check
@@ -561,7 +570,6 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
         }
         if (tc::named_sync_or(kBarRole, kRoleThreads, bad)) {
             // decays too fast for the rebased products: the chain evaluates this chunk exactly
-            if (have_next) load_beta(nxt);
             if (leader) tc::mbar_arrive(&bars.raw_free);
             if (kl >= 1 &&
                 !role_wait(&bars.staging_free, (kl - 1) & 1, leader, kBarRole, kRoleThreads, abort_flag))
@@ -673,7 +681,6 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             }
             tc::mma_commit(&bars.m_ap);
         }
-        if (have_next) load_beta(nxt);
         if (!role_wait(&bars.m_ap, ph_ap, leader, kBarRole, kRoleThreads, abort_flag)) break;
         ph_ap ^= 1u;
 
@@ -960,6 +967,15 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const int h = pi.h;
             for (int c = 0; c < pi.nchunks; ++c, ++t) {
                 const int b = t & 1;
+                // first the image of chunk t + 1, into slot b ^ 1 once the state warps are done with
+                // chunk t - 1 (before this chunk's output, so that the copy starts early)
+                bool lok = true;
+                if (lead && t >= 1 && t + 1 < ttot)
+                    lok = tc::mbar_wait(&bars.slot_free[b ^ 1], ((t - 1) >> 1) & 1, abort_flag) && load_image(t + 1);
+                if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) {
+                    stop = true;
+                    break;
+                }
                 // the state warps have chosen how chunk t is evaluated (outmode) ...
                 if (!out_wait(&bars.outq[b], ph_q[b])) {
                     stop = true;
@@ -1024,20 +1040,6 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
-                }
-                // chunk t's copy out of the ring completed long ago (the state warps are past it): its
-                // ring slot may be rewritten; the image of chunk t + 2 goes into slot b once the state
-                // warps are done with chunk t
-                bool lok = true;
-                if (lead && t + 2 < ttot) {
-                    int never = 0;
-                    tc::mbar_wait(&bars.full[b], (t >> 1) & 1, &never);
-                    tc::st_release_gpu(sched.consumed + kc, t + 1);
-                    lok = tc::mbar_wait(&bars.slot_free[b], (t >> 1) & 1, abort_flag) && load_image(t + 2);
-                }
-                if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) {
-                    stop = true;
-                    break;
                 }
             }
         }
@@ -1130,6 +1132,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 stop = true;
                 break;
             }
+            // chunk t is out of the ring (the copy has completed): its slot may take a later image
+            if (leader) tc::st_relaxed_gpu(sched.consumed + kc, t + 1);
             const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
             if (leader) {
                 // the output warps have read D1^T[b] of chunk t - 2
@@ -1280,7 +1284,7 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
         tc::mbar_init(&bars.m_wu, 1);
         tc::mbar_init(&bars.staged, 1);
         tc::mbar_init(&bars.staging_free, 1);
-        tc::mbar_init(&bars.raw_full, 1);
+        tc::mbar_init(&bars.raw_full, 2);
         tc::mbar_init(&bars.raw_free, 1);
         tc::mbar_init(&bars.fin, 1);
         tc::fence_mbar_init();
@@ -1342,7 +1346,7 @@ inline ChunkGrid chunk_grid(int64_t npairs, int nsm) {
     g.nprod = nsm - g.nchain;
     return g;
 }
-constexpr int kRing = 8;                 // ring slots per chain (workspace variant)
+constexpr int kRing = 12;                // ring slots per chain (workspace variant)
 constexpr int kMinRing = 3;
 constexpr int kMaxChains = 64;
 constexpr size_t kFlagsBytes = 4096 + (size_t)(kMaxChains * kRing + kMaxChains) * 4;   // order + flags

@@ -109,7 +109,7 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
  * Workspace kda_chunk_fwd needs, in bytes, for N sequences (B, or num_seqs with
  * cu_seqlens) of H heads: on the tensor-core path, about 7 KB of schedule
  * tables (ring flags, sequence order) and, for each of up to min(N * H, 64)
- * chains, a ring of 8 chunk images (73 KB each at d_v = 128, 65 KB at
+ * chains, a ring of 12 chunk images (73 KB each at d_v = 128, 65 KB at
  * d_v = 64) through which the CTAs that prepare the chunk operands hand them
  * to the CTA that runs the state recurrence; 0 on the fp32 path.  Pure host
  * computation, never fails for valid sizes.
@@ -161,7 +161,7 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
  * workspace_bytes.  Only the tensor-core path: dtype KDA_BF16, d_k == 128,
  * d_v in {64, 128}.  It allocates nothing (no cudaMalloc, no library
  * allocator).  Any number of (sequence, head) pairs fits: the chains' rings
- * are made shallower (down to 3 images) when the array cannot hold 8 each.
+ * are made shallower (down to 3 images) when the array cannot hold 12 each.
  *
  * The first call on a device looks up that device's copy of the array (with
  * the device current), so make that first call before any stream capture.
