@@ -363,7 +363,8 @@ def run_kda(args):
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps, "clocks": clocks, "decode": decode}
+                # per step: the schedule-table kernel and the chunk kernel
+                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
