@@ -105,8 +105,10 @@ template <int DV> struct Img {
 // ---- chain CTA shared memory ------------------------------------------------------------------
 template <int DV> struct ChainSmem {
     using I = Img<DV>;
-    // one slot of the image ring: A1 = [-W ; Qg] as two 16 KB k-blocks of 128 rows (rows 0-63 -W,
-    // rows 64-127 Qg; the B operand of S^T A1^T), then U^T, then Kd, P, gamma, flag in image order
+    // one slot of the three-slot image ring: A1 = [-W ; Qg] as two 16 KB k-blocks of 128 rows (rows
+    // 0-63 -W, rows 64-127 Qg; the B operand of S^T A1^T), then U^T, then Kd, P, gamma, flag in
+    // image order.  Once MMA1 of the slot's chunk has completed, A1 is dead and stages that chunk's
+    // output (DV / 64 blocks of [64 tokens x 64 values], fp32 or bf16, one TMA tensor store each).
     static constexpr int kA1 = 0;
     static constexpr int kUT = 2 * kChunk * kDK * 2;
     static constexpr int kKd = kUT + kChunk * DV * 2;
@@ -115,15 +117,13 @@ template <int DV> struct ChainSmem {
     static constexpr int kFlag = kKd + (I::kFlag - I::kKd);
     static constexpr int kTailBytes = I::kBytes - I::kKd;
     static constexpr int kSlotBytes = (kKd + kTailBytes + 1023) / 1024 * 1024;
+    static constexpr int kSlots = 3;
+    static_assert(kChunk * DV * 4 <= kUT - kA1, "output staging fits the dead A1 area");
     // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel quarter, k . q
-    static constexpr int kRedPk = 2 * kSlotBytes;
+    static constexpr int kRedPk = kSlots * kSlotBytes;
     static constexpr int kRedPq = kRedPk + 4 * 128 * 4;
     static constexpr int kRedKq = kRedPq + 4 * 128 * 4;
-    // output staging of a full chunk, double-buffered: DV / 64 blocks of [64 tokens x 64 values]
-    // (fp32 or bf16), written by a TMA tensor store per block
-    static constexpr int kOut = (kRedKq + 16 + 1023) / 1024 * 1024;
-    static constexpr int kOutBytes = kChunk * DV * 4;   // two buffers
-    static constexpr int kBytes = kOut + 2 * kOutBytes;
+    static constexpr int kBytes = kRedKq + 16;
 };
 
 // ---- prep CTA shared memory -------------------------------------------------------------------
@@ -356,7 +356,7 @@ struct ChunkCtx {
 // Mbarriers of one CTA (each role uses its own subset).
 struct ChunkBars {
     // chain: image slot full / free, MMA completions
-    uint64_t full[2], slot_free[2], mma1, mma2, mma3[2];
+    uint64_t full[3], slot_free[3], mma1, mma2, mma3[2];
     // chain: chunk evaluation mode handed to the output warps, TMEM accumulator read by them
     uint64_t outq[2], d1_free[2];
     int outmode[2];   // 0: no MMAs issued, 1: MMAs issued but evaluated exactly, 2: tensor output
@@ -901,7 +901,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
 //   D2^T = U~^T Kd                 (the state increment, transposed)
 //   D1^T[:, 64:128] += U~^T P^T    (so that columns 64-127 become O^T)
 // Warps 0-15 own the fp32 state: thread (warp w, lane l) holds value column j = 32 (w % 4) + l and key
-// channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Warps 16-19 store the outputs; lane 0 of warp 16
+// channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Warps 16-19 store the outputs; lane 1 of warp 16
 // also copies the chunk images out of the chain's ring.  Chain kc runs the pairs kc, kc + nchain, ...;
 // its chunks are numbered t across them (image slots, barrier phases and ring slots follow t).
 template <int DV, typename TO>
@@ -923,21 +923,24 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     if (warp >= kRoleWarps) {
         // ---- output and image warps 16-19: warp 16 + w reads TMEM lanes 32 w .. 32 w + 31, i.e. value
         //      columns j = 32 w + lane of O^T (columns 64-127 of D1^T[b]) once [. ; P] U~ completed,
-        //      and stages them for TMA tensor stores (double-buffered); lane 0 of warp 16 also copies
+        //      and stages them for TMA tensor stores (double-buffered); lane 1 of warp 16 copies
         //      the chunk images from the chain's ring in global memory into the two slots ----
         const int jo = (warp & 3) * 32 + lane;
         const bool jov = jo < DV;
         const bool lead = warp == kRoleWarps && lane == 0;
+        // the image copies are issued by another lane than the output stores: its flag waits then do
+        // not wait for the output stores still in flight
+        const bool lead_ld = warp == kRoleWarps && lane == 1;
         const uint32_t tlo = tc::tmem_lane_base(warp);
         constexpr uint32_t kOutThreads = kThreads - kRoleThreads;
         int last_load = -1;
-        auto load_image = [&](int t) -> bool {   // lane 0 of warp 16
+        auto load_image = [&](int t) -> bool {   // lane 1 of warp 16
             const int rs = kc * sched.ring + t % sched.ring;
             if (!tc::flag_wait_ge(sched.ready + rs, t + 1, abort_flag)) return false;
             tc::fence_async_global();
             const uint8_t *src = sched.rings + (size_t)rs * I::kStride;
-            uint8_t *slot = sm + (t & 1) * SM::kSlotBytes;
-            uint64_t *fb = &bars.full[t & 1];
+            uint8_t *slot = sm + (t % SM::kSlots) * SM::kSlotBytes;
+            uint64_t *fb = &bars.full[t % SM::kSlots];
             tc::mbar_arrive_expect_tx(fb, I::kBytes);
             tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
             tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
@@ -948,9 +951,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             last_load = t;
             return true;
         };
-        if (lead)
+        if (lead_ld)
             for (int t = 0; t < 2 && t < ttot; ++t)
                 if (!load_image(t)) break;
+        int stage_pending = -1;   // slot whose output store was issued, its read not yet confirmed
         // a wait by lane 0 of warp 16, whose outcome all four warps share (they leave together)
         auto out_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
             bool ok = true;
@@ -960,18 +964,27 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             return !failed;
         };
         uint32_t ph_q[2] = {0, 0}, ph3[2] = {0, 0};
-        int nstore = 0, t = 0;
+        int t = 0;
         bool stop = false;
         for (int pr = kc; pr < sched.npairs && !stop; pr += sched.nchain) {
             const PairInfo pi = pair_info(sched, pr);
             const int h = pi.h;
             for (int c = 0; c < pi.nchunks; ++c, ++t) {
-                const int b = t & 1;
-                // first the image of chunk t + 1, into slot b ^ 1 once the state warps are done with
-                // chunk t - 1 (before this chunk's output, so that the copy starts early)
+                const int b = t & 1, s3 = t % SM::kSlots;
+                // the previous chunk's output store has read its staging: that slot may be refilled
+                if (lead && stage_pending >= 0) {
+                    tc::bulk_wait_read_all();
+                    tc::mbar_arrive(&bars.slot_free[stage_pending]);
+                    stage_pending = -1;
+                }
+                // first the image of chunk t + 2, into the slot of chunk t - 1 once that slot is free
+                // (two chunks ahead of its use)
                 bool lok = true;
-                if (lead && t >= 1 && t + 1 < ttot)
-                    lok = tc::mbar_wait(&bars.slot_free[b ^ 1], ((t - 1) >> 1) & 1, abort_flag) && load_image(t + 1);
+                if (lead_ld && t + 2 < ttot) {
+                    const int sp2 = (t + 2) % SM::kSlots;
+                    lok = (t < 1 || tc::mbar_wait(&bars.slot_free[sp2], ((t - 1) / SM::kSlots) & 1, abort_flag)) &&
+                          load_image(t + 2);
+                }
                 if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) {
                     stop = true;
                     break;
@@ -995,12 +1008,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     const int64_t tok0 = pi.tok0(c);
                     const int L = pi.len(c);
                     const bool full = L == kChunk;
-                    TO *stage = reinterpret_cast<TO *>(sm + SM::kOut + (nstore & 1) * SM::kOutBytes);
-                    if (full) {
-                        // the stores issued from this buffer two chunks ago have read it
-                        if (lead) tc::bulk_wait_read_1();
-                        tc::named_sync(kBarOut, kOutThreads);
-                    }
+                    // staging: the slot's A1 area, dead since MMA1 of this chunk (before [. ; P] U~)
+                    TO *stage = reinterpret_cast<TO *>(sm + s3 * SM::kSlotBytes + SM::kA1);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
                         float o[32];
@@ -1033,22 +1042,24 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                                 tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0),
                                                  stage + blk * (kChunk * 64));
                             tc::bulk_commit();
+                            stage_pending = s3;
                         }
-                        ++nstore;
                     }
                 } else {
                     tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
                 }
+                // no output store reads this chunk's slot (partial chunk, or no tensor output)
+                if (lead && stage_pending != s3) tc::mbar_arrive(&bars.slot_free[s3]);
             }
         }
-        if (lead) {
-            tc::bulk_wait_all();   // every output store has completed before the CTA leaves
+        if (lead) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
+        if (lead_ld) {
             // no image copy may still be in flight either
             int never = 0;
-            for (int tt = (last_load >= 1 ? last_load - 1 : 0); tt <= last_load; ++tt)
-                tc::mbar_wait(&bars.full[tt & 1], (tt >> 1) & 1, &never);
+            for (int tt = (last_load >= 2 ? last_load - 2 : 0); tt <= last_load; ++tt)
+                tc::mbar_wait(&bars.full[tt % SM::kSlots], (tt / SM::kSlots) & 1, &never);
         }
         return;
     }
@@ -1123,12 +1134,12 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         tc::tc_fence_before();
         bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
         for (int c = 0; c < pi.nchunks; ++c, ++t) {
-            const int s = t & 1, b = t & 1;
+            const int s = t % SM::kSlots, b = t & 1;
             const int64_t tok0 = pi.tok0(c);
             const int L = pi.len(c);
             const uint8_t *slot = sm + s * SM::kSlotBytes;
             const uint32_t sslot = sbase + s * SM::kSlotBytes;
-            if (!role_wait(&bars.full[s], (t >> 1) & 1, leader, kBarRole, kRoleThreads, abort_flag)) {
+            if (!role_wait(&bars.full[s], (t / SM::kSlots) & 1, leader, kBarRole, kRoleThreads, abort_flag)) {
                 stop = true;
                 break;
             }
@@ -1154,6 +1165,27 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 }
             }
             if (!flagged) {
+                // while MMA1 runs: D2^T = S^T Diag(gamma) in fp32, which MMA2 then accumulates onto
+                // (D2^T was last read by the previous chunk's state update)
+                {
+                    const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t u[16];
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 gg = gam4[4 * h2 + i4];
+                            const int i = 16 * h2 + 4 * i4;
+                            u[4 * i4] = __float_as_uint(gg.x * S[i]);
+                            u[4 * i4 + 1] = __float_as_uint(gg.y * S[i + 1]);
+                            u[4 * i4 + 2] = __float_as_uint(gg.z * S[i + 2]);
+                            u[4 * i4 + 3] = __float_as_uint(gg.w * S[i + 3]);
+                        }
+                        tc::tmem_st16(tmem + tl + kTmD2 + c0 + 16 * h2, u);
+                    }
+                    tc::tmem_st_wait();
+                    tc::tc_fence_before();
+                }
                 if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) {
                     stop = true;
                     break;
@@ -1190,13 +1222,13 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
                 if (leader) {
                     tc::tc_fence_after();
-                    // ---- D2^T = U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
+                    // ---- D2^T += U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
                     constexpr uint32_t id2 = tc::make_idesc(128, 128, tc::kF16, false, true);
                     constexpr uint32_t id3 = tc::make_idesc(128, kChunk, tc::kF16, false, false);
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk)
                         tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + SM::kKd, kChunk, kk),
-                                       id2, kk > 0);
+                                       id2, true);
                     tc::mma_commit(&bars.mma2);
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk)
@@ -1212,22 +1244,9 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 }
                 ph2 ^= 1u;
                 if (!bad) {
-                    // ---- S^T = S^T Diag(gamma) + D2^T ----
-                    const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
-                    {
-                        float d[32];
-                        tc::tmem_ld32(tmem + tl + kTmD2 + c0, d);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 gg = gam4[i4];
-                            const int i = 4 * i4;
-                            S[i] = fmaf(gg.x, S[i], d[i]);
-                            S[i + 1] = fmaf(gg.y, S[i + 1], d[i + 1]);
-                            S[i + 2] = fmaf(gg.z, S[i + 2], d[i + 2]);
-                            S[i + 3] = fmaf(gg.w, S[i + 3], d[i + 3]);
-                        }
-                    }
+                    // ---- S^T = D2^T = S^T Diag(gamma) + U~^T Kd ----
+                    tc::tmem_ld32(tmem + tl + kTmD2 + c0, S);
+                    tc::tmem_ld_wait();
                     const bool big = write_state_operand();
                     tc::tc_fence_before();
                     force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
@@ -1268,10 +1287,11 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
     const bool is_chain = static_cast<int>(blockIdx.x) < sched.nchain;
     if (tid == 0) {
         if (!is_chain) s_tmax = chain_tmax(sched);
-        tc::mbar_init(&bars.full[0], 1);
-        tc::mbar_init(&bars.full[1], 1);
-        tc::mbar_init(&bars.slot_free[0], 1);
-        tc::mbar_init(&bars.slot_free[1], 1);
+        for (int i = 0; i < 3; ++i) {
+            tc::mbar_init(&bars.full[i], 1);
+            // the state warps are done with the slot's chunk; its output store has read the slot
+            tc::mbar_init(&bars.slot_free[i], 2);
+        }
         tc::mbar_init(&bars.mma1, 1);
         tc::mbar_init(&bars.mma2, 1);
         tc::mbar_init(&bars.mma3[0], 1);
