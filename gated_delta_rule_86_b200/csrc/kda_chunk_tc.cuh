@@ -360,6 +360,9 @@ struct ChunkBars {
     // chain: chunk evaluation mode handed to the output warps, TMEM accumulator read by them
     uint64_t outq[2], d1_free[2];
     int outmode[2];   // 0: no MMAs issued, 1: MMAs issued but evaluated exactly, 2: tensor output
+    // chain: a state warp's own wait for MMA1 / MMA2 ran out (set before the barrier that follows
+    // the wait, read after it, so that every state warp leaves at the same point)
+    int fail1, fail2;
     // prep: MMA completions, staging image and raw input tiles
     uint64_t m_ap, m_wu, staged, staging_free, raw_full, raw_free;
     uint64_t fin;
@@ -1186,10 +1189,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     tc::tmem_st_wait();
                     tc::tc_fence_before();
                 }
-                if (!role_wait(&bars.mma1, ph1, leader, kBarRole, kRoleThreads, abort_flag)) {
-                    stop = true;
-                    break;
-                }
+                // every state warp waits for MMA1 itself (no barrier round); a timeout is shared through
+                // the barrier after the U~ epilogue
+                if (!tc::mbar_wait(&bars.mma1, ph1, abort_flag)) *reinterpret_cast<volatile int *>(&bars.fail1) = 1;
+                tc::tc_fence_after();
                 ph1 ^= 1u;
                 // ---- U~^T = U^T + (-W S)^T (tokens 16 qd + [0, 16)) -> fp16 A operand in TMEM ----
                 bool mybad = force_exact;
@@ -1220,6 +1223,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 }
                 tc::tc_fence_before();
                 const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
+                if (*reinterpret_cast<volatile int *>(&bars.fail1)) {
+                    stop = true;
+                    break;
+                }
                 if (leader) {
                     tc::tc_fence_after();
                     // ---- D2^T += U~^T Kd;  D1^T[b][:, 64:128] += U~^T P^T ----
@@ -1238,10 +1245,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     bars.outmode[b] = bad ? 1 : 2;   // MMAs issued; O^T is the output unless evaluated exactly
                     tc::mbar_arrive(&bars.outq[b]);
                 }
-                if (!role_wait(&bars.mma2, ph2, leader, kBarRole, kRoleThreads, abort_flag)) {
-                    stop = true;
-                    break;
-                }
+                if (!tc::mbar_wait(&bars.mma2, ph2, abort_flag)) *reinterpret_cast<volatile int *>(&bars.fail2) = 1;
+                tc::tc_fence_after();
                 ph2 ^= 1u;
                 if (!bad) {
                     // ---- S^T = D2^T = S^T Diag(gamma) + U~^T Kd ----
@@ -1250,6 +1255,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     const bool big = write_state_operand();
                     tc::tc_fence_before();
                     force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+                    if (*reinterpret_cast<volatile int *>(&bars.fail2)) {
+                        stop = true;
+                        break;
+                    }
                     if (leader) tc::mbar_arrive(&bars.slot_free[s]);   // done with the slot
                     continue;
                 }
@@ -1258,6 +1267,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const bool big = exact_chunk(tok0, L);
             tc::tc_fence_before();
             force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+            if (*reinterpret_cast<volatile int *>(&bars.fail2)) {
+                stop = true;
+                break;
+            }
             if (leader) tc::mbar_arrive(&bars.slot_free[s]);
         }
         if (!stop && final_state && *abort_flag == 0 && jv) {
@@ -1309,6 +1322,8 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
         tc::mbar_init(&bars.fin, 1);
         tc::fence_mbar_init();
         abort_flag = 0;
+        bars.fail1 = 0;
+        bars.fail2 = 0;
     }
     const uint32_t ncols = is_chain ? kTmChainCols : kTmPrepCols;
     if (warp == 0) {
