@@ -278,9 +278,9 @@ def run_kda(args):
     achieved_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
     dense_flops = token_heads * (12 * w.chunk * w.dk + 6 * w.dk * w.dv)
     # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
-    # this kernel on the B=1, H=32, T=16384 case (831.5 MB), scaled to the launch by tokens (the
+    # this kernel on the B=1, H=32, T=16384 case (842.2 MB), scaled to the launch by tokens (the
     # 4 MB of state traffic does not scale); only valid for the 64K workload of this kernel build.
-    traffic = (831.5e6 - 4.2e6) * (tokens / 16384) + 4.2e6 if (w.B, w.H, w.T) == (1, 32, 65536) else None
+    traffic = (842.2e6 - 4.2e6) * (tokens / 16384) + 4.2e6 if (w.B, w.H, w.T) == (1, 32, 65536) else None
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                 "peak_source": f"{peaks_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"

@@ -12,7 +12,8 @@ KDA_F32, KDA_BF16 = 0, 1
 
 # every symbol include/kda.h declares
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_static_ws", "kda_recurrent_fwd",
-            "kda_decode_step", "kda_status_string", "kda_get_last_device_error", "kda_version")
+            "kda_decode_step", "gdn_chunk_fwd", "gdn_recurrent_fwd", "gdn_decode_step", "kda_status_string",
+            "kda_get_last_device_error", "kda_version")
 
 _lib = None
 
@@ -37,15 +38,20 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, f32p = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     prefill_args = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, i32, i32]
-    lib.kda_chunk_fwd.argtypes = prefill_args + [i32, ctypes.c_int, ctypes.c_int, vp, f32p, vp, ctypes.c_size_t, vp]
-    lib.kda_chunk_fwd.restype = ctypes.c_int
+    for name in ("kda_chunk_fwd", "gdn_chunk_fwd"):
+        fn = getattr(lib, name)
+        fn.argtypes = prefill_args + [i32, ctypes.c_int, ctypes.c_int, vp, f32p, vp, ctypes.c_size_t, vp]
+        fn.restype = ctypes.c_int
     lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_int
-    lib.kda_recurrent_fwd.argtypes = prefill_args + [ctypes.c_int, ctypes.c_int, vp, f32p, vp]
-    lib.kda_recurrent_fwd.restype = ctypes.c_int
-    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,
-                                    vp]
-    lib.kda_decode_step.restype = ctypes.c_int
+    for name in ("kda_recurrent_fwd", "gdn_recurrent_fwd"):
+        fn = getattr(lib, name)
+        fn.argtypes = prefill_args + [ctypes.c_int, ctypes.c_int, vp, f32p, vp]
+        fn.restype = ctypes.c_int
+    for name in ("kda_decode_step", "gdn_decode_step"):
+        fn = getattr(lib, name)
+        fn.argtypes = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int, vp]
+        fn.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_get_last_device_error.argtypes = [vp]

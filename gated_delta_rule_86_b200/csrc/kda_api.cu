@@ -27,10 +27,12 @@ kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR
 kda_status check_prefill(const void *q, const void *k, const void *v, const void *la, const void *beta,
                          const float *init_state, const int32_t *cu, int32_t num_seqs, int32_t B, int32_t T,
                          int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, kda_dtype out_dtype,
-                         const void *out, const float *final_state) {
+                         const void *out, const float *final_state, int gate) {
     if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
-    // token tensors may be empty (NULL) only when there are no tokens
-    if (T > 0 && (!q || !k || !v || !la || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    // token tensors may be empty (NULL) only when there are no tokens; a per-head gate may be NULL
+    // (no decay)
+    if (T > 0 && (!q || !k || !v || (gate == kda::kGateChannel && !la) || !beta || !out))
+        return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (cu) {
@@ -56,27 +58,39 @@ kda_status check_prefill(const void *q, const void *k, const void *v, const void
     return KDA_OK;
 }
 
-template <typename TIO, typename TOUT>
-cudaError_t dispatch_recurrent_t(const void *q, const void *k, const void *v, const void *la, const void *beta,
+template <typename TIO, typename TOUT, int GK>
+cudaError_t dispatch_recurrent_g(const void *q, const void *k, const void *v, const void *la, const void *beta,
                                  const float *s0, const int32_t *cu, int ns, int B, int T, int H, int dk, int dv,
                                  void *out, float *fs, cudaStream_t st) {
-    if (dk == 64) return kda::launch_recurrent<64, TIO, TOUT>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
-    return kda::launch_recurrent<128, TIO, TOUT>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
+    if (dk == 64)
+        return kda::launch_recurrent<64, TIO, TOUT, GK>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
+    return kda::launch_recurrent<128, TIO, TOUT, GK>(q, k, v, la, beta, s0, cu, ns, B, T, H, dv, out, fs, st);
 }
 
-cudaError_t dispatch_recurrent(kda_dtype dt, kda_dtype odt, const void *q, const void *k, const void *v,
-                               const void *la, const void *beta, const float *s0, const int32_t *cu, int ns, int B,
-                               int T, int H, int dk, int dv, void *out, float *fs, cudaStream_t st) {
-    if (dt == KDA_F32 && odt == KDA_F32)
-        return dispatch_recurrent_t<float, float>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs, st);
-    if (dt == KDA_F32)
-        return dispatch_recurrent_t<float, __nv_bfloat16>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs,
-                                                          st);
-    if (odt == KDA_F32)
-        return dispatch_recurrent_t<__nv_bfloat16, float>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs,
-                                                          st);
-    return dispatch_recurrent_t<__nv_bfloat16, __nv_bfloat16>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
+template <typename TIO, typename TOUT>
+cudaError_t dispatch_recurrent_t(int gate, const void *q, const void *k, const void *v, const void *la,
+                                 const void *beta, const float *s0, const int32_t *cu, int ns, int B, int T, int H,
+                                 int dk, int dv, void *out, float *fs, cudaStream_t st) {
+    if (gate == kda::kGateHead)
+        return dispatch_recurrent_g<TIO, TOUT, kda::kGateHead>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
+                                                               fs, st);
+    return dispatch_recurrent_g<TIO, TOUT, kda::kGateChannel>(q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
                                                               fs, st);
+}
+
+cudaError_t dispatch_recurrent(int gate, kda_dtype dt, kda_dtype odt, const void *q, const void *k,
+                               const void *v, const void *la, const void *beta, const float *s0, const int32_t *cu,
+                               int ns, int B, int T, int H, int dk, int dv, void *out, float *fs, cudaStream_t st) {
+    if (dt == KDA_F32 && odt == KDA_F32)
+        return dispatch_recurrent_t<float, float>(gate, q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out, fs, st);
+    if (dt == KDA_F32)
+        return dispatch_recurrent_t<float, __nv_bfloat16>(gate, q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
+                                                          fs, st);
+    if (odt == KDA_F32)
+        return dispatch_recurrent_t<__nv_bfloat16, float>(gate, q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv, out,
+                                                          fs, st);
+    return dispatch_recurrent_t<__nv_bfloat16, __nv_bfloat16>(gate, q, k, v, la, beta, s0, cu, ns, B, T, H, dk, dv,
+                                                              out, fs, st);
 }
 
 // Handoff buffer of kda_chunk_fwd_static_ws: a fixed array in device memory,
@@ -130,16 +144,114 @@ kda_status kda_get_last_device_error(void *stream) {
     return word == 0 ? KDA_OK : static_cast<kda_status>(word);
 }
 
+}  // extern "C"
+
+namespace {
+
+kda_status recurrent_impl(int gate, const void *q, const void *k, const void *v, const void *la, const void *beta,
+                          const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                          int32_t T, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype, kda_dtype out_dtype,
+                          void *out, float *final_state, void *stream) {
+    kda_status s = check_prefill(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v, dtype,
+                                 out_dtype, out, final_state, gate);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return from_cuda(dispatch_recurrent(gate, dtype, out_dtype, q, k, v, la, beta, init_state, cu_seqlens, num_seqs,
+                                        B, T, H, d_k, d_v, out, final_state, st));
+}
+
+// Shared by kda_chunk_fwd / gdn_chunk_fwd (workspace != NULL) and kda_chunk_fwd_static_ws
+// (workspace == NULL: the built-in array).
+kda_status chunk_impl(int gate, bool static_ws, const void *q, const void *k, const void *v, const void *la,
+                      const void *beta, const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs,
+                      int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
+                      kda_dtype out_dtype, void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+    kda_status s = check_prefill(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v, dtype,
+                                 out_dtype, out, final_state, gate);
+    if (s != KDA_OK) return s;
+    if (chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (chunk != 64) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (static_ws) {
+        if (dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
+    } else if (dtype == KDA_F32) {
+        // fp32 I/O asks for fp32 accuracy, which bf16 tensor-core operands
+        // cannot give: evaluate on CUDA cores with the fp32 state.
+        return from_cuda(dispatch_recurrent(gate, dtype, out_dtype, q, k, v, la, beta, init_state, cu_seqlens,
+                                            num_seqs, B, T, H, d_k, d_v, out, final_state, st));
+    }
+    if (d_k != 128) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
+    const int64_t pairs = (int64_t)(cu_seqlens ? num_seqs : B) * H;
+    if (static_ws) {
+        // the schedule tables and rings of at least kMinRing images for each chain always fit
+        const int64_t chains = pairs < kda::kMaxChains ? pairs : kda::kMaxChains;
+        if (kda::flags_region_bytes() + (size_t)chains * kda::kMinRing * kda::img_stride(d_v) > KDA_STATIC_WS_BYTES)
+            return KDA_ERR_UNSUPPORTED;
+        s = static_ws_address(&workspace);
+        if (s != KDA_OK) return s;
+        workspace_bytes = KDA_STATIC_WS_BYTES;
+    } else {
+        const size_t need = kda::chunk_tc_workspace_bytes(pairs, d_v);
+        if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
+    }
+    if (out_dtype == KDA_F32)
+        return from_cuda(kda::launch_chunk_tc<float>(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T, H,
+                                                     d_v, out, final_state, workspace, workspace_bytes, st, gate));
+    return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T,
+                                                         H, d_v, out, final_state, workspace, workspace_bytes, st,
+                                                         gate));
+}
+
+template <int GK>
+kda_status decode_impl(const void *q, const void *k, const void *v, const void *la, const void *beta, float *state,
+                       void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                       kda_dtype out_dtype, void *stream) {
+    if (!q || !k || !v || (GK == kda::kGateChannel && !la) || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, la, beta, state, out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+#define KDA_DECODE_CASE(DK, DV)                                                                                 \
+    if (d_k == DK && d_v == DV) {                                                                               \
+        if (dtype == KDA_F32)                                                                                   \
+            e = out_dtype == KDA_F32                                                                            \
+                    ? kda::launch_decode<DK, DV, float, float, GK>(q, k, v, la, beta, state, out, B, H, st)     \
+                    : kda::launch_decode<DK, DV, float, __nv_bfloat16, GK>(q, k, v, la, beta, state, out, B, H, \
+                                                                           st);                                 \
+        else                                                                                                    \
+            e = out_dtype == KDA_F32                                                                            \
+                    ? kda::launch_decode<DK, DV, __nv_bfloat16, float, GK>(q, k, v, la, beta, state, out, B, H, \
+                                                                           st)                                  \
+                    : kda::launch_decode<DK, DV, __nv_bfloat16, __nv_bfloat16, GK>(q, k, v, la, beta, state,    \
+                                                                                   out, B, H, st);              \
+        return from_cuda(e);                                                                                    \
+    }
+    KDA_DECODE_CASE(128, 128)
+    KDA_DECODE_CASE(128, 64)
+    KDA_DECODE_CASE(64, 128)
+    KDA_DECODE_CASE(64, 64)
+#undef KDA_DECODE_CASE
+    return KDA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
 kda_status kda_recurrent_fwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
                              const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
                              int32_t T, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
                              kda_dtype out_dtype, void *out, float *final_state, void *stream) {
-    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
-                                 dtype, out_dtype, out, final_state);
-    if (s != KDA_OK) return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return from_cuda(dispatch_recurrent(dtype, out_dtype, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                        B, T, H, d_k, d_v, out, final_state, st));
+    return recurrent_impl(kda::kGateChannel, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k,
+                          d_v, dtype, out_dtype, out, final_state, stream);
 }
 
 kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
@@ -157,28 +269,8 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                          int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
                          kda_dtype out_dtype, void *out, float *final_state, void *workspace, size_t workspace_bytes,
                          void *stream) {
-    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
-                                 dtype, out_dtype, out, final_state);
-    if (s != KDA_OK) return s;
-    if (chunk < 1) return KDA_ERR_INVALID_ARG;
-    if (chunk != 64) return KDA_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (dtype == KDA_F32) {
-        // fp32 I/O asks for fp32 accuracy, which bf16 tensor-core operands
-        // cannot give: evaluate on CUDA cores with the fp32 state.
-        return from_cuda(dispatch_recurrent(dtype, out_dtype, q, k, v, log_alpha, beta, init_state, cu_seqlens,
-                                            num_seqs, B, T, H, d_k, d_v, out, final_state, st));
-    }
-    if (d_k != 128) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
-    const size_t need = kda::chunk_tc_workspace_bytes((int64_t)(cu_seqlens ? num_seqs : B) * H, d_v);
-    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
-    if (out_dtype == KDA_F32)
-        return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
-                                                     T, H, d_v, out, final_state, workspace, workspace_bytes, st));
-    return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                                         B, T, H, d_v, out, final_state, workspace, workspace_bytes,
-                                                         st));
+    return chunk_impl(kda::kGateChannel, false, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H,
+                      d_k, d_v, chunk, dtype, out_dtype, out, final_state, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, const void *log_alpha,
@@ -186,64 +278,38 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
                                    int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
                                    int32_t chunk, kda_dtype dtype, kda_dtype out_dtype, void *out,
                                    float *final_state, void *stream) {
-    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
-                                 dtype, out_dtype, out, final_state);
-    if (s != KDA_OK) return s;
-    if (chunk < 1) return KDA_ERR_INVALID_ARG;
-    if (chunk != 64 || dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
-    // the schedule tables and rings of at least kMinRing images for each chain always fit
-    const int64_t pairs = (int64_t)(cu_seqlens ? num_seqs : B) * H;
-    const int64_t chains = pairs < kda::kMaxChains ? pairs : kda::kMaxChains;
-    if (kda::flags_region_bytes() + (size_t)chains * kda::kMinRing * kda::img_stride(d_v) > KDA_STATIC_WS_BYTES)
-        return KDA_ERR_UNSUPPORTED;
-    void *ws = nullptr;
-    s = static_ws_address(&ws);
-    if (s != KDA_OK) return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (out_dtype == KDA_F32)
-        return from_cuda(kda::launch_chunk_tc<float>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
-                                                     T, H, d_v, out, final_state, ws, KDA_STATIC_WS_BYTES, st));
-    return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
-                                                         B, T, H, d_v, out, final_state, ws, KDA_STATIC_WS_BYTES,
-                                                         st));
+    return chunk_impl(kda::kGateChannel, true, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H,
+                      d_k, d_v, chunk, dtype, out_dtype, out, final_state, nullptr, 0, stream);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
                            float *state, void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
                            kda_dtype out_dtype, void *stream) {
-    if (!q || !k || !v || !log_alpha || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
-    if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
-    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, log_alpha, beta, state, out};
-    for (const void *p : ptrs)
-        if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
-    if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)B * H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-#define KDA_DECODE_CASE(DK, DV)                                                                            \
-    if (d_k == DK && d_v == DV) {                                                                          \
-        if (dtype == KDA_F32)                                                                              \
-            e = out_dtype == KDA_F32                                                                       \
-                    ? kda::launch_decode<DK, DV, float, float>(q, k, v, log_alpha, beta, state, out, B, H, st) \
-                    : kda::launch_decode<DK, DV, float, __nv_bfloat16>(q, k, v, log_alpha, beta, state, out, B, \
-                                                                       H, st);                             \
-        else                                                                                               \
-            e = out_dtype == KDA_F32                                                                       \
-                    ? kda::launch_decode<DK, DV, __nv_bfloat16, float>(q, k, v, log_alpha, beta, state, out, B, \
-                                                                       H, st)                              \
-                    : kda::launch_decode<DK, DV, __nv_bfloat16, __nv_bfloat16>(q, k, v, log_alpha, beta, state, \
-                                                                               out, B, H, st);             \
-        return from_cuda(e);                                                                               \
-    }
-    KDA_DECODE_CASE(128, 128)
-    KDA_DECODE_CASE(128, 64)
-    KDA_DECODE_CASE(64, 128)
-    KDA_DECODE_CASE(64, 64)
-#undef KDA_DECODE_CASE
-    return KDA_ERR_UNSUPPORTED;
+    return decode_impl<kda::kGateChannel>(q, k, v, log_alpha, beta, state, out, B, H, d_k, d_v, dtype, out_dtype,
+                                          stream);
+}
+
+kda_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const void *log_g, const void *beta,
+                         const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
+                         kda_dtype out_dtype, void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    return chunk_impl(kda::kGateHead, false, q, k, v, log_g, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k,
+                      d_v, chunk, dtype, out_dtype, out, final_state, workspace, workspace_bytes, stream);
+}
+
+kda_status gdn_recurrent_fwd(const void *q, const void *k, const void *v, const void *log_g, const void *beta,
+                             const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                             int32_t T, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                             kda_dtype out_dtype, void *out, float *final_state, void *stream) {
+    return recurrent_impl(kda::kGateHead, q, k, v, log_g, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
+                          dtype, out_dtype, out, final_state, stream);
+}
+
+kda_status gdn_decode_step(const void *q, const void *k, const void *v, const void *log_g, const void *beta,
+                           float *state, void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                           kda_dtype out_dtype, void *stream) {
+    return decode_impl<kda::kGateHead>(q, k, v, log_g, beta, state, out, B, H, d_k, d_v, dtype, out_dtype, stream);
 }
 
 }  // extern "C"

@@ -403,9 +403,10 @@ __device__ __forceinline__ bool first_item(const ChunkSched &s, int tmax, int j,
     return next_item(s, tmax, it);
 }
 
-template <int DV>
+template <int DV, int GK>
 __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, const ChunkSched &sched, int j,
-                                          int tmax, const RowMaps &maps, const __nv_bfloat16 *beta) {
+                                          int tmax, const RowMaps &maps, const __nv_bfloat16 *log_g,
+                                          const __nv_bfloat16 *beta) {
     using SM = PrepSmem<DV>;
     using I = Img<DV>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -456,10 +457,12 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             const int64_t tok0 = have ? it.pi.tok0(it.c) : 0;
             const int L = have ? it.pi.len(it.c) : -1, h = it.pi.h;
             if (lane == 0) {
-                tc::mbar_arrive_expect_tx(&bars.raw_full, have ? SM::kRawBytes : 0);
+                // a per-head gate comes as 64 scalars (below) instead of a log_alpha tile
+                constexpr uint32_t kTileBytes = GK == kGateChannel ? SM::kRawBytes : SM::kRawBytes - SM::kTile;
+                tc::mbar_arrive_expect_tx(&bars.raw_full, have ? kTileBytes : 0);
                 if (have) {
                     const int t = static_cast<int>(tok0);
-                    tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
+                    if constexpr (GK == kGateChannel) tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
@@ -468,6 +471,12 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             float *bdst = sBetaIn + (kl & 1) * kChunk;
             bdst[lane] = (lane < L) ? __bfloat162float(beta[(tok0 + lane) * H + h]) : 0.f;
             bdst[32 + lane] = (32 + lane < L) ? __bfloat162float(beta[(tok0 + 32 + lane) * H + h]) : 0.f;
+            if constexpr (GK == kGateHead) {   // fp32 log-decays of the 64 tokens, in place of the tile
+                float *gdst = reinterpret_cast<float *>(sm + SM::kRawG);
+                gdst[lane] = (lane < L) ? gate_log<GK>(log_g, (size_t)(tok0 + lane) * H + h, kDK, 0) : 0.f;
+                gdst[32 + lane] =
+                    (32 + lane < L) ? gate_log<GK>(log_g, (size_t)(tok0 + 32 + lane) * H + h, kDK, 0) : 0.f;
+            }
             if (lane == 0) sLenIn[kl & 1] = L;
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars.raw_full);
@@ -531,9 +540,15 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = tg * 2 + rr;
                 float g8[8];
-                const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
-                                        : make_uint4(0, 0, 0, 0);
-                unpack8(raw, g8);
+                if constexpr (GK == kGateChannel) {
+                    const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
+                                            : make_uint4(0, 0, 0, 0);
+                    unpack8(raw, g8);
+                } else {   // one decay for every channel
+                    const float gs = r < L ? reinterpret_cast<const float *>(sm + SM::kRawG)[r] : 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) g8[i] = gs;
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     run[i] += g8[i];
@@ -907,7 +922,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
 // channels [32 (w / 4), 32 (w / 4) + 32) of S^T.  Warps 16-19 store the outputs; lane 1 of warp 16
 // also copies the chunk images out of the chain's ring.  Chain kc runs the pairs kc, kc + nchain, ...;
 // its chunks are numbered t across them (image slots, barrier phases and ring slots follow t).
-template <int DV, typename TO>
+template <int DV, typename TO, int GK>
 __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, const ChunkSched &sched, int kc,
                                            const RowMaps &maps, const __nv_bfloat16 *q,
                                            const __nv_bfloat16 *k, const __nv_bfloat16 *v,
@@ -1097,13 +1112,16 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     auto exact_chunk = [&](int64_t tok0, int L) -> bool {
         for (int r = 0; r < L; ++r) {
             const int64_t trow = (tok0 + r) * H + h;
-            const __nv_bfloat16 *gr = log_alpha + trow * kDK + c0, *kr = k + trow * kDK + c0,
-                                *qr = q + trow * kDK + c0;
+            // a per-head gate: the same log-decay for every channel (none when log_g is null)
+            constexpr int gstride = GK == kGateChannel ? 1 : 0;
+            const __nv_bfloat16 *gr = log_alpha + (GK == kGateChannel ? trow * kDK + c0 : trow),
+                                *kr = k + trow * kDK + c0, *qr = q + trow * kDK + c0;
+            const bool has_gate = GK == kGateChannel || log_alpha != nullptr;
             float pk = 0.f, pq = 0.f, kq = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = expf(__bfloat162float(gr[i])), kk = __bfloat162float(kr[i]),
-                            qq = __bfloat162float(qr[i]);
+                const float a = has_gate ? expf(__bfloat162float(gr[i * gstride])) : 1.f,
+                            kk = __bfloat162float(kr[i]), qq = __bfloat162float(qr[i]);
                 S[i] *= a;
                 pk = fmaf(S[i], kk, pk);
                 pq = fmaf(S[i], qq, pq);
@@ -1282,7 +1300,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
 }
 
 // ====================================== kernel and launch ==========================================
-template <int DV, typename TO>
+template <int DV, typename TO, int GK>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant__ ChunkSched sched,
                     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -1340,10 +1358,10 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
     cx.tmem = tmem_base_sh;
     cx.abort_flag = &abort_flag;
     if (is_chain)
-        chain_role<DV, TO>(cx, bars, sched, blockIdx.x, maps, q, k, v, log_alpha, beta, init_state, out,
-                           final_state);
+        chain_role<DV, TO, GK>(cx, bars, sched, blockIdx.x, maps, q, k, v, log_alpha, beta, init_state, out,
+                               final_state);
     else
-        prep_role<DV>(cx, bars, sched, blockIdx.x - sched.nchain, s_tmax, maps, beta);
+        prep_role<DV, GK>(cx, bars, sched, blockIdx.x - sched.nchain, s_tmax, maps, log_alpha, beta);
 
     tc::tc_fence_before();
     __syncthreads();
@@ -1441,12 +1459,12 @@ inline int device_sm_count() {
 
 // Launches the schedule-table kernel and the chunk kernel.  `ws_bytes` bounds the ring depth: the
 // workspace holds the schedule tables and nchain rings of `ring` images (kMinRing <= ring <= kRing).
-template <int DV, typename TO>
+template <int DV, typename TO, int GK>
 cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, const void *la, const void *beta,
                                const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H,
                                void *out, float *final_state, void *workspace, size_t ws_bytes,
                                cudaStream_t stream) {
-    auto kern = kda_chunk_tc_kernel<DV, TO>;
+    auto kern = kda_chunk_tc_kernel<DV, TO, GK>;
     const int smem = chunk_smem_bytes<DV>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -1466,7 +1484,8 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
     memset(&maps, 0, sizeof(maps));
     const int64_t tokens = (int64_t)B * T;
     if (tokens > 0) {   // with no tokens no chunk is loaded and the maps stay unused
-        if (!encode_row_map(&maps.g, la, kDK, H, tokens) || !encode_row_map(&maps.k, k, kDK, H, tokens) ||
+        if ((GK == kGateChannel && !encode_row_map(&maps.g, la, kDK, H, tokens)) ||
+            !encode_row_map(&maps.k, k, kDK, H, tokens) ||
             !encode_row_map(&maps.q, q, kDK, H, tokens) || !encode_row_map(&maps.v, v, DV, H, tokens) ||
             !encode_row_map(&maps.o, out, DV, H, tokens, 64,
                             sizeof(TO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -1510,15 +1529,23 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
                               init_state, static_cast<TO *>(out), final_state);
 }
 
+// `la`: log_alpha [tokens][H][d_k] (gate kGateChannel), or the per-head log_g [tokens][H] or null
+// (kGateHead).
 template <typename TO>
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *la, const void *beta,
                             const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
-                            void *out, float *final_state, void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    if (DV == 64)
-        return launch_chunk_tc_dv<64, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
-                                          workspace, ws_bytes, stream);
-    return launch_chunk_tc_dv<128, TO>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out, final_state,
-                                       workspace, ws_bytes, stream);
+                            void *out, float *final_state, void *workspace, size_t ws_bytes, cudaStream_t stream,
+                            int gate = kGateChannel) {
+#define KDA_CHUNK_TC_CASE(DVV, GKK)                                                                          \
+    if (DV == DVV && gate == GKK)                                                                            \
+        return launch_chunk_tc_dv<DVV, TO, GKK>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out,   \
+                                                final_state, workspace, ws_bytes, stream);
+    KDA_CHUNK_TC_CASE(64, kGateChannel)
+    KDA_CHUNK_TC_CASE(128, kGateChannel)
+    KDA_CHUNK_TC_CASE(64, kGateHead)
+    KDA_CHUNK_TC_CASE(128, kGateHead)
+#undef KDA_CHUNK_TC_CASE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace kda

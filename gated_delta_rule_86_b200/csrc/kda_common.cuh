@@ -33,6 +33,19 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// How the decay gate is given.  kGateChannel: one log-decay per key channel, log_alpha
+// [..., d_k] (KDA).  kGateHead: one log-decay per head and token, log_g [...] (Gated DeltaNet, the
+// scalar-gate case of the same recurrence); a null log_g means no decay at all, alpha == 1
+// (DeltaNet).  The recurrence is otherwise the same.
+enum GateKind : int { kGateChannel = 0, kGateHead = 1 };
+
+// Log-decay of key channel c at gate row `row` (token * H + head, or batch * H + head).
+template <int GK, typename T>
+__device__ __forceinline__ float gate_log(const T *gate, size_t row, int dk, int c) {
+    if constexpr (GK == kGateChannel) return to_f32(gate[row * dk + c]);
+    else return gate ? to_f32(gate[row]) : 0.f;
+}
+
 // log2(e), used to turn exp(x) into exp2(x * log2e) for the ex2 unit.
 constexpr float kLog2e = 1.4426950408889634f;
 

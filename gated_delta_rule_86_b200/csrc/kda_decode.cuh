@@ -9,6 +9,9 @@
 // memory-bound decode regime that section 1 of "Linear Attention + Sparse
 // Attention: The Hybrid Architecture Trade-off for Large Models" describes.
 //
+// The gate is one log-decay per key channel (KDA) or, with GK = kGateHead, one per head (Gated
+// DeltaNet; a null gate gives DeltaNet, alpha == 1).
+//
 // Mapping: one CTA of 256 threads per (b, h).  Warp w owns state rows
 // [w*DK/8, (w+1)*DK/8); lane l owns columns [l*DV/32, (l+1)*DV/32), so a warp
 // reads and writes whole 128/256/512-byte rows (fully coalesced 16-byte
@@ -30,7 +33,7 @@ __device__ __forceinline__ void fvec_to_arr(const float2 &v, float *a) { a[0] = 
 __device__ __forceinline__ float4 arr_to_fvec4(const float *a) { return make_float4(a[0], a[1], a[2], a[3]); }
 __device__ __forceinline__ float2 arr_to_fvec2(const float *a) { return make_float2(a[0], a[1]); }
 
-template <int DK, int DV, typename TIO, typename TOUT>
+template <int DK, int DV, typename TIO, typename TOUT, int GK>
 __global__ void __launch_bounds__(256, 2)
 kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *__restrict__ v,
                   const TIO *__restrict__ log_alpha, const TIO *__restrict__ beta, float *__restrict__ state,
@@ -60,7 +63,7 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
     if (tid < DK) {
         s_q[tid] = to_f32(q[head * DK + tid]);
         s_k[tid] = to_f32(k[head * DK + tid]);
-        s_a[tid] = expf(to_f32(log_alpha[head * DK + tid]));
+        s_a[tid] = expf(gate_log<GK>(log_alpha, head, DK, tid));
     }
     if (tid >= 256 - DV) s_v[tid - (256 - DV)] = to_f32(v[head * DV + tid - (256 - DV)]);
     if (tid == 0) s_beta = to_f32(beta[head]);
@@ -123,11 +126,11 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
     }
 }
 
-template <int DK, int DV, typename TIO, typename TOUT>
+template <int DK, int DV, typename TIO, typename TOUT, int GK = kGateChannel>
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *beta,
                           float *state, void *out, int B, int H, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H);
-    kda_decode_kernel<DK, DV, TIO, TOUT><<<grid, 256, 0, stream>>>(
+    kda_decode_kernel<DK, DV, TIO, TOUT, GK><<<grid, 256, 0, stream>>>(
         static_cast<const TIO *>(q), static_cast<const TIO *>(k), static_cast<const TIO *>(v),
         static_cast<const TIO *>(la), static_cast<const TIO *>(beta), state, static_cast<TOUT *>(out));
     return cudaGetLastError();

@@ -8,6 +8,9 @@
 // the chunked algorithm; here it serves as the fp32-accurate prefill (fp32 I/O)
 // and as the token-by-token point of comparison for the chunked kernel.
 //
+// The gate is one log-decay per key channel (KDA) or, with GK = kGateHead, one per head and token
+// (Gated DeltaNet; a null gate gives DeltaNet, alpha == 1).
+//
 // Mapping: one CTA of 128 threads per (sequence, head, 32-column slice of d_v).
 // Lane l owns value column l of the slice; warp w owns key rows
 // [w*DK/4, (w+1)*DK/4), so each thread keeps DK/4 state values in registers.
@@ -45,7 +48,7 @@ __device__ __forceinline__ int longest_first_seq(const int32_t *cu, int num_seqs
 
 constexpr int kLongestFirstMaxSeqs = 1024;
 
-template <int DK, typename TIO, typename TOUT>
+template <int DK, typename TIO, typename TOUT, int GK>
 __global__ void __launch_bounds__(128)
 kda_recurrent_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *__restrict__ v,
                      const TIO *__restrict__ log_alpha, const TIO *__restrict__ beta,
@@ -89,7 +92,7 @@ kda_recurrent_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const
         if (tid < DK) {
             rq = to_f32(q[row * DK + tid]);
             rk = to_f32(k[row * DK + tid]);
-            ra = to_f32(log_alpha[row * DK + tid]);
+            ra = gate_log<GK>(log_alpha, row, DK, tid);
         }
         if (tid < 32) rv = to_f32(v[row * DV + slice * 32 + tid]);
         if (tid == 0) rb = to_f32(beta[row]);
@@ -151,13 +154,13 @@ kda_recurrent_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const
     }
 }
 
-template <int DK, typename TIO, typename TOUT>
+template <int DK, typename TIO, typename TOUT, int GK = kGateChannel>
 cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const void *la, const void *beta,
                              const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
                              void *out, float *final_state, cudaStream_t stream) {
     const int N = cu ? num_seqs : B;
     const unsigned grid = static_cast<unsigned>(N) * H * (DV / 32);
-    kda_recurrent_kernel<DK, TIO, TOUT><<<grid, 128, 0, stream>>>(
+    kda_recurrent_kernel<DK, TIO, TOUT, GK><<<grid, 128, 0, stream>>>(
         static_cast<const TIO *>(q), static_cast<const TIO *>(k), static_cast<const TIO *>(v),
         static_cast<const TIO *>(la), static_cast<const TIO *>(beta), init_state, cu, num_seqs, T, H, DV,
         static_cast<TOUT *>(out), final_state);

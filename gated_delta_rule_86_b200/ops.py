@@ -35,8 +35,8 @@ def _io_dtype(*ts):
     if dt not in _DTYPES:
         raise TypeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
     for t in ts:
-        if t.dtype != dt:
-            raise TypeError("q, k, v, log_alpha and beta must share one dtype")
+        if t is not None and t.dtype != dt:
+            raise TypeError("q, k, v, the gate and beta must share one dtype")
     return _DTYPES[dt]
 
 
@@ -46,18 +46,25 @@ def _to_device(t, dev):
     return t.to(dev, non_blocking=True)
 
 
-def _prefill_prepare(q, k, v, log_alpha, beta, initial_state, cu_seqlens):
+def _prefill_prepare(q, k, v, log_alpha, beta, initial_state, cu_seqlens, per_head_gate=False):
     on_host = not q.is_cuda
     dev = torch.device("cuda", torch.cuda.current_device()) if on_host else q.device
     q, k, v, log_alpha, beta, initial_state, cu_seqlens = (
         _to_device(x, dev) for x in (q, k, v, log_alpha, beta, initial_state, cu_seqlens))
-    q, k, v, log_alpha, beta = (x.contiguous() for x in (q, k, v, log_alpha, beta))
+    q, k, v, beta = (x.contiguous() for x in (q, k, v, beta))
+    if log_alpha is not None:
+        log_alpha = log_alpha.contiguous()
     if q.dim() != 4 or v.dim() != 4:
-        raise ValueError("q, k, log_alpha must be [B, T, H, d_k] and v [B, T, H, d_v]")
+        raise ValueError("q, k must be [B, T, H, d_k] and v [B, T, H, d_v]")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
-        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    gate_shape = (B, T, H) if per_head_gate else q.shape
+    if k.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H):
+        raise ValueError("inconsistent shapes among q, k, v, beta")
+    if log_alpha is None and not per_head_gate:
+        raise ValueError("log_alpha is required")
+    if log_alpha is not None and log_alpha.shape != gate_shape:
+        raise ValueError(f"the gate must be {list(gate_shape)}")
     if cu_seqlens is not None:
         cu_seqlens = cu_seqlens.to(torch.int32).contiguous()
         if B != 1:
@@ -82,22 +89,22 @@ def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, outpu
              out_dtype):
     lib = _lib.load()
     on_host, (q, k, v, la, beta, s0, cu), (B, T, H, dk, dv, N) = _prefill_prepare(
-        q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+        q, k, v, log_alpha, beta, initial_state, cu_seqlens, per_head_gate=fn_name.startswith("gdn_"))
     dt = _io_dtype(q, k, v, la, beta)
     odt = _out_dtype(out_dtype)
     out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
     fs = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if output_final_state else None
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(s0), _ptr(cu),
             ctypes.c_int32(N if cu is not None else 0), B, T, H, dk, dv]
-    if fn_name == "kda_chunk_fwd":
+    if fn_name.endswith("_chunk_fwd"):
         ws_bytes = ctypes.c_size_t(0)
         _lib.check(lib.kda_chunk_fwd_workspace_size(N, H, dk, dv, dt, ctypes.byref(ws_bytes)),
                    "kda_chunk_fwd_workspace_size")
         ws = torch.empty(ws_bytes.value, dtype=torch.uint8, device=q.device) if ws_bytes.value else None
-        status = lib.kda_chunk_fwd(*args, ctypes.c_int32(chunk_size), dt, odt, _ptr(out), _ptr(fs), _ptr(ws),
-                                   ctypes.c_size_t(ws_bytes.value), _stream_handle())
+        status = getattr(lib, fn_name)(*args, ctypes.c_int32(chunk_size), dt, odt, _ptr(out), _ptr(fs), _ptr(ws),
+                                       ctypes.c_size_t(ws_bytes.value), _stream_handle())
     else:
-        status = lib.kda_recurrent_fwd(*args, dt, odt, _ptr(out), _ptr(fs), _stream_handle())
+        status = getattr(lib, fn_name)(*args, dt, odt, _ptr(out), _ptr(fs), _stream_handle())
     _lib.check(status, fn_name)
     if on_host:
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
@@ -131,6 +138,36 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=N
                     64, out_dtype)
 
 
+def _decode(fn_name, q, k, v, gate, beta, state, out, out_dtype):
+    lib = _lib.load()
+    if not state.is_cuda or state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError("state must be a contiguous fp32 CUDA tensor (it is updated in place)")
+    on_host = not q.is_cuda
+    q, k, v, beta = (_to_device(x, state.device).contiguous() for x in (q, k, v, beta))
+    la = None if gate is None else _to_device(gate, state.device).contiguous()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    per_head = fn_name.startswith("gdn_")
+    if la is None and not per_head:
+        raise ValueError("log_alpha is required")
+    if k.shape != q.shape or v.shape != (B, H, dv) or beta.shape != (B, H) or state.shape != (B, H, dk, dv) \
+            or (la is not None and la.shape != ((B, H) if per_head else q.shape)):
+        raise ValueError(f"inconsistent shapes for {fn_name}")
+    dt = _io_dtype(q, k, v, la, beta)
+    if out is not None:
+        out_dtype = out.dtype
+    odt = _out_dtype(out_dtype)
+    o = out if (out is not None and out.is_cuda) else torch.empty((B, H, dv), dtype=out_dtype, device=state.device)
+    status = getattr(lib, fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(state), _ptr(o),
+                                   B, H, dk, dv, dt, odt, _stream_handle())
+    _lib.check(status, fn_name)
+    if on_host:
+        oh = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        oh.copy_(o, non_blocking=True)
+        return oh
+    return o
+
+
 def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, out_dtype=torch.float32):
     """One decode step; ``state`` (fp32 [B, H, d_k, d_v], on the GPU) is updated in place.
 
@@ -138,29 +175,28 @@ def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, out_dtype=torch.f
     [B, H, d_v] of ``out_dtype`` (a host tensor when the token inputs were host
     tensors; ``out``, if given, receives the result).
     """
-    lib = _lib.load()
-    if not state.is_cuda or state.dtype != torch.float32 or not state.is_contiguous():
-        raise ValueError("state must be a contiguous fp32 CUDA tensor (it is updated in place)")
-    on_host = not q.is_cuda
-    q, k, v, la, beta = (_to_device(x, state.device).contiguous() for x in (q, k, v, log_alpha, beta))
-    B, H, dk = q.shape
-    dv = v.shape[-1]
-    if k.shape != q.shape or la.shape != q.shape or v.shape != (B, H, dv) or beta.shape != (B, H) \
-            or state.shape != (B, H, dk, dv):
-        raise ValueError("inconsistent shapes for kda_decode_step")
-    dt = _io_dtype(q, k, v, la, beta)
-    if out is not None:
-        out_dtype = out.dtype
-    odt = _out_dtype(out_dtype)
-    o = out if (out is not None and out.is_cuda) else torch.empty((B, H, dv), dtype=out_dtype, device=state.device)
-    status = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(state), _ptr(o),
-                                 B, H, dk, dv, dt, odt, _stream_handle())
-    _lib.check(status, "kda_decode_step")
-    if on_host:
-        oh = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        oh.copy_(o, non_blocking=True)
-        return oh
-    return o
+    return _decode("kda_decode_step", q, k, v, log_alpha, beta, state, out, out_dtype)
+
+
+def gdn_chunk_fwd(q, k, v, log_g, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
+                  chunk_size=64, out_dtype=torch.float32):
+    """Gated DeltaNet prefill (one log-decay per head and token): :func:`kda_chunk_fwd` with
+    ``log_g`` [B, T, H] in place of log_alpha; ``log_g=None`` is DeltaNet (no decay)."""
+    return _prefill("gdn_chunk_fwd", q, k, v, log_g, beta, initial_state, cu_seqlens, output_final_state,
+                    chunk_size, out_dtype)
+
+
+def gdn_recurrent_fwd(q, k, v, log_g, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
+                      out_dtype=torch.float32):
+    """Token-by-token Gated DeltaNet / DeltaNet prefill (same contract as :func:`gdn_chunk_fwd`)."""
+    return _prefill("gdn_recurrent_fwd", q, k, v, log_g, beta, initial_state, cu_seqlens, output_final_state,
+                    64, out_dtype)
+
+
+def gdn_decode_step(q, k, v, log_g, beta, state, out=None, out_dtype=torch.float32):
+    """One Gated DeltaNet / DeltaNet decode step: :func:`kda_decode_step` with ``log_g`` [B, H]
+    (or None: no decay) in place of log_alpha."""
+    return _decode("gdn_decode_step", q, k, v, log_g, beta, state, out, out_dtype)
 
 
 def device_error() -> int:

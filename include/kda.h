@@ -146,6 +146,39 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
                            void *stream);
 
 /*
+ * Gated DeltaNet and DeltaNet -- the same recurrence with a coarser gate.  Gated
+ * DeltaNet decays the whole state of a head by one factor per token,
+ *     S_t = (I - beta_t k_t k_t^T) g_t S_{t-1} + beta_t k_t v_t^T,   g_t = exp(log_g_t),
+ * the scalar-gate case of KDA: every key channel shares alpha_t = g_t, and a
+ * scalar commutes with the erase, so g_t (I - beta k k^T) S equals
+ * (I - beta k k^T) g_t S.  DeltaNet has no decay (g_t = 1).  Stages 1 and 2 of
+ * section "Core Module Design" of "Hybrid Linear Attention Architectures:
+ * Breaking Through the Long-Context Engineering Bottleneck in LLMs" define both.
+ *
+ * gdn_chunk_fwd, gdn_recurrent_fwd and gdn_decode_step take the same arguments,
+ * layouts, paths, workspace (kda_chunk_fwd_workspace_size) and status codes as
+ * kda_chunk_fwd, kda_recurrent_fwd and kda_decode_step, with log_g in place of
+ * log_alpha:
+ *   log_g : [B, T, H] dtype (prefill) or [B, H] dtype (decode), log_g <= 0, or
+ *           NULL for DeltaNet (no decay; allowed whatever T is).
+ */
+kda_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const void *log_g,
+                         const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                         int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k,
+                         int32_t d_v, int32_t chunk, kda_dtype dtype, kda_dtype out_dtype,
+                         void *out, float *final_state, void *workspace, size_t workspace_bytes,
+                         void *stream);
+kda_status gdn_recurrent_fwd(const void *q, const void *k, const void *v, const void *log_g,
+                             const void *beta, const float *init_state,
+                             const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                             int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                             kda_dtype out_dtype, void *out, float *final_state, void *stream);
+kda_status gdn_decode_step(const void *q, const void *k, const void *v, const void *log_g,
+                           const void *beta, float *state, void *out, int32_t B, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, kda_dtype out_dtype,
+                           void *stream);
+
+/*
  * kda_chunk_fwd_static_ws -- kda_chunk_fwd for callers that cannot allocate
  * device memory when they call it.  Examples: an inference engine that has
  * reserved all device memory up front in its own pool and forbids further

@@ -12,6 +12,12 @@ Contents
     Through the Long-Context Engineering Bottleneck in LLMs"), in plain C
     (``kda_oracle.c``), fp64, threaded over (sequence, head) pairs.
   * :func:`decode_step` -- one iteration of the same loop body, in place.
+  * :func:`gdn_recurrent`, :func:`gdn_decode_step` -- Gated DeltaNet (one
+    decay per head and token) and DeltaNet (no decay): the same recurrence
+    with every key channel sharing the head's decay, the scalar-gate and
+    alpha = 1 reductions that ``test_scalar_gate_is_gated_deltanet`` and
+    ``test_alpha_one_is_deltanet`` pin against the matrix forms of Stages 1
+    and 2 of section "Core Module Design" on the same page.
   * :func:`chunkwise` (``chunkwise.py``) -- an independent fp64 NumPy
     restatement of the chunkwise formulas ("Hardware-Aware Chunkwise
     Parallelism" on the same page; section 3 of "Linear Attention KDA Gating in
@@ -124,6 +130,26 @@ def decode_step(q, k, v, log_alpha, beta, state):
     return out, S
 
 
+def _channel_gate(log_g, shape):
+    """A per-head log-decay (or None: none) as the per-channel gate of the same recurrence."""
+    if log_g is None:
+        return np.zeros(shape, dtype=np.float64)
+    return np.ascontiguousarray(np.broadcast_to(_f64(log_g)[..., None], shape))
+
+
+def gdn_recurrent(q, k, v, log_g, beta, init_state=None, cu_seqlens=None, nthreads=None):
+    """Gated DeltaNet over [B, T, H, d] inputs with ``log_g`` [B, T, H] (None: DeltaNet);
+    returns ``(out, final_state)`` in fp64."""
+    q = _f64(q)
+    return recurrent(q, k, v, _channel_gate(log_g, q.shape), beta, init_state, cu_seqlens, nthreads)
+
+
+def gdn_decode_step(q, k, v, log_g, beta, state):
+    """One Gated DeltaNet / DeltaNet step for [B, H, d] inputs, ``log_g`` [B, H] or None."""
+    q = _f64(q)
+    return decode_step(q, k, v, _channel_gate(log_g, q.shape), beta, state)
+
+
 from .chunkwise import chunkwise  # noqa: E402  (NumPy restatement, see module docstring)
 
-__all__ = ["build_oracle", "recurrent", "decode_step", "chunkwise"]
+__all__ = ["build_oracle", "recurrent", "decode_step", "gdn_recurrent", "gdn_decode_step", "chunkwise"]

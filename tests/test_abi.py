@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_symbols():
     text = open(os.path.join(ROOT, "include", "kda.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b((?:kda|gdn)_[a-z_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -77,6 +77,31 @@ def test_rejects_bad_arguments(lib):
     assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
     assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 32, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == U
     assert dec(ODD, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+
+
+def test_gdn_rejects_bad_arguments(lib):
+    E, U = _lib.KDA_ERR_INVALID_ARG, _lib.KDA_ERR_UNSUPPORTED
+
+    def gchunk(q=FAKE, gate=FAKE, B=1, T=128, dk=128, chunk_size=64, ws=FAKE, ws_bytes=1 << 30):
+        return lib.gdn_chunk_fwd(q, FAKE, FAKE, gate, FAKE, None, None, 0, B, T, 2, dk, 128, chunk_size,
+                                 _lib.KDA_BF16, _lib.KDA_F32, FAKE, None, ws, ws_bytes, None)
+
+    assert gchunk(q=None) == E
+    assert gchunk(B=0) == E
+    assert gchunk(gate=ODD) == E                 # a given gate must be 16-byte aligned like every tensor
+    assert gchunk(gate=None, ws=None) == E       # a null gate (DeltaNet) is fine; the missing workspace is not
+    assert gchunk(dk=96) == U
+    assert gchunk(chunk_size=32) == U
+    # the per-channel gate of KDA stays mandatory
+    assert lib.kda_chunk_fwd(FAKE, FAKE, FAKE, None, FAKE, None, None, 0, 1, 128, 2, 128, 128, 64, _lib.KDA_BF16,
+                             _lib.KDA_F32, FAKE, None, FAKE, 1 << 30, None) == E
+    assert lib.gdn_recurrent_fwd(FAKE, FAKE, FAKE, None, None, None, None, 0, 1, 8, 1, 64, 64, _lib.KDA_F32,
+                                 _lib.KDA_F32, FAKE, None, None) == E   # beta missing
+    dec = lib.gdn_decode_step
+    assert dec(FAKE, FAKE, FAKE, None, FAKE, None, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+    assert dec(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 32, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == U
+    assert lib.kda_decode_step(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16,
+                               _lib.KDA_F32, None) == E
 
 
 def test_workspace_size(lib):

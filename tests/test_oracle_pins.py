@@ -161,6 +161,40 @@ def test_scalar_gate_is_gated_deltanet():
     np.testing.assert_allclose(fs[0, 0], S, atol=1e-12, rtol=1e-12)
 
 
+def test_gdn_oracle_matches_matrix_forms():
+    """The Gated DeltaNet / DeltaNet entry points against the Stage 2 and Stage 1 matrix forms,
+    written here with the scalar outside the erase (g (I - b k k^T) S), over two heads and a
+    packed pair of sequences."""
+    rng = np.random.default_rng(61)
+    q, k, v, _, beta, s0 = rand_case(rng, T=13, H=2, dk=5, dv=3)
+    log_g = np.log(rng.uniform(0.2, 1.0, (1, 13, 2)))
+    cu = np.array([0, 6, 13])
+    s0 = rng.standard_normal((2, 2, 5, 3))
+    for gate in (log_g, None):
+        out, fs = oracle.gdn_recurrent(q, k, v, gate, beta, s0, cu_seqlens=cu)
+        for n in range(2):
+            for h in range(2):
+                S = s0[n, h].copy()
+                for t in range(cu[n], cu[n + 1]):
+                    kt, g = k[0, t, h], 1.0 if gate is None else np.exp(gate[0, t, h])
+                    S = g * (np.eye(5) - beta[0, t, h] * np.outer(kt, kt)) @ S + beta[0, t, h] * np.outer(kt, v[0, t, h])
+                    np.testing.assert_allclose(out[0, t, h], S.T @ q[0, t, h], atol=1e-12, rtol=1e-12)
+                np.testing.assert_allclose(fs[n, h], S, atol=1e-12, rtol=1e-12)
+        # one decode step from the final state, the same form again
+        qd, kd, vd = (rng.standard_normal((2, 2, d)) for d in (5, 5, 3))
+        kd /= np.linalg.norm(kd, axis=-1, keepdims=True)
+        bd = rng.uniform(0, 1, (2, 2))
+        gd = None if gate is None else np.log(rng.uniform(0.2, 1.0, (2, 2)))
+        od, Sd = oracle.gdn_decode_step(qd, kd, vd, gd, bd, fs)
+        for n in range(2):
+            for h in range(2):
+                g = 1.0 if gd is None else np.exp(gd[n, h])
+                S = g * (np.eye(5) - bd[n, h] * np.outer(kd[n, h], kd[n, h])) @ fs[n, h] + \
+                    bd[n, h] * np.outer(kd[n, h], vd[n, h])
+                np.testing.assert_allclose(Sd[n, h], S, atol=1e-12, rtol=1e-12)
+                np.testing.assert_allclose(od[n, h], S.T @ qd[n, h], atol=1e-12, rtol=1e-12)
+
+
 # ---- 6. linearity in (V, S_0) ----------------------------------------------------------------
 
 def test_linearity_in_values_and_state():
