@@ -244,7 +244,7 @@ def event_time_ms(fn, n):
 def run_kda(args):
     import torch
 
-    from gated_delta_rule_86_b200 import inputs, kda_chunk_fwd, kda_decode_step, device_error
+    from gated_delta_rule_86_b200 import device_error, inputs, kda_chunk_fwd, kda_chunk_fwd_fused, kda_decode_step
     rank, world, local = dist_setup(args.gpus)
     peaks, peaks_src = load_peaks()
     hbm_peak = peaks["hbm_gbs"]
@@ -308,7 +308,34 @@ def run_kda(args):
     e2e_ms = max_over_ranks(e2e_ms / max(1, args.steps // 2), world)
     h2d = sum(t.numel() * t.element_size() for t in host) + s0_h.numel() * 4
     d2h = token_heads * w.dv * 4 + w.B * w.H * w.dk * w.dv * 4
-    del host, s0_h, x, a, s0
+    del host, s0_h, x, a
+    torch.cuda.empty_cache()
+
+    # ---------------- the same prefill from the raw projections (fused prologue) ----------------
+    xr = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank, raw=True)
+    ar = [xr[n] for n in names]
+
+    def fused_step(_i):
+        return kda_chunk_fwd_fused(*ar, initial_state=s0)
+
+    for _ in range(args.warmup):
+        fused_step(0)
+    barrier(world)
+    fms = event_time_ms(fused_step, args.steps)
+    barrier(world)
+    fms_step = max_over_ranks(fms / args.steps, world)
+    f_gbs = alg_bytes / (fms_step * 1e-3) / 1e9
+    fused = {"entry": "kda_chunk_fwd_fused", "workload": PREFILL_WORKLOAD,
+             "inputs": "raw bf16 q, k (not normalised), g ~ N(4,1), b ~ N(0,1); normalisation, logsigmoid and "
+                       "sigmoid inside the kernel's loads",
+             "ms_per_step": fms_step, "tokens_per_s": world * tokens / (fms_step * 1e-3),
+             "roofline": {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
+                          "frac": f_gbs / hbm_peak, "traffic": None, "kernel": "kda_chunk_tc_kernel",
+                          "alg_bytes_per_launch": alg_bytes},
+             # what a separate prologue pass would add: write and re-read the activated q, k,
+             # log_alpha (bf16) and beta
+             "separate_pass_bytes_saved": 2 * token_heads * (3 * w.dk * 2 + 2)}
+    del xr, ar, s0
     torch.cuda.empty_cache()
 
     # ---------------- decode ----------------
@@ -368,7 +395,7 @@ def run_kda(args):
                 "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 # per step: the schedule-table kernel and the chunk kernel
-                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode}
+                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "fused_prologue": fused}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -12,8 +12,8 @@ KDA_F32, KDA_BF16 = 0, 1
 
 # every symbol include/kda.h declares
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_static_ws", "kda_recurrent_fwd",
-            "kda_decode_step", "gdn_chunk_fwd", "gdn_recurrent_fwd", "gdn_decode_step", "kda_status_string",
-            "kda_get_last_device_error", "kda_version")
+            "kda_decode_step", "gdn_chunk_fwd", "gdn_recurrent_fwd", "gdn_decode_step", "kda_chunk_fwd_fused",
+            "kda_decode_step_fused", "kda_status_string", "kda_get_last_device_error", "kda_version")
 
 _lib = None
 
@@ -38,7 +38,7 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, f32p = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     prefill_args = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, i32, i32]
-    for name in ("kda_chunk_fwd", "gdn_chunk_fwd"):
+    for name in ("kda_chunk_fwd", "gdn_chunk_fwd", "kda_chunk_fwd_fused"):
         fn = getattr(lib, name)
         fn.argtypes = prefill_args + [i32, ctypes.c_int, ctypes.c_int, vp, f32p, vp, ctypes.c_size_t, vp]
         fn.restype = ctypes.c_int
@@ -48,7 +48,7 @@ def load() -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = prefill_args + [ctypes.c_int, ctypes.c_int, vp, f32p, vp]
         fn.restype = ctypes.c_int
-    for name in ("kda_decode_step", "gdn_decode_step"):
+    for name in ("kda_decode_step", "gdn_decode_step", "kda_decode_step_fused"):
         fn = getattr(lib, name)
         fn.argtypes = [vp, vp, vp, vp, vp, f32p, vp, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int, vp]
         fn.restype = ctypes.c_int

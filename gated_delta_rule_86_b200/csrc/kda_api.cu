@@ -31,7 +31,7 @@ kda_status check_prefill(const void *q, const void *k, const void *v, const void
     if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
     // token tensors may be empty (NULL) only when there are no tokens; a per-head gate may be NULL
     // (no decay)
-    if (T > 0 && (!q || !k || !v || (gate == kda::kGateChannel && !la) || !beta || !out))
+    if (T > 0 && (!q || !k || !v || (gate != kda::kGateHead && !la) || !beta || !out))
         return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -173,7 +173,8 @@ kda_status chunk_impl(int gate, bool static_ws, const void *q, const void *k, co
     if (chunk < 1) return KDA_ERR_INVALID_ARG;
     if (chunk != 64) return KDA_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (static_ws) {
+    if (static_ws || gate == kda::kRawInputs) {
+        // the raw-projection form runs on the tensor-core path only
         if (dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
     } else if (dtype == KDA_F32) {
         // fp32 I/O asks for fp32 accuracy, which bf16 tensor-core operands
@@ -208,7 +209,7 @@ template <int GK>
 kda_status decode_impl(const void *q, const void *k, const void *v, const void *la, const void *beta, float *state,
                        void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
                        kda_dtype out_dtype, void *stream) {
-    if (!q || !k || !v || (GK == kda::kGateChannel && !la) || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || (GK != kda::kGateHead && !la) || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -304,6 +305,22 @@ kda_status gdn_recurrent_fwd(const void *q, const void *k, const void *v, const 
                              kda_dtype out_dtype, void *out, float *final_state, void *stream) {
     return recurrent_impl(kda::kGateHead, q, k, v, log_g, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v,
                           dtype, out_dtype, out, final_state, stream);
+}
+
+kda_status kda_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const void *g_raw,
+                               const void *b_raw, const float *init_state, const int32_t *cu_seqlens,
+                               int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                               int32_t chunk, kda_dtype dtype, kda_dtype out_dtype, void *out, float *final_state,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    return chunk_impl(kda::kRawInputs, false, q_raw, k_raw, v, g_raw, b_raw, init_state, cu_seqlens, num_seqs, B, T,
+                      H, d_k, d_v, chunk, dtype, out_dtype, out, final_state, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_decode_step_fused(const void *q_raw, const void *k_raw, const void *v, const void *g_raw,
+                                 const void *b_raw, float *state, void *out, int32_t B, int32_t H, int32_t d_k,
+                                 int32_t d_v, kda_dtype dtype, kda_dtype out_dtype, void *stream) {
+    return decode_impl<kda::kRawInputs>(q_raw, k_raw, v, g_raw, b_raw, state, out, B, H, d_k, d_v, dtype, out_dtype,
+                                        stream);
 }
 
 kda_status gdn_decode_step(const void *q, const void *k, const void *v, const void *log_g, const void *beta,

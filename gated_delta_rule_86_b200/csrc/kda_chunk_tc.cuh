@@ -458,19 +458,19 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             const int L = have ? it.pi.len(it.c) : -1, h = it.pi.h;
             if (lane == 0) {
                 // a per-head gate comes as 64 scalars (below) instead of a log_alpha tile
-                constexpr uint32_t kTileBytes = GK == kGateChannel ? SM::kRawBytes : SM::kRawBytes - SM::kTile;
+                constexpr uint32_t kTileBytes = GK != kGateHead ? SM::kRawBytes : SM::kRawBytes - SM::kTile;
                 tc::mbar_arrive_expect_tx(&bars.raw_full, have ? kTileBytes : 0);
                 if (have) {
                     const int t = static_cast<int>(tok0);
-                    if constexpr (GK == kGateChannel) tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
+                    if constexpr (GK != kGateHead) tc::tma_load_3d(sm + SM::kRawG, &maps.g, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawK, &maps.k, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawQ, &maps.q, 0, h, t, &bars.raw_full);
                     tc::tma_load_3d(sm + SM::kRawV, &maps.v, 0, h, t, &bars.raw_full);
                 }
             }
             float *bdst = sBetaIn + (kl & 1) * kChunk;
-            bdst[lane] = (lane < L) ? __bfloat162float(beta[(tok0 + lane) * H + h]) : 0.f;
-            bdst[32 + lane] = (32 + lane < L) ? __bfloat162float(beta[(tok0 + 32 + lane) * H + h]) : 0.f;
+            bdst[lane] = (lane < L) ? beta_of<GK>(beta, (size_t)(tok0 + lane) * H + h) : 0.f;
+            bdst[32 + lane] = (32 + lane < L) ? beta_of<GK>(beta, (size_t)(tok0 + 32 + lane) * H + h) : 0.f;
             if constexpr (GK == kGateHead) {   // fp32 log-decays of the 64 tokens, in place of the tile
                 float *gdst = reinterpret_cast<float *>(sm + SM::kRawG);
                 gdst[lane] = (lane < L) ? gate_log<GK>(log_g, (size_t)(tok0 + lane) * H + h, kDK, 0) : 0.f;
@@ -540,10 +540,14 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = tg * 2 + rr;
                 float g8[8];
-                if constexpr (GK == kGateChannel) {
+                if constexpr (GK != kGateHead) {
                     const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
                                             : make_uint4(0, 0, 0, 0);
                     unpack8(raw, g8);
+                    if constexpr (GK == kRawInputs) {   // the gate's pre-activation: log_alpha = logsigmoid
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) g8[i] = r < L ? log_sigmoid(g8[i]) : 0.f;
+                    }
                 } else {   // one decay for every channel
                     const float gs = r < L ? reinterpret_cast<const float *>(sm + SM::kRawG)[r] : 0.f;
 #pragma unroll
@@ -646,6 +650,27 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                 float kf[8], qf[8];
                 unpack8(rk[rr], kf);
                 unpack8(rq[rr], qf);
+                if constexpr (GK == kRawInputs) {
+                    // raw q and k rows: L2-normalise over the 128 channels, which the 16 lanes of this
+                    // half-warp hold 8 each
+                    float sk = 0.f, sq = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        sk = fmaf(kf[i], kf[i], sk);
+                        sq = fmaf(qf[i], qf[i], sq);
+                    }
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) {
+                        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    }
+                    const float nk = rsqrtf(sk + kNormEps), nq = rsqrtf(sq + kNormEps);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        kf[i] *= nk;
+                        qf[i] *= nq;
+                    }
+                }
                 // per-channel constants, re-read from shared memory for each token (fewer live registers)
                 float gref[8], eref[8], elast[8];
                 const float *sEref = reinterpret_cast<const float *>(sm + SM::kEref) + cg * 8;
@@ -1113,15 +1138,35 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         for (int r = 0; r < L; ++r) {
             const int64_t trow = (tok0 + r) * H + h;
             // a per-head gate: the same log-decay for every channel (none when log_g is null)
-            constexpr int gstride = GK == kGateChannel ? 1 : 0;
-            const __nv_bfloat16 *gr = log_alpha + (GK == kGateChannel ? trow * kDK + c0 : trow),
+            constexpr int gstride = GK != kGateHead ? 1 : 0;
+            const __nv_bfloat16 *gr = log_alpha + (GK != kGateHead ? trow * kDK + c0 : trow),
                                 *kr = k + trow * kDK + c0, *qr = q + trow * kDK + c0;
-            const bool has_gate = GK == kGateChannel || log_alpha != nullptr;
+            const bool has_gate = GK != kGateHead || log_alpha != nullptr;
+            // raw inputs: the 1 / L2 norms of the whole q and k rows
+            float nk = 1.f, nq = 1.f;
+            if constexpr (GK == kRawInputs) {
+                const uint4 *k8 = reinterpret_cast<const uint4 *>(k + trow * kDK);
+                const uint4 *q8 = reinterpret_cast<const uint4 *>(q + trow * kDK);
+                float sk = 0.f, sq = 0.f;
+                for (int c8 = 0; c8 < kDK / 8; ++c8) {
+                    float f[8];
+                    unpack8(k8[c8], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sk = fmaf(f[i], f[i], sk);
+                    unpack8(q8[c8], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sq = fmaf(f[i], f[i], sq);
+                }
+                nk = rsqrtf(sk + kNormEps);
+                nq = rsqrtf(sq + kNormEps);
+            }
             float pk = 0.f, pq = 0.f, kq = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = has_gate ? expf(__bfloat162float(gr[i * gstride])) : 1.f,
-                            kk = __bfloat162float(kr[i]), qq = __bfloat162float(qr[i]);
+                float lg = __bfloat162float(gr[i * gstride]);
+                if constexpr (GK == kRawInputs) lg = log_sigmoid(lg);
+                const float a = has_gate ? expf(lg) : 1.f, kk = __bfloat162float(kr[i]) * nk,
+                            qq = __bfloat162float(qr[i]) * nq;
                 S[i] *= a;
                 pk = fmaf(S[i], kk, pk);
                 pq = fmaf(S[i], qq, pq);
@@ -1134,10 +1179,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const float skq = (redKq[0] + redKq[1]) + (redKq[2] + redKq[3]);
             const float spk = (redPk[j] + redPk[128 + j]) + (redPk[256 + j] + redPk[384 + j]);
             const float spq = (redPq[j] + redPq[128 + j]) + (redPq[256 + j] + redPq[384 + j]);
-            const float u = jv ? __bfloat162float(beta[trow]) * (__bfloat162float(v[trow * DV + j]) - spk) : 0.f;
+            const float u = jv ? beta_of<GK>(beta, trow) * (__bfloat162float(v[trow * DV + j]) - spk) : 0.f;
             if (qd == 0 && jv) out[trow * DV + j] = from_f32<TO>(fmaf(u, skq, spq));
 #pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] = fmaf(__bfloat162float(kr[i]), u, S[i]);
+            for (int i = 0; i < 32; ++i) S[i] = fmaf(__bfloat162float(kr[i]) * nk, u, S[i]);
             tc::named_sync(kBarRole, kRoleThreads);
         }
         return write_state_operand();
@@ -1484,7 +1529,7 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
     memset(&maps, 0, sizeof(maps));
     const int64_t tokens = (int64_t)B * T;
     if (tokens > 0) {   // with no tokens no chunk is loaded and the maps stay unused
-        if ((GK == kGateChannel && !encode_row_map(&maps.g, la, kDK, H, tokens)) ||
+        if ((GK != kGateHead && !encode_row_map(&maps.g, la, kDK, H, tokens)) ||
             !encode_row_map(&maps.k, k, kDK, H, tokens) ||
             !encode_row_map(&maps.q, q, kDK, H, tokens) || !encode_row_map(&maps.v, v, DV, H, tokens) ||
             !encode_row_map(&maps.o, out, DV, H, tokens, 64,
@@ -1529,8 +1574,8 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
                               init_state, static_cast<TO *>(out), final_state);
 }
 
-// `la`: log_alpha [tokens][H][d_k] (gate kGateChannel), or the per-head log_g [tokens][H] or null
-// (kGateHead).
+// `la`: log_alpha [tokens][H][d_k] (kGateChannel), the per-head log_g [tokens][H] or null
+// (kGateHead), or the gate's pre-activation [tokens][H][d_k] (kRawInputs, with raw q, k, beta).
 template <typename TO>
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *la, const void *beta,
                             const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
@@ -1544,6 +1589,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const v
     KDA_CHUNK_TC_CASE(128, kGateChannel)
     KDA_CHUNK_TC_CASE(64, kGateHead)
     KDA_CHUNK_TC_CASE(128, kGateHead)
+    KDA_CHUNK_TC_CASE(64, kRawInputs)
+    KDA_CHUNK_TC_CASE(128, kRawInputs)
 #undef KDA_CHUNK_TC_CASE
     return cudaErrorInvalidValue;
 }

@@ -33,17 +33,31 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
-// How the decay gate is given.  kGateChannel: one log-decay per key channel, log_alpha
-// [..., d_k] (KDA).  kGateHead: one log-decay per head and token, log_g [...] (Gated DeltaNet, the
+// How the inputs are given.  kGateChannel: one log-decay per key channel, log_alpha [..., d_k]
+// (KDA).  kGateHead: one log-decay per head and token, log_g [...] (Gated DeltaNet, the
 // scalar-gate case of the same recurrence); a null log_g means no decay at all, alpha == 1
-// (DeltaNet).  The recurrence is otherwise the same.
-enum GateKind : int { kGateChannel = 0, kGateHead = 1 };
+// (DeltaNet).  kRawInputs: KDA from the raw projections (the fused prologue): q and k are
+// L2-normalised over d_k here, log_alpha = logsigmoid(g) of a per-channel pre-activation g, and
+// beta = sigmoid(b) of a pre-activation b.
+enum GateKind : int { kGateChannel = 0, kGateHead = 1, kRawInputs = 2 };
+
+// logsigmoid(x) = -log(1 + exp(-x)), in the form that neither overflows nor loses small values.
+__device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
+__device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
+// L2 normalisation of q and k (kRawInputs): x * rsqrt(sum x^2 + kNormEps)
+constexpr float kNormEps = 1e-6f;
 
 // Log-decay of key channel c at gate row `row` (token * H + head, or batch * H + head).
 template <int GK, typename T>
 __device__ __forceinline__ float gate_log(const T *gate, size_t row, int dk, int c) {
     if constexpr (GK == kGateChannel) return to_f32(gate[row * dk + c]);
+    else if constexpr (GK == kRawInputs) return log_sigmoid(to_f32(gate[row * dk + c]));
     else return gate ? to_f32(gate[row]) : 0.f;
+}
+// beta of a row as the kernel uses it
+template <int GK, typename T> __device__ __forceinline__ float beta_of(const T *beta, size_t row) {
+    if constexpr (GK == kRawInputs) return sigmoidf(to_f32(beta[row]));
+    else return to_f32(beta[row]);
 }
 
 // log2(e), used to turn exp(x) into exp2(x * log2e) for the ex2 unit.

@@ -10,7 +10,8 @@
 // Attention: The Hybrid Architecture Trade-off for Large Models" describes.
 //
 // The gate is one log-decay per key channel (KDA) or, with GK = kGateHead, one per head (Gated
-// DeltaNet; a null gate gives DeltaNet, alpha == 1).
+// DeltaNet; a null gate gives DeltaNet, alpha == 1).  With GK = kRawInputs the token inputs are
+// the raw projections: q and k are L2-normalised here, alpha = sigmoid(g), beta = sigmoid(b).
 //
 // Mapping: one CTA of 256 threads per (b, h).  Warp w owns state rows
 // [w*DK/8, (w+1)*DK/8); lane l owns columns [l*DV/32, (l+1)*DV/32), so a warp
@@ -46,6 +47,7 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
     __shared__ __align__(16) float s_red[2][8][DV];
     __shared__ float s_kq[8];
     __shared__ float s_beta;
+    __shared__ float s_nrm[2][DK / 32];   // raw inputs: per-warp sums of q^2 and k^2
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t head = blockIdx.x;
@@ -61,13 +63,38 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
 
     // 2. stage the token vectors
     if (tid < DK) {
-        s_q[tid] = to_f32(q[head * DK + tid]);
-        s_k[tid] = to_f32(k[head * DK + tid]);
+        const float qv = to_f32(q[head * DK + tid]), kv = to_f32(k[head * DK + tid]);
+        s_q[tid] = qv;
+        s_k[tid] = kv;
         s_a[tid] = expf(gate_log<GK>(log_alpha, head, DK, tid));
+        if constexpr (GK == kRawInputs) {   // partial sums for the L2 norms of the raw q and k
+            float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+            }
+            if (lane == 0) {
+                s_nrm[0][warp] = sq;
+                s_nrm[1][warp] = sk;
+            }
+        }
     }
     if (tid >= 256 - DV) s_v[tid - (256 - DV)] = to_f32(v[head * DV + tid - (256 - DV)]);
-    if (tid == 0) s_beta = to_f32(beta[head]);
+    if (tid == 0) s_beta = beta_of<GK>(beta, head);
     __syncthreads();
+    // 1 / L2 norms of q and k (1 unless the inputs are raw projections)
+    float nq = 1.f, nk = 1.f;
+    if constexpr (GK == kRawInputs) {
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int w = 0; w < DK / 32; ++w) {
+            sq += s_nrm[0][w];
+            sk += s_nrm[1][w];
+        }
+        nq = rsqrtf(sq + kNormEps);
+        nk = rsqrtf(sk + kNormEps);
+    }
 
     // 3. decay in registers and per-warp partial reductions over this warp's rows
     float pa[CPL], pb[CPL];
@@ -77,7 +104,7 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
 #pragma unroll
     for (int m = 0; m < RPW; ++m) {
         const int row = warp * RPW + m;
-        const float a = s_a[row], kk = s_k[row], qq = s_q[row];
+        const float a = s_a[row], kk = s_k[row] * nk, qq = s_q[row] * nq;
         kq = fmaf(kk, qq, kq);
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
@@ -117,7 +144,7 @@ kda_decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TI
     for (int c = 0; c < CPL; ++c) u[c] = s_u[lane * CPL + c];
 #pragma unroll
     for (int m = 0; m < RPW; ++m) {
-        const float kk = s_k[warp * RPW + m];
+        const float kk = s_k[warp * RPW + m] * nk;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) s[m][c] = fmaf(kk, u[c], s[m][c]);
         VecT x;

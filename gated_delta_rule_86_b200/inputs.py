@@ -93,22 +93,30 @@ def varlen_lengths(n: int, lo: int, hi: int, seed: int) -> list:
     return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
 
 
-def token_inputs(B, T, H, dk, dv, mu, dtype, gen, device):
-    """q, k, v, log_alpha, beta for [B, T, H, .] in the storage dtype."""
-    q = _unit((B, T, H, dk), gen, device)
-    k = _unit((B, T, H, dk), gen, device)
+def token_inputs(B, T, H, dk, dv, mu, dtype, gen, device, raw=False):
+    """q, k, v, log_alpha, beta for [B, T, H, .] in the storage dtype.
+
+    With ``raw`` the same draws are returned before their activations (the raw projections):
+    q and k not normalised, the gate's and beta's pre-activations N(mu, 1) and N(0, 1).
+    """
+    q = _normal((B, T, H, dk), gen, device) if raw else _unit((B, T, H, dk), gen, device)
+    k = _normal((B, T, H, dk), gen, device) if raw else _unit((B, T, H, dk), gen, device)
     v = _normal((B, T, H, dv), gen, device)
-    beta = torch.sigmoid(_normal((B, T, H), gen, device))
-    log_alpha = torch.nn.functional.logsigmoid(_normal((B, T, H, dk), gen, device, mean=mu))
+    beta = _normal((B, T, H), gen, device)
+    log_alpha = _normal((B, T, H, dk), gen, device, mean=mu)
+    if not raw:
+        beta = torch.sigmoid(beta)
+        log_alpha = torch.nn.functional.logsigmoid(log_alpha)
     return tuple(x.to(dtype) for x in (q, k, v, log_alpha, beta))
 
 
-def make_prefill(w: Workload | str, device="cpu", seed: int | None = None, **override):
+def make_prefill(w: Workload | str, device="cpu", seed: int | None = None, raw: bool = False, **override):
     """Inputs for a prefill workload as a dict of tensors on ``device``.
 
     Keys: q, k, v, log_alpha, beta, init_state (None or fp32 [N,H,dk,dv]),
     cu_seqlens (None or int32 [N+1]).  ``override`` replaces Workload fields
-    (e.g. T=300 for a shortened parity case).
+    (e.g. T=300 for a shortened parity case).  With ``raw`` the keys q, k,
+    log_alpha and beta hold the raw projections (see :func:`token_inputs`).
     """
     if isinstance(w, str):
         w = WORKLOADS[w]
@@ -125,18 +133,19 @@ def make_prefill(w: Workload | str, device="cpu", seed: int | None = None, **ove
                           device=device)
     else:
         B, T, N = w.B, w.T, w.B
-    q, k, v, la, beta = token_inputs(B, T, w.H, w.dk, w.dv, w.mu, w.dtype, gen, device)
+    q, k, v, la, beta = token_inputs(B, T, w.H, w.dk, w.dv, w.mu, w.dtype, gen, device, raw=raw)
     s0 = _normal((N, w.H, w.dk, w.dv), gen, device, std=0.1) if w.init_state else None
     return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, init_state=s0, cu_seqlens=cu,
                 workload=w)
 
 
 def make_decode(w: Workload | str = "decode_bf16", device="cpu", seed: int | None = None,
-                steps: int | None = None, **override):
+                steps: int | None = None, raw: bool = False, **override):
     """Inputs for a decode workload: per-step tokens stacked on a leading axis.
 
     Returns q, k, log_alpha [steps, B, H, dk], v [steps, B, H, dv], beta
-    [steps, B, H] in the storage dtype, and state fp32 [B, H, dk, dv].
+    [steps, B, H] in the storage dtype, and state fp32 [B, H, dk, dv] (raw
+    projections with ``raw``, as in :func:`make_prefill`).
     """
     if isinstance(w, str):
         w = WORKLOADS[w]
@@ -146,5 +155,5 @@ def make_decode(w: Workload | str = "decode_bf16", device="cpu", seed: int | Non
     steps = w.decode_steps if steps is None else steps
     gen = generator(seed, device)
     state = _normal((w.B, w.H, w.dk, w.dv), gen, device, std=0.1)
-    q, k, v, la, beta = token_inputs(steps, w.B, w.H, w.dk, w.dv, w.mu, w.dtype, gen, device)
+    q, k, v, la, beta = token_inputs(steps, w.B, w.H, w.dk, w.dv, w.mu, w.dtype, gen, device, raw=raw)
     return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, state=state, workload=w)

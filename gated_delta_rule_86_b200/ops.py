@@ -96,7 +96,7 @@ def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, outpu
     fs = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if output_final_state else None
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(s0), _ptr(cu),
             ctypes.c_int32(N if cu is not None else 0), B, T, H, dk, dv]
-    if fn_name.endswith("_chunk_fwd"):
+    if "_chunk_fwd" in fn_name:
         ws_bytes = ctypes.c_size_t(0)
         _lib.check(lib.kda_chunk_fwd_workspace_size(N, H, dk, dv, dt, ctypes.byref(ws_bytes)),
                    "kda_chunk_fwd_workspace_size")
@@ -197,6 +197,20 @@ def gdn_decode_step(q, k, v, log_g, beta, state, out=None, out_dtype=torch.float
     """One Gated DeltaNet / DeltaNet decode step: :func:`kda_decode_step` with ``log_g`` [B, H]
     (or None: no decay) in place of log_alpha."""
     return _decode("gdn_decode_step", q, k, v, log_g, beta, state, out, out_dtype)
+
+
+def kda_chunk_fwd_fused(q_raw, k_raw, v, g_raw, b_raw, initial_state=None, cu_seqlens=None,
+                        output_final_state=True, chunk_size=64, out_dtype=torch.float32):
+    """:func:`kda_chunk_fwd` from the raw projections, activated inside the kernel's loads:
+    q, k = L2-normalised q_raw, k_raw (over d_k, eps 1e-6 under the root), log_alpha =
+    logsigmoid(g_raw), beta = sigmoid(b_raw).  Same shapes as kda_chunk_fwd; bf16 only."""
+    return _prefill("kda_chunk_fwd_fused", q_raw, k_raw, v, g_raw, b_raw, initial_state, cu_seqlens,
+                    output_final_state, chunk_size, out_dtype)
+
+
+def kda_decode_step_fused(q_raw, k_raw, v, g_raw, b_raw, state, out=None, out_dtype=torch.float32):
+    """:func:`kda_decode_step` from the raw projections (see :func:`kda_chunk_fwd_fused`)."""
+    return _decode("kda_decode_step_fused", q_raw, k_raw, v, g_raw, b_raw, state, out, out_dtype)
 
 
 def device_error() -> int:

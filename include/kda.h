@@ -179,6 +179,32 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v, const vo
                            void *stream);
 
 /*
+ * kda_chunk_fwd_fused / kda_decode_step_fused -- KDA from the raw projections,
+ * with the step just before the recurrence done inside the kernels' loads
+ * (the per-chunk gating parameters of the "Implementation checklist" of
+ * "Hybrid Linear Attention Architectures: Breaking Through the Long-Context
+ * Engineering Bottleneck in LLMs"), so that no separate pass writes the
+ * normalised inputs to memory and reads them back:
+ *     q = q_raw * rsqrt(sum(q_raw^2) + 1e-6),  k likewise   (L2 over d_k, per token and head)
+ *     log_alpha = logsigmoid(g_raw),  beta = sigmoid(b_raw)
+ * q_raw, k_raw, g_raw take the places (and layouts) of q, k, log_alpha and
+ * b_raw that of beta; everything else is as in kda_chunk_fwd / kda_decode_step.
+ * kda_chunk_fwd_fused runs on the tensor-core path only (dtype KDA_BF16,
+ * d_k == 128; KDA_ERR_UNSUPPORTED otherwise); kda_decode_step_fused supports
+ * what kda_decode_step does.
+ */
+kda_status kda_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const void *g_raw,
+                               const void *b_raw, const float *init_state,
+                               const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                               int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype,
+                               kda_dtype out_dtype, void *out, float *final_state, void *workspace,
+                               size_t workspace_bytes, void *stream);
+kda_status kda_decode_step_fused(const void *q_raw, const void *k_raw, const void *v,
+                                 const void *g_raw, const void *b_raw, float *state, void *out,
+                                 int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
+                                 kda_dtype out_dtype, void *stream);
+
+/*
  * kda_chunk_fwd_static_ws -- kda_chunk_fwd for callers that cannot allocate
  * device memory when they call it.  Examples: an inference engine that has
  * reserved all device memory up front in its own pool and forbids further

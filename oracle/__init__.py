@@ -18,6 +18,9 @@ Contents
     alpha = 1 reductions that ``test_scalar_gate_is_gated_deltanet`` and
     ``test_alpha_one_is_deltanet`` pin against the matrix forms of Stages 1
     and 2 of section "Core Module Design" on the same page.
+  * :func:`prologue` -- the raw projections to the recurrence's inputs (the
+    fused entry points): q, k L2-normalised over d_k with eps 1e-6 under the
+    root, log_alpha = logsigmoid(g), beta = sigmoid(b); fp64 NumPy.
   * :func:`chunkwise` (``chunkwise.py``) -- an independent fp64 NumPy
     restatement of the chunkwise formulas ("Hardware-Aware Chunkwise
     Parallelism" on the same page; section 3 of "Linear Attention KDA Gating in
@@ -130,6 +133,23 @@ def decode_step(q, k, v, log_alpha, beta, state):
     return out, S
 
 
+NORM_EPS = 1e-6
+
+
+def prologue(q_raw, k_raw, g_raw, b_raw):
+    """Raw projections -> (q, k, log_alpha, beta), fp64.
+
+    ``q = q_raw / sqrt(sum(q_raw**2) + 1e-6)`` over the last axis (k likewise),
+    ``log_alpha = logsigmoid(g_raw) = -log(1 + exp(-g_raw))``, ``beta = sigmoid(b_raw)``.
+    """
+    q_raw, k_raw, g_raw, b_raw = (_f64(x) for x in (q_raw, k_raw, g_raw, b_raw))
+    q = q_raw / np.sqrt(np.sum(q_raw * q_raw, axis=-1, keepdims=True) + NORM_EPS)
+    k = k_raw / np.sqrt(np.sum(k_raw * k_raw, axis=-1, keepdims=True) + NORM_EPS)
+    log_alpha = -np.logaddexp(0.0, -g_raw)
+    beta = 1.0 / (1.0 + np.exp(-b_raw))
+    return q, k, log_alpha, beta
+
+
 def _channel_gate(log_g, shape):
     """A per-head log-decay (or None: none) as the per-channel gate of the same recurrence."""
     if log_g is None:
@@ -152,4 +172,4 @@ def gdn_decode_step(q, k, v, log_g, beta, state):
 
 from .chunkwise import chunkwise  # noqa: E402  (NumPy restatement, see module docstring)
 
-__all__ = ["build_oracle", "recurrent", "decode_step", "gdn_recurrent", "gdn_decode_step", "chunkwise"]
+__all__ = ["build_oracle", "recurrent", "decode_step", "gdn_recurrent", "gdn_decode_step", "prologue", "chunkwise"]

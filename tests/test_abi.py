@@ -104,6 +104,23 @@ def test_gdn_rejects_bad_arguments(lib):
                                _lib.KDA_F32, None) == E
 
 
+def test_fused_rejects_bad_arguments(lib):
+    E, U = _lib.KDA_ERR_INVALID_ARG, _lib.KDA_ERR_UNSUPPORTED
+
+    def fchunk(q=FAKE, g=FAKE, dtype=_lib.KDA_BF16, dk=128, ws=FAKE):
+        return lib.kda_chunk_fwd_fused(q, FAKE, FAKE, g, FAKE, None, None, 0, 1, 128, 2, dk, 128, 64, dtype,
+                                       _lib.KDA_F32, FAKE, None, ws, 1 << 30, None)
+
+    assert fchunk(q=None) == E
+    assert fchunk(g=None) == E                    # the gate's pre-activation is required
+    assert fchunk(dtype=_lib.KDA_F32, dk=64) == U  # tensor-core path only
+    assert fchunk(dk=64) == U
+    assert fchunk(ws=None) == E
+    dec = lib.kda_decode_step_fused
+    assert dec(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 96, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == U
+
+
 def test_workspace_size(lib):
     n = ctypes.c_size_t(7)
     assert lib.kda_chunk_fwd_workspace_size(2, 16, 128, 128, _lib.KDA_BF16, ctypes.byref(n)) == _lib.KDA_OK

@@ -195,6 +195,31 @@ def test_gdn_oracle_matches_matrix_forms():
                 np.testing.assert_allclose(od[n, h], S.T @ qd[n, h], atol=1e-12, rtol=1e-12)
 
 
+def test_prologue_closed_forms():
+    """The raw-projection prologue: unit rows (up to the 1e-6 under the root), sigmoid(0) = 1/2,
+    logsigmoid(0) = -log 2, logsigmoid = log(sigmoid) computed the other way, its asymptotes
+    (x for x -> -inf, -exp(-x) for x -> +inf), and 1 - sigmoid(x) = sigmoid(-x)."""
+    rng = np.random.default_rng(71)
+    qr, kr = rng.standard_normal((2, 3, 4, 16)) * 5.0
+    g = np.array([0.0, -40.0, 40.0, 3.0, -3.0])
+    b = np.array([0.0, 2.0, -2.0, 30.0, -30.0])
+    q, k, la, beta = oracle.prologue(qr, kr, g, b)
+    for x, xr in ((q, qr), (k, kr)):
+        n2 = np.sum(xr * xr, axis=-1)
+        np.testing.assert_allclose(np.sum(x * x, axis=-1), n2 / (n2 + 1e-6), rtol=1e-14)
+        np.testing.assert_allclose(x / np.linalg.norm(x, axis=-1, keepdims=True),
+                                   xr / np.linalg.norm(xr, axis=-1, keepdims=True), rtol=1e-14)
+    assert la[0] == -np.log(2.0) and beta[0] == 0.5
+    np.testing.assert_allclose(la[3:], np.log(1.0 / (1.0 + np.exp(-g[3:]))), rtol=1e-14)
+    np.testing.assert_allclose(la[1], -40.0, rtol=1e-15)            # logsigmoid(x) ~ x - exp(x)
+    np.testing.assert_allclose(la[2], -np.exp(-40.0), rtol=1e-12)   # ~ -exp(-x)
+    np.testing.assert_allclose(beta[1] + beta[2], 1.0, rtol=1e-15)
+    np.testing.assert_allclose(beta[4], np.exp(-30.0) / (1 + np.exp(-30.0)), rtol=1e-12)
+    # a zero row stays zero
+    z = oracle.prologue(np.zeros((1, 4)), np.zeros((1, 4)), np.zeros(1), np.zeros(1))
+    assert np.all(z[0] == 0.0) and np.all(z[1] == 0.0)
+
+
 # ---- 6. linearity in (V, S_0) ----------------------------------------------------------------
 
 def test_linearity_in_values_and_state():
