@@ -546,7 +546,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                     unpack8(raw, g8);
                     if constexpr (GK == kRawInputs) {   // the gate's pre-activation: log_alpha = logsigmoid
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) g8[i] = r < L ? log_sigmoid(g8[i]) : 0.f;
+                        for (int i = 0; i < 8; ++i) g8[i] = r < L ? log_sigmoid_fast(g8[i]) : 0.f;
                     }
                 } else {   // one decay for every channel
                     const float gs = r < L ? reinterpret_cast<const float *>(sm + SM::kRawG)[r] : 0.f;

@@ -44,6 +44,11 @@ enum GateKind : int { kGateChannel = 0, kGateHead = 1, kRawInputs = 2 };
 // logsigmoid(x) = -log(1 + exp(-x)), in the form that neither overflows nor loses small values.
 __device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
 __device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
+// The same with the SFU intrinsics (__expf, __logf): an absolute error below 1e-6 in the log-decay
+// (1 + y rounds y < 2^-24 away, a loss below 6e-8), for the per-element work of the decay scan.
+__device__ __forceinline__ float log_sigmoid_fast(float x) {
+    return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
+}
 // L2 normalisation of q and k (kRawInputs): x * rsqrt(sum x^2 + kNormEps)
 constexpr float kNormEps = 1e-6f;
 
