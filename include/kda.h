@@ -14,6 +14,12 @@
  * in a 3:1 Hybrid Architecture"); the output is read after the write; q is not
  * scaled.
  *
+ * Entry points: KDA prefill (kda_chunk_fwd, its static-workspace form
+ * kda_chunk_fwd_static_ws, and the token-by-token kda_recurrent_fwd) and decode
+ * (kda_decode_step); the same from the raw projections (kda_chunk_fwd_fused,
+ * kda_decode_step_fused); Gated DeltaNet and DeltaNet (gdn_chunk_fwd,
+ * gdn_recurrent_fwd, gdn_decode_step); status helpers.
+ *
  * Conventions for every call
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    allocates no device memory and keeps no pointer after the call returns.
@@ -21,7 +27,8 @@
  *    means the legacy default stream).  Arguments are validated on the host
  *    before anything is launched; a rejected call launches nothing.
  *  - Tensors are dense, row-major, with every pointer 16-byte aligned.
- *  - `dtype` is the element type of q, k, v, log_alpha and beta; `out_dtype`
+ *  - `dtype` is the element type of q, k, v, log_alpha and beta (or of the
+ *    tensors in their places: log_g, the raw projections); `out_dtype`
  *    that of out (KDA_F32 keeps the full accuracy of the fp32 accumulators:
  *    rounding the output to bf16 alone moves it by up to 2^-8 of its
  *    magnitude).  Recurrent states are always fp32.
