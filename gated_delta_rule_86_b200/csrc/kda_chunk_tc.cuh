@@ -21,7 +21,8 @@
 // resident at once (cooperative launch), one CTA per SM:
 //   * chain CTAs (one per (sequence, head) pair in flight; a chain runs its
 //     pairs one after another) copy each chunk image from the chain's ring in a
-//     global workspace (it stays in L2) into a two-deep shared-memory ring and
+//     global workspace (it stays in L2) into a three-slot shared-memory ring,
+//     two chunks ahead of their use, and
 //     run, per chunk, one MMA group [-W ; Qg] S (rows 0-63 give U~ - U, rows
 //     64-127 give Qg S), the U~ epilogue, the MMAs Kd^T U~ and [. ; P] U~ (adding
 //     P U~ to rows 64-127) and the fp32 state update, while dedicated warps store
@@ -31,8 +32,9 @@
 //     transform, then W and U on the tensor cores.  The finished chunk image (-W,
 //     U, Qg = Q exp(G), Kd = K exp(G_last - G), P, gamma = exp(G_last) and a
 //     flag) is bulk-stored into its ring slot and announced through a flag in
-//     global memory (release / acquire at GPU scope); the chain announces in turn
-//     which slots it has copied out.
+//     global memory (a release store; the chain polls it with relaxed loads, as
+//     only its asynchronous copies, which read L2, depend on it); the chain
+//     announces in turn which slots it has copied out.
 // Every producer serves every chain, so the preparation throughput per pair is
 // (SMs - chains) / chains producer CTAs rather than a fixed cluster share.
 // The chain CTA computes all d_v columns of S at once: a tcgen05.mma costs about
@@ -60,6 +62,10 @@
 // result.
 //
 // Packed variable-length batches are scheduled longest-first.
+//
+// Input forms (template argument GK, see GateKind): one log-decay per key channel (KDA), one per
+// head and token (Gated DeltaNet; none at all for DeltaNet), or KDA from the raw projections (q
+// and k L2-normalised, log_alpha = logsigmoid(g), beta = sigmoid(b), all as they are loaded).
 #pragma once
 
 #include <cuda.h>
@@ -439,10 +445,11 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     }
     if (warp >= kRoleWarps + 2) return;   // warps 18, 19 serve the chain CTA only
     if (warp == kRoleWarps + 1) {
-        // ---- item loader: for each item, lane 0 issues the 64-token TMA tiles of log_alpha, k, q,
+        // ---- item loader: for each item, lane 0 issues the 64-token TMA tiles of the gate, k, q,
         //      v (rows past the tensor end read as zero, rows past the sequence end are masked by the
         //      readers) into the A/P operand area once the previous item's UT scratch is dead; the
-        //      warp then stores the item's beta and length into shared memory.  raw_full completes
+        //      warp then stores the item's beta (and, for a per-head gate, the 64 log-decays in place
+        //      of the gate tile) and length into shared memory.  raw_full completes
         //      with both arrivals and the tile bytes.  After the last item a length of -1 (no tiles)
         //      tells the compute warps to stop ----
         float *sBetaIn = reinterpret_cast<float *>(sm + SM::kBetaIn);
