@@ -3,8 +3,11 @@ header declares, and rejects malformed calls on the host before launching."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
+import torch
 
 from gated_delta_rule_86_b200 import _lib
 
@@ -143,3 +146,24 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libkda_b200.so"))
     with pytest.raises(ImportError):
         _lib.load()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_no_cpu_fallback_without_gpu():
+    """Without a GPU every public call raises; nothing is computed on the CPU."""
+    import gated_delta_rule_86_b200 as kda
+    q = torch.zeros(1, 4, 1, 64)
+    g = torch.zeros(1, 4, 1)
+    calls = [
+        lambda: kda.kda_chunk_fwd(q, q, q, q, g),
+        lambda: kda.kda_recurrent_fwd(q, q, q, q, g),
+        lambda: kda.gdn_chunk_fwd(q, q, q, g, g),
+        lambda: kda.kda_chunk_fwd_fused(q, q, q, q, g),
+        lambda: kda.kda_decode_step(q[:, 0], q[:, 0], q[:, 0], q[:, 0], g[:, 0], torch.zeros(1, 1, 64, 64)),
+    ]
+    for call in calls:
+        with pytest.raises((RuntimeError, ValueError, AssertionError)):
+            call()
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1", "--warmup", "3",
+                        "--no-cpu-baseline"], capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert r.returncode != 0 and not any(ln.startswith("{") for ln in r.stdout.splitlines())
