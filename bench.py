@@ -241,6 +241,31 @@ def event_time_ms(fn, n):
     return e0.elapsed_time(e1)
 
 
+def gdn_prefill_block(args, world, a, s0, tokens, token_heads, hbm_peak):
+    """Time gdn_chunk_fwd on the bench workload's q, k, v, beta with the first key channel of its
+    log_alpha as the per-head gate.  Algorithmic bytes: those of the KDA prefill less the
+    per-channel gate (254 B per token-head)."""
+    from gated_delta_rule_86_b200 import gdn_chunk_fwd
+    log_g = a[3][..., 0].contiguous()
+
+    def step(_i):
+        return gdn_chunk_fwd(a[0], a[1], a[2], log_g, a[4], initial_state=s0)
+
+    for _ in range(args.warmup):
+        step(0)
+    barrier(world)
+    ms = event_time_ms(step, args.steps)
+    barrier(world)
+    ms_step = max_over_ranks(ms / args.steps, world)
+    heads = a[0].shape[0] * a[0].shape[2]
+    alg = prefill_alg_bytes(token_heads, heads) - token_heads * (a[3].shape[-1] - 1) * 2
+    gbs = alg / (ms_step * 1e-3) / 1e9
+    return {"entry": "gdn_chunk_fwd", "gate": "log_g [B,T,H] = the first key channel of the workload's log_alpha",
+            "ms_per_step": ms_step, "tokens_per_s": world * tokens / (ms_step * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": None, "kernel": "kda_chunk_tc_kernel", "alg_bytes_per_launch": alg}}
+
+
 def run_kda(args):
     import torch
 
@@ -308,6 +333,8 @@ def run_kda(args):
     e2e_ms = max_over_ranks(e2e_ms / max(1, args.steps // 2), world)
     h2d = sum(t.numel() * t.element_size() for t in host) + s0_h.numel() * 4
     d2h = token_heads * w.dv * 4 + w.B * w.H * w.dk * w.dv * 4
+    # ---------------- Gated DeltaNet on the same workload (one log-decay per head and token) --------
+    gdn = gdn_prefill_block(args, world, a, s0, tokens, token_heads, hbm_peak)
     del host, s0_h, x, a
     torch.cuda.empty_cache()
 
@@ -395,7 +422,8 @@ def run_kda(args):
                 "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 # per step: the schedule-table kernel and the chunk kernel
-                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "fused_prologue": fused}
+                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "fused_prologue": fused,
+                "gated_deltanet": gdn}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
