@@ -38,6 +38,58 @@ DECODE_WORKLOAD = "decode_bf16"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+LIB_SOURCES = ("gated_delta_rule_86_b200/csrc", "include")
+
+
+def build_hash():
+    """Hash of the library's sources (csrc/*.cu, *.cuh, include/*.h): names the build that a
+    profile summary was captured on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = []
+    for d in LIB_SOURCES:
+        for ext in ("*.cu", "*.cuh", "*.h"):
+            files += glob.glob(os.path.join(ROOT, d, ext))
+    for f in sorted(files):
+        h.update(os.path.relpath(f, ROOT).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel, workload):
+    """The DRAM traffic record of `kernel` on `workload` from profiles/*.md (a line
+    `traffic-record: {json}` written next to the ncu summary), if it was captured on the current
+    build; else None.  Keys: build, kernel, workload, dram_bytes, units, units_per_launch."""
+    import glob
+    want = build_hash()
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(f) as fh:
+            for line in fh:
+                if line.startswith("traffic-record:"):
+                    try:
+                        rec = json.loads(line.split(":", 1)[1])
+                    except ValueError:
+                        continue
+                    if rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("build") == want:
+                        rec["file"] = os.path.relpath(f, ROOT)
+                        return rec
+    return None
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -241,6 +293,64 @@ def event_time_ms(fn, n):
     return e0.elapsed_time(e1)
 
 
+def flushed_time_ms(fn, n, flush):
+    """Sum of n per-call CUDA-event times, with `flush` (a write of a buffer larger than L2)
+    before each call and outside its timed interval."""
+    import torch
+    total = 0.0
+    for i in range(n):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn(i)
+        e1.record()
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    return total
+
+
+def timed_steps(fn, args, world, flush=None):
+    """Warm-up, then the device time of args.steps calls between barriers; the max over ranks of
+    the per-call time in ms."""
+    for _ in range(args.warmup):
+        fn(0)
+    barrier(world)
+    ms = event_time_ms(fn, args.steps) if flush is None else flushed_time_ms(fn, args.steps, flush)
+    barrier(world)
+    return max_over_ranks(ms / args.steps, world)
+
+
+def hbm_roofline(alg_bytes, ms, hbm_peak, kernel="kda_chunk_tc_kernel", traffic=None):
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+            "traffic": traffic, "kernel": kernel, "alg_bytes_per_launch": alg_bytes}
+
+
+def prefill_block(args, world, x, hbm_peak, entry="kda_chunk_fwd", out_dtype=None, flush=None, label=None):
+    """Time one prefill entry point on the inputs x (a make_prefill dict on the GPU)."""
+    import torch
+
+    import gated_delta_rule_86_b200 as kda
+    fn = getattr(kda, entry)
+    out_dtype = out_dtype or torch.float32
+    a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+    B, T, H, dk = a[0].shape
+    dv = a[2].shape[-1]
+    N = B if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
+
+    def step(_i):
+        return fn(*a, initial_state=x["init_state"], cu_seqlens=x["cu_seqlens"], out_dtype=out_dtype)
+
+    ms = timed_steps(step, args, world, flush)
+    tokens = B * T
+    alg = prefill_alg_bytes(tokens * H, N * H, dk, dv, out_bytes=4 if out_dtype == torch.float32 else 2)
+    w = x["workload"]
+    return {"entry": entry, "workload": label or w.name, "B": B, "T": T, "H": H, "N": N, "d_k": dk, "d_v": dv,
+            "out_dtype": "f32" if out_dtype == torch.float32 else "bf16", "ms_per_step": ms,
+            "tokens_per_s": world * tokens / (ms * 1e-3), "roofline": hbm_roofline(alg, ms, hbm_peak),
+            "l2": "flushed before each call" if flush is not None else "inputs larger than L2"}
+
+
 def gdn_prefill_block(args, world, a, s0, tokens, token_heads, hbm_peak):
     """Time gdn_chunk_fwd on the bench workload's q, k, v, beta with the first key channel of its
     log_alpha as the per-head gate.  Algorithmic bytes: those of the KDA prefill less the
@@ -251,19 +361,28 @@ def gdn_prefill_block(args, world, a, s0, tokens, token_heads, hbm_peak):
     def step(_i):
         return gdn_chunk_fwd(a[0], a[1], a[2], log_g, a[4], initial_state=s0)
 
-    for _ in range(args.warmup):
-        step(0)
-    barrier(world)
-    ms = event_time_ms(step, args.steps)
-    barrier(world)
-    ms_step = max_over_ranks(ms / args.steps, world)
+    ms_step = timed_steps(step, args, world)
     heads = a[0].shape[0] * a[0].shape[2]
     alg = prefill_alg_bytes(token_heads, heads) - token_heads * (a[3].shape[-1] - 1) * 2
-    gbs = alg / (ms_step * 1e-3) / 1e9
     return {"entry": "gdn_chunk_fwd", "gate": "log_g [B,T,H] = the first key channel of the workload's log_alpha",
             "ms_per_step": ms_step, "tokens_per_s": world * tokens / (ms_step * 1e-3),
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                         "traffic": None, "kernel": "kda_chunk_tc_kernel", "alg_bytes_per_launch": alg}}
+            "roofline": hbm_roofline(alg, ms_step, hbm_peak)}
+
+
+def oracle_single_thread(workload, T_s=4096):
+    """Single-thread oracle tokens/s on one head of the workload (its first T_s tokens)."""
+    import numpy as np
+
+    import oracle
+    from gated_delta_rule_86_b200 import inputs
+    w = inputs.WORKLOADS[workload]
+    x = inputs.make_prefill(w, device="cpu", T=T_s, H=1, B=1)
+    args = [x[n].float().numpy().astype(np.float64) for n in ("q", "k", "v", "log_alpha", "beta")]
+    s0 = None if x["init_state"] is None else x["init_state"].numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.recurrent(*args, init_state=s0, nthreads=1)
+    dt = time.perf_counter() - t0
+    return T_s / dt, f"first {T_s} tokens of one head, 1 thread"
 
 
 def run_kda(args):
@@ -276,7 +395,7 @@ def run_kda(args):
     tc_peak_burst = peaks["bf16_tflops"]
     tc_peak_sust = peaks.get("bf16_tflops_sustained", tc_peak_burst)
 
-    # ---------------- prefill ----------------
+    # ---------------- prefill (the headline: fp32 output, the accumulator precision) ----------------
     w = inputs.WORKLOADS[PREFILL_WORKLOAD]
     x = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank)
     names = ("q", "k", "v", "log_alpha", "beta")
@@ -300,23 +419,31 @@ def run_kda(args):
     value = weak_scaling_value(tokens, world, ms_step)
     alg_bytes = prefill_alg_bytes(token_heads, w.B * w.H)
     alg_flops = prefill_alg_flops(token_heads)
-    achieved_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
     dense_flops = token_heads * (12 * w.chunk * w.dk + 6 * w.dk * w.dv)
-    # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
-    # this kernel on the B=1, H=32, T=16384 case (842.2 MB), scaled to the launch by tokens (the
-    # 4 MB of state traffic does not scale); only valid for the 64K workload of this kernel build.
-    traffic = (842.2e6 - 4.2e6) * (tokens / 16384) + 4.2e6 if (w.B, w.H, w.T) == (1, 32, 65536) else None
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "peak_source": f"{peaks_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                if peaks_src == "measured" else "fallback 6650 GB/s",
-                "kernel": "kda_chunk_tc_kernel", "alg_bytes_per_launch": alg_bytes,
-                "tensor": {"alg_flops_per_launch": alg_flops,
-                           "achieved_tflops": alg_flops / (ms_step * 1e-3) / 1e12,
-                           "frac_of_burst_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst,
-                           "frac_of_sustained_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_sust,
-                           "dense_tile_frac_of_burst_peak":
-                               dense_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst}}
+    # DRAM traffic per launch: from an ncu capture of this very build (a traffic-record line in
+    # profiles/, matched by the hash of the library sources), scaled to this launch by the units it
+    # processes; null when no capture of this build exists
+    rec = traffic_record("kda_chunk_tc_kernel", PREFILL_WORKLOAD)
+    traffic = None
+    if rec is not None:
+        traffic = rec["dram_bytes"] * token_heads / rec["units"]
+    roofline = hbm_roofline(alg_bytes, ms_step, hbm_peak, traffic=traffic)
+    roofline.update({
+        "peak_source": f"{peaks_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+        if peaks_src == "measured" else "fallback 6650 GB/s",
+        "traffic_source": None if rec is None else
+        f"{rec['file']}: ncu dram__bytes_read.sum + dram__bytes_write.sum on {rec['units']} token-heads "
+        f"(build {rec['build']}), scaled by token-heads",
+        "build": build_hash(),
+        "tensor": {"alg_flops_per_launch": alg_flops,
+                   "achieved_tflops": alg_flops / (ms_step * 1e-3) / 1e12,
+                   "frac_of_burst_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst,
+                   "frac_of_sustained_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_sust,
+                   "dense_tile_frac_of_burst_peak": dense_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst}})
+    # the same launch with bf16 output: the byte count of the survey's roofline (1282 B per token-head)
+    bf16_out = prefill_block(args, world, x, hbm_peak, out_dtype=torch.bfloat16)
+    bf16_out["roofline"]["tensor_frac_of_burst_peak"] = alg_flops / (bf16_out["ms_per_step"] * 1e-3) / 1e12 / \
+        tc_peak_burst
     # end to end through the public API from pinned host memory
     host = [t.cpu().pin_memory() for t in a]
     s0_h = s0.cpu().pin_memory()
@@ -327,7 +454,6 @@ def run_kda(args):
 
     e2e_step(0)
     barrier(world)
-    t0 = time.perf_counter()
     e2e_ms = event_time_ms(e2e_step, max(1, args.steps // 2))
     barrier(world)
     e2e_ms = max_over_ranks(e2e_ms / max(1, args.steps // 2), world)
@@ -340,29 +466,32 @@ def run_kda(args):
 
     # ---------------- the same prefill from the raw projections (fused prologue) ----------------
     xr = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank, raw=True)
-    ar = [xr[n] for n in names]
+    fused = prefill_block(args, world, xr, hbm_peak, entry="kda_chunk_fwd_fused")
+    fused["inputs"] = ("raw bf16 q, k (not normalised), g ~ N(4,1), b ~ N(0,1); normalisation, logsigmoid and "
+                       "sigmoid inside the kernel's loads")
+    # what a separate prologue pass would add: write and re-read the activated q, k, log_alpha and beta
+    fused["separate_pass_bytes_saved"] = 2 * token_heads * (3 * w.dk * 2 + 2)
+    del xr
+    torch.cuda.empty_cache()
 
-    def fused_step(_i):
-        return kda_chunk_fwd_fused(*ar, initial_state=s0)
+    # ---------------- the other prefill workloads ----------------
+    others = {}
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
 
-    for _ in range(args.warmup):
-        fused_step(0)
-    barrier(world)
-    fms = event_time_ms(fused_step, args.steps)
-    barrier(world)
-    fms_step = max_over_ranks(fms / args.steps, world)
-    f_gbs = alg_bytes / (fms_step * 1e-3) / 1e9
-    fused = {"entry": "kda_chunk_fwd_fused", "workload": PREFILL_WORKLOAD,
-             "inputs": "raw bf16 q, k (not normalised), g ~ N(4,1), b ~ N(0,1); normalisation, logsigmoid and "
-                       "sigmoid inside the kernel's loads",
-             "ms_per_step": fms_step, "tokens_per_s": world * tokens / (fms_step * 1e-3),
-             "roofline": {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
-                          "frac": f_gbs / hbm_peak, "traffic": None, "kernel": "kda_chunk_tc_kernel",
-                          "alg_bytes_per_launch": alg_bytes},
-             # what a separate prologue pass would add: write and re-read the activated q, k,
-             # log_alpha (bf16) and beta
-             "separate_pass_bytes_saved": 2 * token_heads * (3 * w.dk * 2 + 2)}
-    del xr, ar, s0
+    def flush():
+        flush_buf.zero_()
+
+    for name, fl in (("prefill_bf16", flush), ("varlen_bf16", None)):
+        wo = inputs.WORKLOADS[name]
+        xo = inputs.make_prefill(wo, device="cuda", seed=inputs.BASE_SEED + wo.wid + 1000 * rank)
+        others[name] = prefill_block(args, world, xo, hbm_peak, flush=fl)
+        if wo.varlen:
+            lens = (xo["cu_seqlens"][1:] - xo["cu_seqlens"][:-1]).tolist()
+            others[name]["seq_lens"] = lens
+            # the longest sequence's chain is the critical path of a longest-first schedule
+            others[name]["longest_seq_tokens"] = max(lens)
+        del xo
+    del flush_buf
     torch.cuda.empty_cache()
 
     # ---------------- decode ----------------
@@ -409,7 +538,10 @@ def run_kda(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             tps, sample, threads, _ = time_oracle(PREFILL_WORKLOAD, target_s=args.ref_seconds)
-            cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+            tps1, sample1 = oracle_single_thread(PREFILL_WORKLOAD)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample,
+                   "cpu_model": cpu_model(), "single_thread": {"value": tps1, "unit": "tokens/s (one head)",
+                                                               "sample": sample1}}
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -422,8 +554,8 @@ def run_kda(args):
                 "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 # per step: the schedule-table kernel and the chunk kernel
-                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "fused_prologue": fused,
-                "gated_deltanet": gdn}
+                "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "bf16_output": bf16_out,
+                "fused_prologue": fused, "gated_deltanet": gdn, "other_prefill_workloads": others}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -13,7 +13,8 @@ KDA_F32, KDA_BF16 = 0, 1
 # every symbol include/kda.h declares
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_static_ws", "kda_recurrent_fwd",
             "kda_decode_step", "gdn_chunk_fwd", "gdn_recurrent_fwd", "gdn_decode_step", "kda_chunk_fwd_fused",
-            "kda_decode_step_fused", "kda_status_string", "kda_get_last_device_error", "kda_version")
+            "kda_decode_step_fused", "kda_status_string", "kda_get_last_device_error", "kda_version",
+            "kda_testing_set_chunk_fault")
 
 _lib = None
 
@@ -58,6 +59,8 @@ def load() -> ctypes.CDLL:
     lib.kda_get_last_device_error.restype = ctypes.c_int
     lib.kda_version.argtypes = []
     lib.kda_version.restype = ctypes.c_char_p
+    lib.kda_testing_set_chunk_fault.argtypes = [i32, ctypes.c_uint32]
+    lib.kda_testing_set_chunk_fault.restype = ctypes.c_int
     _lib = lib
     return lib
 

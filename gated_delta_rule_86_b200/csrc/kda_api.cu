@@ -102,14 +102,18 @@ constexpr int kMaxDevices = 64;
 std::mutex g_static_ws_mutex;
 void *g_static_ws_addr[kMaxDevices] = {};
 
-// Device address of the current device's copy of g_static_ws, looked up once
-// per device (with that device current) and cached.
-kda_status static_ws_address(void **addr) {
+// Device address of the current device's copy of g_static_ws.  It is looked up with that device
+// current and cached per device.  Outside stream capture it is looked up again on every call (a
+// cheap runtime query), so that a cached address never outlives a device reset; during capture
+// the cached address is used, because the lookup may load the module, which capture forbids.
+kda_status static_ws_address(void **addr, cudaStream_t stream) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-    if (!g_static_ws_addr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone || !g_static_ws_addr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return KDA_ERR_CUDA;
         g_static_ws_addr[dev] = p;
@@ -133,7 +137,15 @@ const char *kda_status_string(kda_status s) {
     return "KDA_ERR_UNKNOWN";
 }
 
-const char *kda_version(void) { return "kda_b200 0.1.0 sm_100a"; }
+const char *kda_version(void) { return "kda_b200 0.2.0 sm_100a"; }
+
+kda_status kda_testing_set_chunk_fault(int32_t skip_item, uint32_t flag_wait_us) {
+    if (skip_item < -1) return KDA_ERR_INVALID_ARG;
+    kda::ChunkFault &f = kda::chunk_fault();
+    f.skip_item = skip_item;
+    f.flag_wait_ns = flag_wait_us ? (uint64_t)flag_wait_us * 1000u : kda::tc::kFlagWaitNs;
+    return KDA_OK;
+}
 
 kda_status kda_get_last_device_error(void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -190,7 +202,7 @@ kda_status chunk_impl(int gate, bool static_ws, const void *q, const void *k, co
         const int64_t chains = pairs < kda::kMaxChains ? pairs : kda::kMaxChains;
         if (kda::flags_region_bytes() + (size_t)chains * kda::kMinRing * kda::img_stride(d_v) > KDA_STATIC_WS_BYTES)
             return KDA_ERR_UNSUPPORTED;
-        s = static_ws_address(&workspace);
+        s = static_ws_address(&workspace, st);
         if (s != KDA_OK) return s;
         workspace_bytes = KDA_STATIC_WS_BYTES;
     } else {
@@ -261,6 +273,8 @@ kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     *bytes = 0;
     if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    // the bf16 tensor-core path takes d_k == 128 only (kda_chunk_fwd rejects the rest)
+    if (dtype == KDA_BF16 && d_k != 128) return KDA_ERR_UNSUPPORTED;
     if (dtype == KDA_BF16) *bytes = kda::chunk_tc_workspace_bytes((int64_t)N * H, d_v);
     return KDA_OK;
 }

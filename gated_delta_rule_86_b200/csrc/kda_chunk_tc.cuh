@@ -290,6 +290,8 @@ struct ChunkSched {
     int *ready;             // [nchain][ring]: 1 + number of the chunk whose image the slot holds
     int *consumed;          // [nchain]: chunks the chain has copied out of its ring
     uint8_t *rings;         // [nchain][ring] chunk images (Img layout, Img::kStride apart)
+    tc::FlagWait fw;        // limit of the waits on the flags above, and the launch's abort word
+    int skip_item;          // testing hook: the producer item whose image is never published (-1: none)
 };
 
 // One (sequence, head) pair.
@@ -429,8 +431,12 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                 const int slot = it.t % sched.ring;
                 uint8_t *gimg = sched.rings + ((size_t)it.k * sched.ring + slot) * I::kStride;
                 // the chain has copied out the slot's previous image (chunk t - ring)
-                if (!tc::flag_wait_ge(sched.consumed + it.k, it.t - sched.ring + 1, abort_flag)) break;
+                if (!tc::flag_wait_ge(sched.consumed + it.k, it.t - sched.ring + 1, abort_flag, sched.fw)) break;
                 if (!tc::mbar_wait(&bars.staged, kl & 1, abort_flag)) break;
+                if (it.i == sched.skip_item) {   // testing hook: this image is never published
+                    tc::mbar_arrive(&bars.staging_free);
+                    continue;
+                }
                 tc::fence_async_global();
                 tc::bulk_store_nc(gimg, sm + SM::kImg, I::kBytes);
                 tc::bulk_commit();
@@ -983,10 +989,16 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         const bool lead_ld = warp == kRoleWarps && lane == 1;
         const uint32_t tlo = tc::tmem_lane_base(warp);
         constexpr uint32_t kOutThreads = kThreads - kRoleThreads;
-        int last_load = -1;
+        // chunk whose image copy was issued last into each shared-memory slot (-1: none); the CTA
+        // waits for exactly these copies before it leaves
+        int pend[SM::kSlots];
+#pragma unroll
+        for (int i = 0; i < SM::kSlots; ++i) pend[i] = -1;
         auto load_image = [&](int t) -> bool {   // lane 1 of warp 16
+            if (*abort_flag) return false;
             const int rs = kc * sched.ring + t % sched.ring;
-            if (!tc::flag_wait_ge(sched.ready + rs, t + 1, abort_flag)) return false;
+            if (!tc::flag_wait_ge(sched.ready + rs, t + 1, abort_flag, sched.fw)) return false;
+            if (*abort_flag) return false;
             tc::fence_async_global();
             const uint8_t *src = sched.rings + (size_t)rs * I::kStride;
             uint8_t *slot = sm + (t % SM::kSlots) * SM::kSlotBytes;
@@ -998,7 +1010,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
             tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
             tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
-            last_load = t;
+            pend[t % SM::kSlots] = t;
             return true;
         };
         if (lead_ld)
@@ -1106,10 +1118,12 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         }
         if (lead) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
         if (lead_ld) {
-            // no image copy may still be in flight either
+            // no image copy may still be in flight either (only copies that were issued are awaited:
+            // after an abort some chunks' copies never were)
             int never = 0;
-            for (int tt = (last_load >= 2 ? last_load - 2 : 0); tt <= last_load; ++tt)
-                tc::mbar_wait(&bars.full[tt % SM::kSlots], (tt / SM::kSlots) & 1, &never);
+#pragma unroll
+            for (int i = 0; i < SM::kSlots; ++i)
+                if (pend[i] >= 0) tc::mbar_wait(&bars.full[i], (pend[i] / SM::kSlots) & 1, &never);
         }
         return;
     }
@@ -1454,7 +1468,8 @@ inline ChunkGrid chunk_grid(int64_t npairs, int nsm) {
 constexpr int kRing = 12;                // ring slots per chain (workspace variant)
 constexpr int kMinRing = 3;
 constexpr int kMaxChains = 64;
-constexpr size_t kFlagsBytes = 4096 + (size_t)(kMaxChains * kRing + kMaxChains) * 4;   // order + flags
+// sequence order (4 KB), then the ready flags, the consumed counters and the abort word
+constexpr size_t kFlagsBytes = 4096 + (size_t)(kMaxChains * kRing + kMaxChains + 1) * 4;
 template <int DV> constexpr size_t ring_stride() { return Img<DV>::kStride; }
 inline size_t img_stride(int DV) { return DV == 64 ? Img<64>::kStride : Img<128>::kStride; }
 inline size_t flags_region_bytes() { return (kFlagsBytes + 1023) / 1024 * 1024; }
@@ -1509,6 +1524,17 @@ inline int device_sm_count() {
     return cache[dev];
 }
 
+// Testing hook of the chunk kernel: the producer item whose image is never published (-1: none)
+// and the limit of the waits on the ring flags.  Process-wide, read at each launch.
+struct ChunkFault {
+    int skip_item = -1;
+    uint64_t flag_wait_ns = tc::kFlagWaitNs;
+};
+inline ChunkFault &chunk_fault() {
+    static ChunkFault f;
+    return f;
+}
+
 // Launches the schedule-table kernel and the chunk kernel.  `ws_bytes` bounds the ring depth: the
 // workspace holds the schedule tables and nchain rings of `ring` images (kMinRing <= ring <= kRing).
 template <int DV, typename TO, int GK>
@@ -1558,7 +1584,10 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
     sched.ready = reinterpret_cast<int *>(ws + 4096);
     sched.consumed = sched.ready + grid.nchain * sched.ring;
     sched.rings = ws + flags;
-    const int nflags = grid.nchain * sched.ring + grid.nchain;
+    sched.fw.abort_all = sched.consumed + grid.nchain;
+    sched.fw.limit_ns = chunk_fault().flag_wait_ns;
+    sched.skip_item = chunk_fault().skip_item;
+    const int nflags = grid.nchain * sched.ring + grid.nchain + 1;
     kda_chunk_sched_kernel<<<1, 256, 0, stream>>>(cu, num_seqs, sorted ? reinterpret_cast<int32_t *>(ws) : nullptr,
                                                   sched.ready, nflags);
     e = cudaGetLastError();

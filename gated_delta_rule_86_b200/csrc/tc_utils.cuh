@@ -123,22 +123,42 @@ __device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
     asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Wait until *p >= v, bounded by kFlagWaitNs; same contract as mbar_wait.  The flags are progress
-// counters whose writers completed the data they announce (to global memory, the coherence point)
-// before the store; the waiting thread only lets asynchronous copies (which read from L2) or its
-// own later bulk stores depend on them, so relaxed polling suffices (an acquire fence here cost
-// about 0.8 us per wait).
-__device__ __forceinline__ bool flag_wait_ge(const int *p, int v, volatile int *abort) {
-    if (ld_relaxed_gpu(p) >= v) return true;
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Launch-wide limits of the waits on global flags, and the launch's abort word (in the workspace,
+// zeroed before each launch): a CTA whose wait runs out sets it, and every other CTA's flag waits
+// see it within a few microseconds and give up too, so that one timeout ends the whole grid
+// quickly instead of one wait limit per dependent CTA.
+struct FlagWait {
+    uint64_t limit_ns;
+    int *abort_all;
+};
+// Wait until *p >= v; same contract as mbar_wait (records the error word and sets *abort on
+// timeout, returns false at once once *abort is set).  The flags are progress counters released
+// by their writers (st.release.gpu after the data they announce is complete in global memory);
+// every poll is an acquire load, so the waiting thread's later accesses, including the bulk copies
+// it issues after a proxy fence, are ordered after the announced data.
+__device__ __forceinline__ bool flag_wait_ge(const int *p, int v, volatile int *abort, const FlagWait &fw) {
+    if (ld_acquire_gpu(p) >= v) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0;; ++i) {
         __nanosleep(32);
-        if (ld_relaxed_gpu(p) >= v) return true;
+        if (ld_acquire_gpu(p) >= v) return true;
         if (*abort) return false;
-        if ((i & 255u) == 255u && global_ns() - t0 > kFlagWaitNs) break;
+        if ((i & 255u) == 255u) {
+            if (ld_relaxed_gpu(fw.abort_all) != 0) {   // another CTA gave up: leave as well
+                *abort = 1;
+                return false;
+            }
+            if (global_ns() - t0 > fw.limit_ns) break;
+        }
     }
     record_device_error(kDevErrTimeout);
     *abort = 1;
+    st_relaxed_gpu(fw.abort_all, 1);
     return false;
 }
 

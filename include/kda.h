@@ -119,7 +119,9 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
  * chains, a ring of 12 chunk images (73 KB each at d_v = 128, 65 KB at
  * d_v = 64) through which the CTAs that prepare the chunk operands hand them
  * to the CTA that runs the state recurrence; 0 on the fp32 path.  Pure host
- * computation, never fails for valid sizes.
+ * computation.  KDA_ERR_UNSUPPORTED (and *bytes = 0) for the shapes that
+ * kda_chunk_fwd rejects with that status: d_k or d_v outside {64, 128}, and
+ * KDA_BF16 with d_k != 128.
  */
 kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32_t d_v,
                                         kda_dtype dtype, size_t *bytes);
@@ -229,8 +231,12 @@ kda_status kda_decode_step_fused(const void *q_raw, const void *k_raw, const voi
  * allocator).  Any number of (sequence, head) pairs fits: the chains' rings
  * are made shallower (down to 3 images) when the array cannot hold 12 each.
  *
- * The first call on a device looks up that device's copy of the array (with
- * the device current), so make that first call before any stream capture.
+ * Each call looks up the current device's copy of the array (with that
+ * device current) and caches its address per device; during stream capture
+ * the cached address is used, so make the first call on a device before any
+ * capture.  Outside capture the address is looked up again on every call, so
+ * a device reset (cudaDeviceReset) between calls is harmless; a graph captured
+ * before such a reset keeps the old address and must be captured again.
  * Every call on a device shares the one array and leaves its last contents
  * there; nothing in it needs to start at zero, since each chunk image is
  * written before it is read.  Two calls that run on the same GPU at the same
@@ -255,8 +261,27 @@ const char *kda_status_string(kda_status s);
  */
 kda_status kda_get_last_device_error(void *stream);
 
-/* Library version string, e.g. "kda_b200 0.1.0 sm_100a". */
+/* Library version string, e.g. "kda_b200 0.2.0 sm_100a". */
 const char *kda_version(void);
+
+/*
+ * Testing hook (not part of the operator): makes the tensor-core prefill's
+ * failure path observable without a GPU fault.  After this call, every
+ * launch of the prefill's tensor-core kernel (kda_chunk_fwd, gdn_chunk_fwd,
+ * kda_chunk_fwd_fused, kda_chunk_fwd_static_ws) leaves the chunk image of
+ * producer item `skip_item` unpublished (-1: none, the default), and every
+ * wait on a ring flag gives up after `flag_wait_us` microseconds (0: the
+ * default of 2 s).  A launch whose image is missing then ends on its own:
+ * the waiting CTA records KDA_ERR_TIMEOUT in the device error word, raises
+ * the launch's abort word, and every CTA leaves its loops and frees its
+ * Tensor Memory; the outputs of that launch are undefined, and
+ * kda_get_last_device_error reports KDA_ERR_TIMEOUT.  Items are numbered in
+ * schedule order (item i is chunk i / C of chain i % C for C chains), so any
+ * value below the number of chunks of the launch takes effect.  Process-wide;
+ * not thread-safe against concurrent prefill calls.  KDA_ERR_INVALID_ARG for
+ * skip_item < -1.
+ */
+kda_status kda_testing_set_chunk_fault(int32_t skip_item, uint32_t flag_wait_us);
 
 #ifdef __cplusplus
 }

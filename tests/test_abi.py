@@ -141,6 +141,20 @@ def test_workspace_size(lib):
         _lib.KDA_ERR_INVALID_ARG
 
 
+def test_workspace_size_rejects_what_the_prefill_rejects(lib):
+    """The size query answers KDA_ERR_UNSUPPORTED (size 0) exactly for the head sizes that
+    kda_chunk_fwd itself rejects as unsupported, so a query never succeeds for a shape the
+    prefill cannot run."""
+    n = ctypes.c_size_t(7)
+    for dk, dv, dt in [(96, 128, _lib.KDA_BF16), (128, 96, _lib.KDA_BF16), (96, 64, _lib.KDA_F32)]:
+        n.value = 7
+        assert lib.kda_chunk_fwd_workspace_size(2, 16, dk, dv, dt, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+        assert n.value == 0
+    # shapes the prefill accepts get a size (fp32: the CUDA-core path, no workspace)
+    for dk, dv, dt in [(128, 64, _lib.KDA_BF16), (64, 64, _lib.KDA_F32), (64, 128, _lib.KDA_F32)]:
+        assert lib.kda_chunk_fwd_workspace_size(2, 16, dk, dv, dt, ctypes.byref(n)) == _lib.KDA_OK
+
+
 def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libkda_b200.so"))

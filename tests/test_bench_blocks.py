@@ -39,3 +39,54 @@ def test_gdn_prefill_block(monkeypatch):
     assert out["roofline"]["alg_bytes_per_launch"] == alg
     assert abs(out["roofline"]["frac"] - alg / 2e-3 / 1e9 / 6000.0) < 1e-12
     json.dumps(out)
+
+
+def test_prefill_block_bytes_follow_out_dtype(monkeypatch):
+    seen = []
+
+    def fake_chunk(q, k, v, la, beta, initial_state=None, cu_seqlens=None, out_dtype=None):
+        seen.append(out_dtype)
+        return None, None
+
+    monkeypatch.setattr(pkg, "kda_chunk_fwd", fake_chunk)
+    monkeypatch.setattr(bench, "barrier", lambda world, device="cuda": None)
+    monkeypatch.setattr(bench, "event_time_ms", lambda fn, n: [fn(i) for i in range(n)] and 3.0 * n)
+    B, T, H, d = 1, 256, 2, 128
+    z = torch.zeros(B, T, H, d)
+    from gated_delta_rule_86_b200 import inputs
+    x = dict(q=z, k=z, v=z, log_alpha=z, beta=torch.zeros(B, T, H), init_state=None, cu_seqlens=None,
+             workload=inputs.WORKLOADS["prefill_bf16"])
+    args = SimpleNamespace(warmup=3, steps=4)
+    o32 = bench.prefill_block(args, 1, x, 6000.0)
+    o16 = bench.prefill_block(args, 1, x, 6000.0, out_dtype=torch.bfloat16)
+    assert seen == [torch.float32] * 7 + [torch.bfloat16] * 7
+    assert o32["ms_per_step"] == 3.0 and o32["tokens_per_s"] == B * T / 3e-3
+    # fp32 output: 1538 B per token-head; bf16 output: 1282 B (plus the state once per sequence-head)
+    state = B * H * 2 * d * d * 4
+    assert o32["roofline"]["alg_bytes_per_launch"] == B * T * H * 1538 + state
+    assert o16["roofline"]["alg_bytes_per_launch"] == B * T * H * 1282 + state
+    json.dumps(o32)
+
+
+def test_traffic_record_needs_the_current_build(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    for d in bench.LIB_SOURCES:
+        (tmp_path / d).mkdir(parents=True)
+    (tmp_path / "include" / "kda.h").write_text("int x;\n")
+    h = bench.build_hash()
+    assert h == bench.build_hash() and len(h) == 16
+    rec = {"build": h, "kernel": "kda_chunk_tc_kernel", "workload": "long_bf16", "dram_bytes": 1000, "units": 10}
+    (tmp_path / "profiles" / "k.md").write_text("# summary\ntraffic-record: " + json.dumps(rec) + "\n")
+    got = bench.traffic_record("kda_chunk_tc_kernel", "long_bf16")
+    assert got is not None and got["dram_bytes"] == 1000 and got["file"] == os.path.join("profiles", "k.md")
+    assert bench.traffic_record("kda_chunk_tc_kernel", "prefill_bf16") is None
+    # any change to the library sources makes the record stale
+    (tmp_path / "include" / "kda.h").write_text("int y;\n")
+    assert bench.build_hash() != h
+    assert bench.traffic_record("kda_chunk_tc_kernel", "long_bf16") is None
+
+
+def test_cpu_model_is_text_or_none():
+    m = bench.cpu_model()
+    assert m is None or (isinstance(m, str) and m)

@@ -8,7 +8,7 @@ import torch
 import oracle
 from gated_delta_rule_86_b200 import (KdaError, device_error, inputs, kda_chunk_fwd, kda_chunk_fwd_fused,
                                       kda_decode_step_fused)
-from parity import BF16_TOL, FP32_TOL, NAMES, np64, rel_err
+from parity import BF16_TOL, FP32_TOL, NAMES, check_heads_in_groups, np64, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +43,7 @@ def test_fused_chunk_ragged(cuda_lib, T):
 @pytest.mark.parametrize("dv", [64, 128])
 def test_fused_chunk_many_pairs(cuda_lib, dv):
     x = inputs.make_prefill("prefill_bf16", device="cpu", raw=True, B=2, T=150, H=40, dv=dv, init_state=True)
-    check_chunk(x, heads=[0, 21, 39])
+    check_chunk(x)
 
 
 def test_fused_chunk_strong_decay(cuda_lib):
@@ -61,8 +61,19 @@ def test_fused_chunk_varlen(cuda_lib):
     check_chunk(x)
 
 
-def test_fused_long_full_sampled(cuda_lib):
-    check_chunk(inputs.make_prefill("long_bf16", device="cuda", raw=True), heads=[0, 31])
+def test_fused_long_full(cuda_lib):
+    """The long workload from its raw projections, every head against oracle.prologue + the
+    recurrence."""
+    x = inputs.make_prefill("long_bf16", device="cuda", raw=True)
+    out, fs = kda_chunk_fwd_fused(*(x[n] for n in NAMES), initial_state=x["init_state"])
+    torch.cuda.synchronize()
+    assert device_error() == 0
+
+    def ref(xs):
+        q, k, la, beta = oracle.prologue(*(np64(xs[n]) for n in ("q", "k", "log_alpha", "beta")))
+        return oracle.recurrent(q, k, np64(xs["v"]), la, beta, init_state=np64(xs["init_state"]))
+
+    check_heads_in_groups(out, fs, x, ref, BF16_TOL)
 
 
 def test_fused_equals_unfused_on_activated_inputs(cuda_lib):
