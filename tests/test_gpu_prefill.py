@@ -196,8 +196,18 @@ def test_varlen_bf16_full(cuda_lib):
 
 
 def test_long_bf16_full_bf16_output(cuda_lib):
-    """The bench's bf16-output variant of the long workload, every head."""
-    run_full("long_bf16", out_dtype=torch.bfloat16)
+    """The bench's bf16-output variant of the long workload, every head: bitwise the fp32 output
+    rounded to nearest bf16 (the fp32 output's parity is test_long_bf16_full).  The bf16 rounding
+    alone moves the largest outputs by up to 2^-9 of their magnitude, which on this workload is
+    about 2e-2 of rms(out): the parity bound is met by the fp32 output, not by its bf16 copy."""
+    x = inputs.make_prefill("long_bf16", device="cuda")
+    a = [x[n] for n in NAMES]
+    o32, f32 = kda_chunk_fwd(*a, initial_state=x["init_state"])
+    o16, f16 = kda_chunk_fwd(*a, initial_state=x["init_state"], out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(f16, f32)
 
 
 @pytest.mark.parametrize("fn", [kda_chunk_fwd, kda_recurrent_fwd])
