@@ -12,6 +12,8 @@ Contents
     Through the Long-Context Engineering Bottleneck in LLMs"), in plain C
     (``kda_oracle.c``), fp64, threaded over (sequence, head) pairs.
   * :func:`decode_step` -- one iteration of the same loop body, in place.
+  * :func:`backward` -- the gradient of :func:`recurrent` with respect to every
+    input (reverse mode through the same token steps, fp64 C).
   * :func:`gdn_recurrent`, :func:`gdn_decode_step` -- Gated DeltaNet (one
     decay per head and token) and DeltaNet (no decay): the same recurrence
     with every key channel sharing the head's decay, the scalar-gate and
@@ -69,6 +71,9 @@ def _load():
         lib.kda_oracle_recurrent.restype = ctypes.c_int
         lib.kda_oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, dp, i64, i64, i64, i64]
         lib.kda_oracle_decode_step.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [dp, dp, dp, dp, dp, dp, i64p, i64, i64, i64, i64, i64, i64,
+                                            dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.kda_oracle_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -133,6 +138,40 @@ def decode_step(q, k, v, log_alpha, beta, state):
     return out, S
 
 
+def backward(q, k, v, log_alpha, beta, d_out, init_state=None, d_final_state=None, cu_seqlens=None,
+             nthreads=None):
+    """Gradients of :func:`recurrent` (reverse mode, fp64): given ``d_out`` = dLoss/dout
+    [B, T, H, d_v] and ``d_final_state`` = dLoss/dfinal_state [N, H, d_k, d_v] (None: zero),
+    returns ``(dq, dk, dv, dlog_alpha, dbeta, d_init_state)`` with the shapes of q, k, v,
+    log_alpha, beta and the initial state.  The adjoint of each token step is written out in
+    ``kda_oracle.c``; the forward states are kept for the whole sequence."""
+    q, k, v, log_alpha, beta, d_out = (_f64(x) for x in (q, k, v, log_alpha, beta, d_out))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and log_alpha.shape == q.shape and d_out.shape == v.shape
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    s0 = None if init_state is None else _f64(init_state)
+    dfin = None if d_final_state is None else _f64(d_final_state)
+    for x in (s0, dfin):
+        if x is not None:
+            assert x.shape == (N, H, dk, dv)
+    grads = [np.zeros(q.shape), np.zeros(q.shape), np.zeros(v.shape), np.zeros(q.shape), np.zeros(beta.shape),
+             np.zeros((N, H, dk, dv))]
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().kda_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(s0),
+                                     _ptr(cu, ctypes.c_int64), N, B, T, H, dk, dv, _ptr(d_out), _ptr(dfin),
+                                     *(_ptr(g) for g in grads), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments" if rc == -1 else "oracle ran out of memory")
+    return tuple(grads)
+
+
 NORM_EPS = 1e-6
 
 
@@ -172,4 +211,5 @@ def gdn_decode_step(q, k, v, log_g, beta, state):
 
 from .chunkwise import chunkwise  # noqa: E402  (NumPy restatement, see module docstring)
 
-__all__ = ["build_oracle", "recurrent", "decode_step", "gdn_recurrent", "gdn_decode_step", "prologue", "chunkwise"]
+__all__ = ["build_oracle", "recurrent", "decode_step", "backward", "gdn_recurrent", "gdn_decode_step", "prologue",
+           "chunkwise"]
