@@ -94,37 +94,35 @@ constexpr int kRoleWarps = 16;                        // warps 0-15 run the role
 constexpr int kRoleThreads = kRoleWarps * 32;
 constexpr int kThreads = kRoleThreads + 128;          // + four helper warps that move data
 constexpr uint32_t kBarRole = 1, kBarOut = 2;          // named barriers: role warps, helper warps
+constexpr uint32_t kBarUt = 3;                         // producer warps 0-7 inside the UT transform
 
-// ---- chunk image in the global workspace (fp16 tiles in their shared-memory layouts) ----------
+// ---- chunk image (fp16 tiles in their shared-memory layouts) -----------------------------------
+// The same bytes serve as the producer's staging area, the ring slot in the global workspace and the
+// chain's shared-memory slot, so that one bulk copy moves a whole image.  A1 = [-W ; Qg] as two 16 KB
+// k-blocks of 128 rows (rows 0-63 -W, rows 64-127 Qg: the B operand of S^T [-W ; Qg]^T), then U^T,
+// Kd, tril(P), gamma = exp(G_last) and the exact-path flag.
 template <int DV> struct Img {
-    static constexpr int kNW = 0;                          // -W  [64 x 128]
-    static constexpr int kUT = kNW + kChunk * kDK * 2;     // U^T [DV x 64]
-    static constexpr int kQt = kUT + kChunk * DV * 2;      // Qg  [64 x 128]
-    static constexpr int kKd = kQt + kChunk * kDK * 2;     // Kd  [64 x 128]
-    static constexpr int kP = kKd + kChunk * kDK * 2;      // tril(P) [64 x 64] (after Kd: [Kd ; P] rows)
+    static constexpr int kA1 = 0;                          // [-W ; Qg] [128 x 128]
+    static constexpr int kUT = kA1 + 2 * kChunk * kDK * 2; // U^T [DV x 64]
+    static constexpr int kKd = kUT + kChunk * DV * 2;      // Kd  [64 x 128]
+    static constexpr int kP = kKd + kChunk * kDK * 2;      // tril(P) [64 x 64]
     static constexpr int kGam = kP + kChunk * kChunk * 2;  // fp32 [128] exp(G_last)
     static constexpr int kFlag = kGam + kDK * 4;           // int: 1 = evaluate exactly
     static constexpr int kBytes = kFlag + 16;
     static constexpr int kStride = (kBytes + 1023) / 1024 * 1024;
+    static_assert(kBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
+// Byte offsets of row r's 16-byte chunk j (8 channels) of -W and of Qg inside A1.
+__device__ __forceinline__ uint32_t a1_nw(int r, int j) { return (j >> 3) * (2 * kChunk * 128) + tc::sw128(r, j & 7); }
+__device__ __forceinline__ uint32_t a1_qg(int r, int j) { return a1_nw(r + kChunk, j); }
 
 // ---- chain CTA shared memory ------------------------------------------------------------------
 template <int DV> struct ChainSmem {
     using I = Img<DV>;
-    // one slot of the three-slot image ring: A1 = [-W ; Qg] as two 16 KB k-blocks of 128 rows (rows
-    // 0-63 -W, rows 64-127 Qg; the B operand of S^T A1^T), then U^T, then Kd, P, gamma, flag in
-    // image order.  Once MMA1 of the slot's chunk has completed, A1 is dead and stages that chunk's
-    // output (DV / 64 blocks of [64 tokens x 64 values], fp32 or bf16, one TMA tensor store each).
-    static constexpr int kA1 = 0;
-    static constexpr int kUT = 2 * kChunk * kDK * 2;
-    static constexpr int kKd = kUT + kChunk * DV * 2;
-    static constexpr int kP = kKd + (I::kP - I::kKd);
-    static constexpr int kGam = kKd + (I::kGam - I::kKd);
-    static constexpr int kFlag = kKd + (I::kFlag - I::kKd);
-    static constexpr int kTailBytes = I::kBytes - I::kKd;
-    static constexpr int kSlotBytes = (kKd + kTailBytes + 1023) / 1024 * 1024;
+    // three image slots (Img layout); a slot is free again once the last MMA of its chunk completed
+    static constexpr int kSlotBytes = I::kStride;
     static constexpr int kSlots = 3;
-    static_assert(kChunk * DV * 4 <= kUT - kA1, "output staging fits the dead A1 area");
+    static_assert(kChunk * DV * 4 <= I::kUT - I::kA1, "output staging fits the dead A1 area");
     // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel quarter, k . q
     static constexpr int kRedPk = kSlots * kSlotBytes;
     static constexpr int kRedPq = kRedPk + 4 * 128 * 4;
@@ -365,6 +363,9 @@ struct ChunkCtx {
 struct ChunkBars {
     // chain: image slot full / free, MMA completions
     uint64_t full[3], slot_free[3], mma1, mma2, mma3[2];
+    // chain: 1 + the chunk in which some state thread saw an fp16 overflow of U~ (ut) or of the state
+    // operand (st); set before a plain barrier and compared with the chunk after it
+    int ovf_ut, ovf_st;
     // chain: chunk evaluation mode handed to the output warps, TMEM accumulator read by them
     uint64_t outq[2], d1_free[2];
     int outmode[2];   // 0: no MMAs issued, 1: MMAs issued but evaluated exactly, 2: tensor output
@@ -381,6 +382,46 @@ struct ChunkBars {
 struct RowMaps {
     CUtensorMap g, k, q, v, o;
 };
+
+// ---- warp-level tf32 MMAs for the small products of the UT transform ----------------------------
+// Fragment layouts of mma.sync m16n8k8 (tf32): with g = lane / 4 and t = lane % 4, A (16 x 8) holds
+// (g, t), (g + 8, t), (g, t + 4), (g + 8, t + 4); B (8 x 8) holds (t, g), (t + 4, g); C (16 x 8) holds
+// (g, 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// acc (+)= A[16 x 8 KS] B[8 KS x 8], row-major fp32 operands in shared memory (leading dimensions la, lb)
+template <int KS>
+__device__ __forceinline__ void mma_tile_16x8(float (&acc)[4], const float *A, int la, const float *B, int lb, int g,
+                                              int t) {
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        const float *a = A + 8 * ks, *b = B + 8 * ks * lb;
+        const uint32_t af[4] = {to_tf32(a[g * la + t]), to_tf32(a[(g + 8) * la + t]), to_tf32(a[g * la + t + 4]),
+                                to_tf32(a[(g + 8) * la + t + 4])};
+        const uint32_t bf[2] = {to_tf32(b[t * lb + g]), to_tf32(b[(t + 4) * lb + g])};
+        mma_16x8x8_tf32(acc, af, bf);
+    }
+}
+// acc = A[16 x K] B[K x 16] as two 16 x 8 column tiles (K = 16)
+template <int K>
+__device__ __forceinline__ void mma_block_16x16(float (&acc)[2][4], const float *A, int la, const float *B, int lb,
+                                                int g, int t) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+        mma_tile_16x8<K / 8>(acc[nt], A, la, B + 8 * nt, lb, g, t);
+    }
+}
 
 // ======================================== producer role ==========================================
 // Producer j prepares its items (see ChunkSched) with warps 0-15.  Lane 0 of warp 16 stores each
@@ -708,7 +749,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                 }
                 const uint32_t o128 = tile_chunk(r, cg, kChunk);   // [64 x 128] tiles
                 *reinterpret_cast<uint4 *>(sm + SM::kKgV + o128) = pack8_h(kg);
-                *reinterpret_cast<uint4 *>(img + I::kQt + o128) = pack8_h(qg);
+                *reinterpret_cast<uint4 *>(img + I::kA1 + a1_qg(r, cg)) = pack8_h(qg);
                 unpack8(rv[rr], vf);   // zero past DV
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ovf |= !(fabsf(vf[i]) <= 65000.f);
@@ -809,77 +850,61 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
         }
         tc::named_sync(kBarRole, kRoleThreads);
         // (b) the blocks below the diagonal, as two levels of the 2x2 block inverse
-        //     [[Ta, 0], [Lba, Tb']]^{-1} = [[Ta, 0], [-Tb' Lba Ta, Tb']], fp32 on CUDA cores.
-        //     Level 1 (16-row blocks): T10 and T32; level 2 (32-row blocks): the lower-left 32x32
-        //     block.  Each product goes through the scratch tile X; a thread reads a row of the left
-        //     factor as float4 (shared by the 16 lanes of that row) and the right factor's values
-        //     for its own columns (consecutive over the lanes).
+        //     [[Ta, 0], [Lba, Tb']]^{-1} = [[Ta, 0], [-Tb' Lba Ta, Tb']]: level 1 (16-row blocks) gives
+        //     T10 and T32, level 2 (32-row blocks) the lower-left 32x32 block.  The products run on
+        //     warp-level tensor-core MMAs (m16n8k8, tf32 operands rounded to nearest, fp32
+        //     accumulation); each product's result goes through the scratch tile to become the
+        //     next product's operand.
         {
-            float *sXs = sS;   // level 1: [2][16][16];  level 2: [32][32]
-            {
-                const int blk = tp >> 8, r = (tp >> 4) & 15, n = tp & 15;
-                const int j = 2 * blk, i = j + 1;
-                const float *arow = sA + (16 * i + r) * ld + 16 * j;
-                float acc = 0.f;
+            float *sXs = sS;   // level 1: [2][16][kXld];  level 2: [32][kYld]
+            constexpr int kXld = 20, kYld = 36;
+            const int g = lane >> 2, t4 = lane & 3;
+            // level 1: warp w < 2 forms T_ij for (i, j) = (2w + 1, 2w)
+            if (warp < 2) {
+                const int i = 2 * warp + 1, j = 2 * warp;
+                float *X = sXs + warp * 16 * kXld;
+                float acc[2][4];
+                // X = A_ij T_jj
+                mma_block_16x16<16>(acc, sA + 16 * i * ld + 16 * j, ld, sT + 16 * j * ld + 16 * j, ld, g, t4);
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
-                    const float *tk = sT + (16 * j + 4 * k4) * ld + 16 * j + n;
-                    acc = fmaf(a4.x, tk[0], acc);
-                    acc = fmaf(a4.y, tk[ld], acc);
-                    acc = fmaf(a4.z, tk[2 * ld], acc);
-                    acc = fmaf(a4.w, tk[3 * ld], acc);
+                for (int nt = 0; nt < 2; ++nt) {
+                    X[g * kXld + 8 * nt + 2 * t4] = acc[nt][0];
+                    X[g * kXld + 8 * nt + 2 * t4 + 1] = acc[nt][1];
+                    X[(g + 8) * kXld + 8 * nt + 2 * t4] = acc[nt][2];
+                    X[(g + 8) * kXld + 8 * nt + 2 * t4 + 1] = acc[nt][3];
                 }
-                sXs[blk * 256 + r * 16 + n] = acc;                       // X = A_ij T_jj
-                tc::named_sync(kBarRole, kRoleThreads);
-                const float *trow = sT + (16 * i + r) * ld + 16 * i;
-                const float *xk = sXs + blk * 256 + n;
-                acc = 0.f;
+                __syncwarp();
+                // T_ij = -T_ii X
+                mma_block_16x16<16>(acc, sT + 16 * i * ld + 16 * i, ld, X, kXld, g, t4);
+                float *Tij = sT + 16 * i * ld + 16 * j;
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 t4 = *reinterpret_cast<const float4 *>(trow + 4 * k4);
-                    acc = fmaf(t4.x, xk[(4 * k4) * 16], acc);
-                    acc = fmaf(t4.y, xk[(4 * k4 + 1) * 16], acc);
-                    acc = fmaf(t4.z, xk[(4 * k4 + 2) * 16], acc);
-                    acc = fmaf(t4.w, xk[(4 * k4 + 3) * 16], acc);
+                for (int nt = 0; nt < 2; ++nt) {
+                    *reinterpret_cast<float2 *>(Tij + g * ld + 8 * nt + 2 * t4) = make_float2(-acc[nt][0], -acc[nt][1]);
+                    *reinterpret_cast<float2 *>(Tij + (g + 8) * ld + 8 * nt + 2 * t4) =
+                        make_float2(-acc[nt][2], -acc[nt][3]);
                 }
-                sT[(16 * i + r) * ld + 16 * j + n] = -acc;               // T_ij = -T_ii X
             }
             tc::named_sync(kBarRole, kRoleThreads);
-            {
-                const int r = tp >> 4, n = 2 * (tp & 15);
-                const float *arow = sA + (32 + r) * ld;
-                float y0 = 0.f, y1 = 0.f;
+            // level 2: warp w < 8 forms the 16 x 8 tile (mt, nt) = (w / 4, w % 4) of Y = Lba Ta, then of
+            // Tba = -Tb' Y (Tb' is block lower triangular: rows 0-15 of it need only k < 16)
+            if (warp < 8) {
+                const int mt = warp >> 2, nt = warp & 3;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_tile_16x8<4>(acc, sA + (32 + 16 * mt) * ld, ld, sT + 8 * nt, ld, g, t4);
+                float *Y = sXs;
+                *reinterpret_cast<float2 *>(Y + (16 * mt + g) * kYld + 8 * nt + 2 * t4) = make_float2(acc[0], acc[1]);
+                *reinterpret_cast<float2 *>(Y + (16 * mt + g + 8) * kYld + 8 * nt + 2 * t4) =
+                    make_float2(acc[2], acc[3]);
+                tc::named_sync(kBarUt, 256);
 #pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
-                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 t2 = *reinterpret_cast<const float2 *>(sT + (4 * k4 + e) * ld + n);
-                        y0 = fmaf(av[e], t2.x, y0);
-                        y1 = fmaf(av[e], t2.y, y1);
-                    }
-                }
-                *reinterpret_cast<float2 *>(sXs + r * 32 + n) = make_float2(y0, y1);   // Y = Lba Ta
-                tc::named_sync(kBarRole, kRoleThreads);
-                const float *trow = sT + (32 + r) * ld + 32;
-                const int k4n = (r >> 4) * 4 + 4;   // Tb'[r][k] = 0 for k > r: whole 16-blocks skipped
-                y0 = 0.f;
-                y1 = 0.f;
-#pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    if (k4 >= k4n) break;
-                    const float4 t4 = *reinterpret_cast<const float4 *>(trow + 4 * k4);
-                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x2 = *reinterpret_cast<const float2 *>(sXs + (4 * k4 + e) * 32 + n);
-                        y0 = fmaf(tv[e], x2.x, y0);
-                        y1 = fmaf(tv[e], x2.y, y1);
-                    }
-                }
-                *reinterpret_cast<float2 *>(sT + (32 + r) * ld + n) = make_float2(-y0, -y1);   // Tba = -Tb' Y
+                for (int e = 0; e < 4; ++e) acc[e] = 0.f;
+                if (mt == 0)
+                    mma_tile_16x8<2>(acc, sT + 32 * ld + 32, ld, Y + 8 * nt, kYld, g, t4);
+                else
+                    mma_tile_16x8<4>(acc, sT + 48 * ld + 32, ld, Y + 8 * nt, kYld, g, t4);
+                float *Tba = sT + (32 + 16 * mt) * ld + 8 * nt;
+                *reinterpret_cast<float2 *>(Tba + g * ld + 2 * t4) = make_float2(-acc[0], -acc[1]);
+                *reinterpret_cast<float2 *>(Tba + (g + 8) * ld + 2 * t4) = make_float2(-acc[2], -acc[3]);
             }
             tc::named_sync(kBarRole, kRoleThreads);
         }
@@ -932,8 +957,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                 x[i] = -x[i];
                 ovf |= !(fabsf(x[i]) <= 65000.f);
             }
-            *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, cw / 8, kChunk)) = pack8_h(x);
-            *reinterpret_cast<uint4 *>(img + I::kNW + tile_chunk(r, cw / 8 + 1, kChunk)) = pack8_h(x + 8);
+            *reinterpret_cast<uint4 *>(img + I::kA1 + a1_nw(r, cw / 8)) = pack8_h(x);
+            *reinterpret_cast<uint4 *>(img + I::kA1 + a1_nw(r, cw / 8 + 1)) = pack8_h(x + 8);
             const int j = sp * 32 + lane;
             tc::tmem_ld16(tmem + tl + kTmUT + q4 * 16, x);
             tc::tmem_ld_wait();
@@ -1004,12 +1029,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             uint8_t *slot = sm + (t % SM::kSlots) * SM::kSlotBytes;
             uint64_t *fb = &bars.full[t % SM::kSlots];
             tc::mbar_arrive_expect_tx(fb, I::kBytes);
-            tc::bulk_load(slot + SM::kA1, src + I::kNW, 8192, fb);
-            tc::bulk_load(slot + SM::kA1 + 16384, src + I::kNW + 8192, 8192, fb);
-            tc::bulk_load(slot + SM::kA1 + 8192, src + I::kQt, 8192, fb);
-            tc::bulk_load(slot + SM::kA1 + 24576, src + I::kQt + 8192, 8192, fb);
-            tc::bulk_load(slot + SM::kUT, src + I::kUT, kChunk * DV * 2, fb);
-            tc::bulk_load(slot + SM::kKd, src + I::kKd, SM::kTailBytes, fb);
+            tc::bulk_load(slot, src, I::kBytes, fb);   // the image has the slot's layout: one copy
             pend[t % SM::kSlots] = t;
             return true;
         };
@@ -1071,7 +1091,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     const int L = pi.len(c);
                     const bool full = L == kChunk;
                     // staging: the slot's A1 area, dead since MMA1 of this chunk (before [. ; P] U~)
-                    TO *stage = reinterpret_cast<TO *>(sm + s3 * SM::kSlotBytes + SM::kA1);
+                    TO *stage = reinterpret_cast<TO *>(sm + s3 * SM::kSlotBytes + I::kA1);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
                         float o[32];
@@ -1220,19 +1240,26 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
         for (int i = 0; i < 32; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
         tc::tc_fence_before();
         bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
+        bool have_image = false;   // the previous chunk's last barrier already covered this chunk's image
         for (int c = 0; c < pi.nchunks; ++c, ++t) {
             const int s = t % SM::kSlots, b = t & 1;
             const int64_t tok0 = pi.tok0(c);
             const int L = pi.len(c);
             const uint8_t *slot = sm + s * SM::kSlotBytes;
             const uint32_t sslot = sbase + s * SM::kSlotBytes;
-            if (!role_wait(&bars.full[s], (t / SM::kSlots) & 1, leader, kBarRole, kRoleThreads, abort_flag)) {
+            if (!have_image &&
+                !role_wait(&bars.full[s], (t / SM::kSlots) & 1, leader, kBarRole, kRoleThreads, abort_flag)) {
+                stop = true;
+                break;
+            }
+            have_image = false;
+            if (*abort_flag) {
                 stop = true;
                 break;
             }
             // chunk t is out of the ring (the copy has completed): its slot may take a later image
             if (leader) tc::st_relaxed_gpu(sched.consumed + kc, t + 1);
-            const bool flagged = *reinterpret_cast<const volatile int *>(slot + SM::kFlag) != 0;
+            const bool flagged = *reinterpret_cast<const volatile int *>(slot + I::kFlag) != 0;
             if (leader) {
                 // the output warps have read D1^T[b] of chunk t - 2
                 bool ok = t < 2 || tc::mbar_wait(&bars.d1_free[b], ((t >> 1) - 1) & 1, abort_flag);
@@ -1243,7 +1270,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
 #pragma unroll
                     for (int kk = 0; kk < kDK / 16; ++kk)
                         tc::mma_f16_ta(tmem + kTmD1 + b * 128, tmem + kTmS + kk * 8,
-                                       desc_kmajor(sslot + SM::kA1, 128, kk), id1, kk > 0);
+                                       desc_kmajor(sslot + I::kA1, 128, kk), id1, kk > 0);
                     tc::mma_commit(&bars.mma1);
                 }
                 if (flagged) {
@@ -1255,7 +1282,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 // while MMA1 runs: D2^T = S^T Diag(gamma) in fp32, which MMA2 then accumulates onto
                 // (D2^T was last read by the previous chunk's state update)
                 {
-                    const float4 *gam4 = reinterpret_cast<const float4 *>(slot + SM::kGam) + c0 / 4;
+                    const float4 *gam4 = reinterpret_cast<const float4 *>(slot + I::kGam) + c0 / 4;
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         uint32_t u[16];
@@ -1289,7 +1316,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
                             float u8[8];
-                            unpack8_h(*reinterpret_cast<const uint4 *>(slot + SM::kUT + tile_chunk(j, 2 * qd + h2, DV)),
+                            unpack8_h(*reinterpret_cast<const uint4 *>(slot + I::kUT + tile_chunk(j, 2 * qd + h2, DV)),
                                       u8);
 #pragma unroll
                             for (int i = 0; i < 8; ++i) x[8 * h2 + i] += u8[i];
@@ -1306,7 +1333,9 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     tc::tmem_st_wait();
                 }
                 tc::tc_fence_before();
-                const bool bad = tc::named_sync_or(kBarRole, kRoleThreads, mybad);
+                if (mybad) *reinterpret_cast<volatile int *>(&bars.ovf_ut) = t + 1;
+                tc::named_sync(kBarRole, kRoleThreads);
+                const bool bad = *reinterpret_cast<volatile int *>(&bars.ovf_ut) == t + 1;
                 if (*reinterpret_cast<volatile int *>(&bars.fail1)) {
                     stop = true;
                     break;
@@ -1318,13 +1347,13 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     constexpr uint32_t id3 = tc::make_idesc(128, kChunk, tc::kF16, false, false);
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk)
-                        tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + SM::kKd, kChunk, kk),
+                        tc::mma_f16_ta(tmem + kTmD2, tmem + kTmUt + kk * 8, desc_mnmajor(sslot + I::kKd, kChunk, kk),
                                        id2, true);
                     tc::mma_commit(&bars.mma2);
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk)
                         tc::mma_f16_ta(tmem + kTmD1 + b * 128 + 64, tmem + kTmUt + kk * 8,
-                                       desc_kmajor(sslot + SM::kP, kChunk, kk), id3, true);
+                                       desc_kmajor(sslot + I::kP, kChunk, kk), id3, true);
                     tc::mma_commit(&bars.mma3[b]);
                     bars.outmode[b] = bad ? 1 : 2;   // MMAs issued; O^T is the output unless evaluated exactly
                     tc::mbar_arrive(&bars.outq[b]);
@@ -1338,7 +1367,17 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     tc::tmem_ld_wait();
                     const bool big = write_state_operand();
                     tc::tc_fence_before();
-                    force_exact = tc::named_sync_or(kBarRole, kRoleThreads, big);
+                    if (big) *reinterpret_cast<volatile int *>(&bars.ovf_st) = t + 1;
+                    // the next chunk's image (two chunks ahead, normally landed long ago): the leader waits
+                    // for it here, so that this barrier serves both
+                    if (c + 1 < pi.nchunks) {
+                        if (leader) tc::mbar_wait(&bars.full[(t + 1) % SM::kSlots], ((t + 1) / SM::kSlots) & 1,
+                                                  abort_flag);
+                        have_image = true;
+                    }
+                    tc::named_sync(kBarRole, kRoleThreads);
+                    tc::tc_fence_after();
+                    force_exact = *reinterpret_cast<volatile int *>(&bars.ovf_st) == t + 1;
                     if (*reinterpret_cast<volatile int *>(&bars.fail2)) {
                         stop = true;
                         break;
@@ -1408,6 +1447,8 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
         abort_flag = 0;
         bars.fail1 = 0;
         bars.fail2 = 0;
+        bars.ovf_ut = 0;
+        bars.ovf_st = 0;
     }
     const uint32_t ncols = is_chain ? kTmChainCols : kTmPrepCols;
     if (warp == 0) {
