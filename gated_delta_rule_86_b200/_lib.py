@@ -14,7 +14,7 @@ KDA_F32, KDA_BF16 = 0, 1
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd_static_ws", "kda_recurrent_fwd",
             "kda_decode_step", "gdn_chunk_fwd", "gdn_recurrent_fwd", "gdn_decode_step", "kda_chunk_fwd_fused",
             "kda_decode_step_fused", "kda_status_string", "kda_get_last_device_error", "kda_version",
-            "kda_testing_set_chunk_fault")
+            "kda_testing_set_chunk_fault", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size")
 
 _lib = None
 
@@ -61,6 +61,12 @@ def load() -> ctypes.CDLL:
     lib.kda_version.restype = ctypes.c_char_p
     lib.kda_testing_set_chunk_fault.argtypes = [i32, ctypes.c_uint32]
     lib.kda_testing_set_chunk_fault.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = prefill_args + [i32, ctypes.c_int, vp, ctypes.c_int, f32p] + [f32p] * 6 + \
+        [vp, ctypes.c_size_t, vp]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
+    lib.kda_chunk_bwd_workspace_size.argtypes = [i32, i32, ctypes.c_int64, i32, i32, i32,
+                                                 ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_chunk_bwd_workspace_size.restype = ctypes.c_int
     _lib = lib
     return lib
 

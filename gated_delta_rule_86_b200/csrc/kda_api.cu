@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/kda.h"
+#include "kda_backward.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
@@ -341,6 +342,61 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v, const vo
                            float *state, void *out, int32_t B, int32_t H, int32_t d_k, int32_t d_v, kda_dtype dtype,
                            kda_dtype out_dtype, void *stream) {
     return decode_impl<kda::kGateHead>(q, k, v, log_g, beta, state, out, B, H, d_k, d_v, dtype, out_dtype, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+kda_status kda_chunk_bwd_workspace_size(int32_t N, int32_t H, int64_t total_tokens, int32_t d_k, int32_t d_v,
+                                        int32_t chunk, size_t *bytes) {
+    if (!bytes || N < 1 || H < 1 || total_tokens < 0 || chunk < 1) return KDA_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (!head_ok(d_k) || !head_ok(d_v) || chunk > 256) return KDA_ERR_UNSUPPORTED;
+    *bytes = kda::bwd_workspace_bytes(N, H, total_tokens, d_k, d_v, chunk);
+    return KDA_OK;
+}
+
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, const void *beta,
+                         const float *init_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype dtype, const void *d_out,
+                         kda_dtype d_out_dtype, const float *d_final_state, float *dq, float *dk, float *dv,
+                         float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    // the forward arguments are checked as for the prefill (d_out plays the part of `out`)
+    kda_status s = check_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H, d_k, d_v, dtype,
+                                 d_out_dtype, d_out, d_final_state, kda::kGateChannel);
+    if (s != KDA_OK) return s;
+    if (T > 0 && (!dq || !dk || !dv || !dlog_alpha || !dbeta)) return KDA_ERR_INVALID_ARG;
+    const void *outs[] = {dq, dk, dv, dlog_alpha, dbeta, d_init_state};
+    for (const void *p : outs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (chunk > 256) return KDA_ERR_UNSUPPORTED;
+    const int N = cu_seqlens ? num_seqs : B;
+    const int64_t total = cu_seqlens ? (int64_t)T : (int64_t)B * T;
+    const size_t need = kda::bwd_workspace_bytes(N, H, total, d_k, d_v, chunk);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dtype == KDA_F32)
+        e = d_out_dtype == KDA_F32
+                ? kda::launch_bwd<float, float>(d_k, d_v, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B,
+                                                T, H, chunk, d_out, d_final_state, dq, dk, dv, dlog_alpha, dbeta,
+                                                d_init_state, workspace, st)
+                : kda::launch_bwd<float, __nv_bfloat16>(d_k, d_v, q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                                        num_seqs, B, T, H, chunk, d_out, d_final_state, dq, dk, dv,
+                                                        dlog_alpha, dbeta, d_init_state, workspace, st);
+    else
+        e = d_out_dtype == KDA_F32
+                ? kda::launch_bwd<__nv_bfloat16, float>(d_k, d_v, q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                                        num_seqs, B, T, H, chunk, d_out, d_final_state, dq, dk, dv,
+                                                        dlog_alpha, dbeta, d_init_state, workspace, st)
+                : kda::launch_bwd<__nv_bfloat16, __nv_bfloat16>(d_k, d_v, q, k, v, log_alpha, beta, init_state,
+                                                                cu_seqlens, num_seqs, B, T, H, chunk, d_out,
+                                                                d_final_state, dq, dk, dv, dlog_alpha, dbeta,
+                                                                d_init_state, workspace, st);
+    return from_cuda(e);
 }
 
 }  // extern "C"

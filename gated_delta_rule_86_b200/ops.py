@@ -213,6 +213,53 @@ def kda_decode_step_fused(q_raw, k_raw, v, g_raw, b_raw, state, out=None, out_dt
     return _decode("kda_decode_step_fused", q_raw, k_raw, v, g_raw, b_raw, state, out, out_dtype)
 
 
+def kda_chunk_bwd(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None, cu_seqlens=None,
+                  chunk_size=64):
+    """Gradient of :func:`kda_chunk_fwd` (reverse mode through the recurrence, fp32).
+
+    Takes the forward's inputs and ``d_out`` = dLoss/dout ([B, T, H, d_v], fp32 or bf16) and,
+    optionally, ``d_final_state`` = dLoss/dfinal_state (fp32 [N, H, d_k, d_v]).  Returns
+    ``(dq, dk, dv, dlog_alpha, dbeta, d_initial_state)`` in fp32 with the shapes of q, k, v,
+    log_alpha, beta and the initial state.  ``chunk_size`` is the checkpoint interval.
+    """
+    lib = _lib.load()
+    on_host = not q.is_cuda
+    _, (q, k, v, la, beta, s0, cu), (B, T, H, dk, dv, N) = _prefill_prepare(
+        q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    dt = _io_dtype(q, k, v, la, beta)
+    d_out = _to_device(d_out, q.device).contiguous()
+    if d_out.shape != (B, T, H, dv):
+        raise ValueError("d_out must have the shape of the output")
+    dodt = _out_dtype(d_out.dtype)
+    dfin = None
+    if d_final_state is not None:
+        dfin = _to_device(d_final_state, q.device).to(torch.float32).contiguous()
+        if dfin.shape != (N, H, dk, dv):
+            raise ValueError(f"d_final_state must be [{N}, {H}, {dk}, {dv}]")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = [torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H, dv), **f32),
+         torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H), **f32), torch.empty((N, H, dk, dv), **f32)]
+    total = T if cu is not None else B * T
+    ws_bytes = ctypes.c_size_t(0)
+    _lib.check(lib.kda_chunk_bwd_workspace_size(N, H, total, dk, dv, chunk_size, ctypes.byref(ws_bytes)),
+               "kda_chunk_bwd_workspace_size")
+    ws = torch.empty(max(ws_bytes.value, 16), dtype=torch.uint8, device=q.device)
+    status = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(beta), _ptr(s0), _ptr(cu),
+                               ctypes.c_int32(N if cu is not None else 0), B, T, H, dk, dv,
+                               ctypes.c_int32(chunk_size), dt, _ptr(d_out), dodt, _ptr(dfin),
+                               *(_ptr(x) for x in g), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle())
+    _lib.check(status, "kda_chunk_bwd")
+    if on_host:
+        out = []
+        for x in g:
+            hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+            hx.copy_(x, non_blocking=True)
+            out.append(hx)
+        torch.cuda.current_stream().synchronize()
+        return tuple(out)
+    return tuple(g)
+
+
 def device_error() -> int:
     """Sync the current stream and return-and-clear the device error word (KDA_OK or KDA_ERR_TIMEOUT)."""
     return _lib.load().kda_get_last_device_error(_stream_handle())

@@ -18,7 +18,8 @@
  * kda_chunk_fwd_static_ws, and the token-by-token kda_recurrent_fwd) and decode
  * (kda_decode_step); the same from the raw projections (kda_chunk_fwd_fused,
  * kda_decode_step_fused); Gated DeltaNet and DeltaNet (gdn_chunk_fwd,
- * gdn_recurrent_fwd, gdn_decode_step); status helpers.
+ * gdn_recurrent_fwd, gdn_decode_step); the gradient of the prefill
+ * (kda_chunk_bwd); status helpers.
  *
  * Conventions for every call
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -250,6 +251,54 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
                                    int32_t T, int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
                                    kda_dtype dtype, kda_dtype out_dtype, void *out,
                                    float *final_state, void *stream);
+
+/*
+ * kda_chunk_bwd -- gradient of kda_chunk_fwd with respect to every input
+ * (reverse mode through the recurrence of "Core Module Design", Stage 3, of
+ * the page named above; the pages train the layer -- the implementation
+ * checklist there asks for FP32 intermediates and gradient clipping, and
+ * section 3 of "Linear Attention KDA Gating in a 3:1 Hybrid Architecture"
+ * asks for gradient checks -- but print no backward pass).  With w = S'^T k,
+ * S' = Diag(alpha) S_prev and u = beta (v - w), one reverse token step is
+ *     dS += q do^T;  dq = S do;  du = dS^T k;  dk = dS u - beta S' du;
+ *     dbeta = du . (v - w);  dv = beta du;  dS' = dS - beta k du^T;
+ *     dlog_alpha = rowsum(dS' * S');  dS_prev = Diag(alpha) dS'.
+ * All arithmetic is fp32 on CUDA cores; one CTA per (sequence, head) keeps
+ * the state and its gradient in registers and reduces over d_k and d_v in a
+ * fixed order (results are reproducible run to run).
+ *
+ *   q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H,
+ *   d_k, d_v, dtype : as for kda_chunk_fwd (the forward's inputs).
+ *   chunk           : states are checkpointed every `chunk` tokens and each
+ *                     chunk's per-token states recomputed from its checkpoint
+ *                     (1 <= chunk <= 256; it changes no result).
+ *   d_out           : [B, T, H, d_v] d_out_dtype, dLoss/dout.
+ *   d_final_state   : [N, H, d_k, d_v] fp32 dLoss/dfinal_state, or NULL (zero).
+ *   dq, dk, dlog_alpha : [B, T, H, d_k] fp32 (written).
+ *   dv              : [B, T, H, d_v] fp32 (written).
+ *   dbeta           : [B, T, H] fp32 (written).
+ *   d_init_state    : [N, H, d_k, d_v] fp32 dLoss/dinit_state, or NULL to skip.
+ *   workspace       : at least kda_chunk_bwd_workspace_size bytes (16-byte
+ *                     aligned, owned by the caller): the checkpoints and one
+ *                     chunk of per-token states for every (sequence, head).
+ * Supported: d_k, d_v in {64, 128}; either dtype and d_out dtype.
+ */
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                         const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                         int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t d_k,
+                         int32_t d_v, int32_t chunk, kda_dtype dtype, const void *d_out,
+                         kda_dtype d_out_dtype, const float *d_final_state, float *dq, float *dk,
+                         float *dv, float *dlog_alpha, float *dbeta, float *d_init_state,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Workspace of kda_chunk_bwd, in bytes, for N sequences of H heads holding
+ * total_tokens tokens in all (B * T, or the packed length with cu_seqlens).
+ * Pure host computation; KDA_ERR_UNSUPPORTED for the shapes kda_chunk_bwd
+ * rejects with that status.
+ */
+kda_status kda_chunk_bwd_workspace_size(int32_t N, int32_t H, int64_t total_tokens, int32_t d_k,
+                                        int32_t d_v, int32_t chunk, size_t *bytes);
 
 /* Human-readable name of a status (static string, never NULL). */
 const char *kda_status_string(kda_status s);

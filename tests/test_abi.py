@@ -181,3 +181,29 @@ def test_no_cpu_fallback_without_gpu():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1", "--warmup", "3",
                         "--no-cpu-baseline"], capture_output=True, text=True, cwd=ROOT, timeout=300)
     assert r.returncode != 0 and not any(ln.startswith("{") for ln in r.stdout.splitlines())
+
+
+def test_backward_argument_checks(lib):
+    """kda_chunk_bwd validates on the host before launching anything."""
+    n = ctypes.c_size_t(7)
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 64, ctypes.byref(n)) == _lib.KDA_OK
+    # checkpoints (total/C + N + 1 per head) and one chunk of per-token states per (sequence, head)
+    kv = 128 * 128 * 4
+    assert n.value == 4 * (1000 // 64 + 2 + 1) * kv + 2 * 4 * 64 * kv
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 96, 128, 64, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 0, ctypes.byref(n)) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 512, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+    F = ctypes.c_void_p(4096)
+    bwd = lib.kda_chunk_bwd
+
+    def call(dk=128, dq=F, ws=F, ws_bytes=1 << 40, chunk=64, T=16):
+        return bwd(F, F, F, F, F, None, None, 0, 1, T, 2, dk, 128, chunk, _lib.KDA_BF16, F, _lib.KDA_F32, None,
+                   dq, F, F, F, F, None, ws, ctypes.c_size_t(ws_bytes), None)
+
+    assert call(dk=96) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(dq=None) == _lib.KDA_ERR_INVALID_ARG
+    assert call(ws=None) == _lib.KDA_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == _lib.KDA_ERR_INVALID_ARG
+    assert call(chunk=0) == _lib.KDA_ERR_INVALID_ARG
+    assert call(chunk=300) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(dq=ctypes.c_void_p(4100)) == _lib.KDA_ERR_INVALID_ARG   # misaligned
