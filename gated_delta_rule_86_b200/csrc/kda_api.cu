@@ -184,18 +184,19 @@ kda_status chunk_impl(int gate, bool static_ws, const void *q, const void *k, co
                                  out_dtype, out, final_state, gate);
     if (s != KDA_OK) return s;
     if (chunk < 1) return KDA_ERR_INVALID_ARG;
-    if (chunk != 64) return KDA_ERR_UNSUPPORTED;
+    // chunks of up to 64 tokens (the tensor-core kernel's tile height); 128 would need a larger image
+    // than the chain's shared memory holds three of
+    if (chunk > kda::kChunk) return KDA_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (static_ws || gate == kda::kRawInputs) {
         // the raw-projection form runs on the tensor-core path only
-        if (dtype != KDA_BF16 || d_k != 128) return KDA_ERR_UNSUPPORTED;
+        if (dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
     } else if (dtype == KDA_F32) {
         // fp32 I/O asks for fp32 accuracy, which bf16 tensor-core operands
         // cannot give: evaluate on CUDA cores with the fp32 state.
         return from_cuda(dispatch_recurrent(gate, dtype, out_dtype, q, k, v, la, beta, init_state, cu_seqlens,
                                             num_seqs, B, T, H, d_k, d_v, out, final_state, st));
     }
-    if (d_k != 128) return KDA_ERR_UNSUPPORTED;
     if ((int64_t)B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;   // 32-bit token coordinates
     const int64_t pairs = (int64_t)(cu_seqlens ? num_seqs : B) * H;
     if (static_ws) {
@@ -212,10 +213,11 @@ kda_status chunk_impl(int gate, bool static_ws, const void *q, const void *k, co
     }
     if (out_dtype == KDA_F32)
         return from_cuda(kda::launch_chunk_tc<float>(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T, H,
-                                                     d_v, out, final_state, workspace, workspace_bytes, st, gate));
+                                                     d_k, d_v, chunk, out, final_state, workspace, workspace_bytes,
+                                                     st, gate));
     return from_cuda(kda::launch_chunk_tc<__nv_bfloat16>(q, k, v, la, beta, init_state, cu_seqlens, num_seqs, B, T,
-                                                         H, d_v, out, final_state, workspace, workspace_bytes, st,
-                                                         gate));
+                                                         H, d_k, d_v, chunk, out, final_state, workspace,
+                                                         workspace_bytes, st, gate));
 }
 
 template <int GK>
@@ -274,8 +276,6 @@ kda_status kda_chunk_fwd_workspace_size(int32_t N, int32_t H, int32_t d_k, int32
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     *bytes = 0;
     if (!head_ok(d_k) || !head_ok(d_v)) return KDA_ERR_UNSUPPORTED;
-    // the bf16 tensor-core path takes d_k == 128 only (kda_chunk_fwd rejects the rest)
-    if (dtype == KDA_BF16 && d_k != 128) return KDA_ERR_UNSUPPORTED;
     if (dtype == KDA_BF16) *bytes = kda::chunk_tc_workspace_bytes((int64_t)N * H, d_v);
     return KDA_OK;
 }

@@ -283,6 +283,10 @@ __device__ __forceinline__ void drain_mma(uint64_t *bar, uint32_t parity) {
 // its image into slot t % ring of chain k's ring in the workspace.
 struct ChunkSched {
     int npairs, nchain, nprod, ring, H, T;
+    int C;                  // chunk length (1 <= C <= kChunk; a chunk of C < kChunk tokens fills the first C
+                            // rows of the 64-row tiles, the rest are zero, as for the short last chunk)
+    int dk;                 // key width of the inputs, 64 or kDK: with 64 the key channels 64-127 are zero
+                            // (their state rows stay zero and never reach an output)
     const int32_t *cu;      // cu_seqlens, or null for [B, T] inputs
     const int32_t *order;   // sequences longest-first (packed inputs), or null for the identity
     int *ready;             // [nchain][ring]: 1 + number of the chunk whose image the slot holds
@@ -294,13 +298,13 @@ struct ChunkSched {
 
 // One (sequence, head) pair.
 struct PairInfo {
-    int n, h, nchunks;
+    int n, h, nchunks, C;
     int64_t t0, t1;
-    // chunk c: first token and valid length
-    __device__ __forceinline__ int64_t tok0(int c) const { return t0 + (int64_t)c * kChunk; }
+    // chunk c (C tokens, the last one shorter): first token and valid length (at most C <= kChunk)
+    __device__ __forceinline__ int64_t tok0(int c) const { return t0 + (int64_t)c * C; }
     __device__ __forceinline__ int len(int c) const {
         const int64_t r = t1 - tok0(c);
-        return static_cast<int>(r < kChunk ? r : kChunk);
+        return static_cast<int>(r < C ? r : C);
     }
 };
 __device__ __forceinline__ PairInfo pair_info(const ChunkSched &s, int p) {
@@ -316,7 +320,8 @@ __device__ __forceinline__ PairInfo pair_info(const ChunkSched &s, int p) {
         r.t0 = (int64_t)rank * s.T;
         r.t1 = r.t0 + s.T;
     }
-    r.nchunks = static_cast<int>((r.t1 - r.t0 + kChunk - 1) / kChunk);
+    r.C = s.C;
+    r.nchunks = static_cast<int>((r.t1 - r.t0 + s.C - 1) / s.C);
     return r;
 }
 // Chunk t of chain k: its pair and chunk index there; false if the chain has fewer chunks.
@@ -512,7 +517,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
             const int L = have ? it.pi.len(it.c) : -1, h = it.pi.h;
             if (lane == 0) {
                 // a per-head gate comes as 64 scalars (below) instead of a log_alpha tile
-                constexpr uint32_t kTileBytes = GK != kGateHead ? SM::kRawBytes : SM::kRawBytes - SM::kTile;
+                const uint32_t kTileBytes = (GK != kGateHead ? 3u : 2u) * kChunk * sched.dk * 2 + kChunk * DV * 2;
                 tc::mbar_arrive_expect_tx(&bars.raw_full, have ? kTileBytes : 0);
                 if (have) {
                     const int t = static_cast<int>(tok0);
@@ -547,6 +552,7 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
     }
 
     // ---- compute warps 0-15 ----
+    const int dkin = sched.dk;   // key channels present in the input rows (the rest read as zero)
     const int tp = tid;
     const bool leader = tp == 0;
     const int cg = tp & 15, tg = tp >> 4;   // channels [8cg, 8cg+8), tokens 2tg, 2tg + 1
@@ -595,7 +601,8 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
                 const int r = tg * 2 + rr;
                 float g8[8];
                 if constexpr (GK != kGateHead) {
-                    const uint4 raw = r < L ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * 256 + cg * 16)
+                    const uint4 raw = (r < L && cg * 8 < dkin)
+                                          ? *reinterpret_cast<const uint4 *>(sm + SM::kRawG + r * dkin * 2 + cg * 16)
                                             : make_uint4(0, 0, 0, 0);
                     unpack8(raw, g8);
                     if constexpr (GK == kRawInputs) {   // the gate's pre-activation: log_alpha = logsigmoid
@@ -674,8 +681,9 @@ __device__ __forceinline__ void prep_role(const ChunkCtx &cx, ChunkBars &bars, c
         for (int rr = 0; rr < 2; ++rr) {
             const int r = tg * 2 + rr;
             const bool in = r < L;
-            rk[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawK + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
-            rq[rr] = in ? *reinterpret_cast<const uint4 *>(sm + SM::kRawQ + r * 256 + cg * 16) : make_uint4(0, 0, 0, 0);
+            const bool kin = in && cg * 8 < dkin;
+            rk[rr] = kin ? *reinterpret_cast<const uint4 *>(sm + SM::kRawK + r * dkin * 2 + cg * 16) : make_uint4(0, 0, 0, 0);
+            rq[rr] = kin ? *reinterpret_cast<const uint4 *>(sm + SM::kRawQ + r * dkin * 2 + cg * 16) : make_uint4(0, 0, 0, 0);
             rv[rr] = (in && cg * 8 < DV) ? *reinterpret_cast<const uint4 *>(sm + SM::kRawV + r * DV * 2 + cg * 16)
                                          : make_uint4(0, 0, 0, 0);
         }
@@ -1153,6 +1161,8 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     const int j = sp * 32 + lane;            // value column (TMEM lane)
     const bool jv = j < DV;
     const int c0 = qd * 32;                  // key channels [c0, c0 + 32)
+    const int dkin = sched.dk;               // key channels present in the inputs
+    const bool kin = c0 < dkin;              // this thread's channels are (not padding)
     const uint32_t tl = tc::tmem_lane_base(warp);
     float *redPk = reinterpret_cast<float *>(sm + SM::kRedPk);
     float *redPq = reinterpret_cast<float *>(sm + SM::kRedPq);
@@ -1180,16 +1190,16 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const int64_t trow = (tok0 + r) * H + h;
             // a per-head gate: the same log-decay for every channel (none when log_g is null)
             constexpr int gstride = GK != kGateHead ? 1 : 0;
-            const __nv_bfloat16 *gr = log_alpha + (GK != kGateHead ? trow * kDK + c0 : trow),
-                                *kr = k + trow * kDK + c0, *qr = q + trow * kDK + c0;
+            const __nv_bfloat16 *gr = log_alpha + (GK != kGateHead ? trow * dkin + c0 : trow),
+                                *kr = k + trow * dkin + c0, *qr = q + trow * dkin + c0;
             const bool has_gate = GK != kGateHead || log_alpha != nullptr;
             // raw inputs: the 1 / L2 norms of the whole q and k rows
             float nk = 1.f, nq = 1.f;
             if constexpr (GK == kRawInputs) {
-                const uint4 *k8 = reinterpret_cast<const uint4 *>(k + trow * kDK);
-                const uint4 *q8 = reinterpret_cast<const uint4 *>(q + trow * kDK);
+                const uint4 *k8 = reinterpret_cast<const uint4 *>(k + trow * dkin);
+                const uint4 *q8 = reinterpret_cast<const uint4 *>(q + trow * dkin);
                 float sk = 0.f, sq = 0.f;
-                for (int c8 = 0; c8 < kDK / 8; ++c8) {
+                for (int c8 = 0; c8 < dkin / 8; ++c8) {
                     float f[8];
                     unpack8(k8[c8], f);
 #pragma unroll
@@ -1204,10 +1214,11 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             float pk = 0.f, pq = 0.f, kq = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                float lg = __bfloat162float(gr[i * gstride]);
-                if constexpr (GK == kRawInputs) lg = log_sigmoid(lg);
-                const float a = has_gate ? expf(lg) : 1.f, kk = __bfloat162float(kr[i]) * nk,
-                            qq = __bfloat162float(qr[i]) * nq;
+                // key channels past the input's width: no decay, zero key and query
+                float lg = kin ? __bfloat162float(gr[i * gstride]) : 0.f;
+                if constexpr (GK == kRawInputs) lg = kin ? log_sigmoid(lg) : 0.f;
+                const float a = has_gate ? expf(lg) : 1.f, kk = kin ? __bfloat162float(kr[i]) * nk : 0.f,
+                            qq = kin ? __bfloat162float(qr[i]) * nq : 0.f;
                 S[i] *= a;
                 pk = fmaf(S[i], kk, pk);
                 pq = fmaf(S[i], qq, pq);
@@ -1222,8 +1233,10 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const float spq = (redPq[j] + redPq[128 + j]) + (redPq[256 + j] + redPq[384 + j]);
             const float u = jv ? beta_of<GK>(beta, trow) * (__bfloat162float(v[trow * DV + j]) - spk) : 0.f;
             if (qd == 0 && jv) out[trow * DV + j] = from_f32<TO>(fmaf(u, skq, spq));
+            if (kin) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] = fmaf(__bfloat162float(kr[i]) * nk, u, S[i]);
+                for (int i = 0; i < 32; ++i) S[i] = fmaf(__bfloat162float(kr[i]) * nk, u, S[i]);
+            }
             tc::named_sync(kBarRole, kRoleThreads);
         }
         return write_state_operand();
@@ -1235,9 +1248,9 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
     for (int pr = kc; pr < sched.npairs && !stop; pr += sched.nchain) {
         const PairInfo pi = pair_info(sched, pr);
         h = pi.h;
-        const size_t state_base = ((size_t)pi.n * H + h) * kDK * DV + (size_t)c0 * DV + j;
+        const size_t state_base = ((size_t)pi.n * H + h) * dkin * DV + (size_t)c0 * DV + j;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] = (init_state && jv) ? init_state[state_base + (size_t)i * DV] : 0.f;
+        for (int i = 0; i < 32; ++i) S[i] = (init_state && jv && kin) ? init_state[state_base + (size_t)i * DV] : 0.f;
         tc::tc_fence_before();
         bool force_exact = tc::named_sync_or(kBarRole, kRoleThreads, write_state_operand());
         bool have_image = false;   // the previous chunk's last barrier already covered this chunk's image
@@ -1396,7 +1409,7 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             }
             if (leader) tc::mbar_arrive(&bars.slot_free[s]);
         }
-        if (!stop && final_state && *abort_flag == 0 && jv) {
+        if (!stop && final_state && *abort_flag == 0 && jv && kin) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) final_state[state_base + (size_t)i * DV] = S[i];
         }
@@ -1581,8 +1594,9 @@ inline ChunkFault &chunk_fault() {
 template <int DV, typename TO, int GK>
 cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, const void *la, const void *beta,
                                const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H,
-                               void *out, float *final_state, void *workspace, size_t ws_bytes,
+                               int DKIN, int C, void *out, float *final_state, void *workspace, size_t ws_bytes,
                                cudaStream_t stream) {
+    if (C < 1 || C > kChunk || (DKIN != 64 && DKIN != kDK)) return cudaErrorInvalidValue;
     auto kern = kda_chunk_tc_kernel<DV, TO, GK>;
     const int smem = chunk_smem_bytes<DV>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1603,9 +1617,9 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
     memset(&maps, 0, sizeof(maps));
     const int64_t tokens = (int64_t)B * T;
     if (tokens > 0) {   // with no tokens no chunk is loaded and the maps stay unused
-        if ((GK != kGateHead && !encode_row_map(&maps.g, la, kDK, H, tokens)) ||
-            !encode_row_map(&maps.k, k, kDK, H, tokens) ||
-            !encode_row_map(&maps.q, q, kDK, H, tokens) || !encode_row_map(&maps.v, v, DV, H, tokens) ||
+        if ((GK != kGateHead && !encode_row_map(&maps.g, la, DKIN, H, tokens)) ||
+            !encode_row_map(&maps.k, k, DKIN, H, tokens) ||
+            !encode_row_map(&maps.q, q, DKIN, H, tokens) || !encode_row_map(&maps.v, v, DV, H, tokens) ||
             !encode_row_map(&maps.o, out, DV, H, tokens, 64,
                             sizeof(TO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                             static_cast<int>(sizeof(TO))))
@@ -1619,6 +1633,8 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
     sched.ring = static_cast<int>(ring);
     sched.H = H;
     sched.T = T;
+    sched.C = C;
+    sched.dk = DKIN;
     sched.cu = cu;
     const bool sorted = cu && num_seqs <= kLongestFirstMaxSeqs;
     sched.order = sorted ? reinterpret_cast<const int32_t *>(ws) : nullptr;
@@ -1655,12 +1671,12 @@ cudaError_t launch_chunk_tc_dv(const void *q, const void *k, const void *v, cons
 // (kGateHead), or the gate's pre-activation [tokens][H][d_k] (kRawInputs, with raw q, k, beta).
 template <typename TO>
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const void *la, const void *beta,
-                            const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DV,
-                            void *out, float *final_state, void *workspace, size_t ws_bytes, cudaStream_t stream,
-                            int gate = kGateChannel) {
+                            const float *init_state, const int32_t *cu, int num_seqs, int B, int T, int H, int DKIN,
+                            int DV, int C, void *out, float *final_state, void *workspace, size_t ws_bytes,
+                            cudaStream_t stream, int gate = kGateChannel) {
 #define KDA_CHUNK_TC_CASE(DVV, GKK)                                                                          \
     if (DV == DVV && gate == GKK)                                                                            \
-        return launch_chunk_tc_dv<DVV, TO, GKK>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, out,   \
+        return launch_chunk_tc_dv<DVV, TO, GKK>(q, k, v, la, beta, init_state, cu, num_seqs, B, T, H, DKIN, C, out, \
                                                 final_state, workspace, ws_bytes, stream);
     KDA_CHUNK_TC_CASE(64, kGateChannel)
     KDA_CHUNK_TC_CASE(128, kGateChannel)

@@ -88,7 +88,12 @@ typedef enum {
  *                     reading it would need a device sync).  Chunks never
  *                     cross sequences; empty sequences are allowed.
  *   N               : num_seqs when cu_seqlens is given, else B.
- *   chunk           : chunk length; 64 is supported.
+ *   chunk           : chunk length C, 1 <= C <= 64 (KDA_ERR_UNSUPPORTED above:
+ *                     the tensor-core kernel's tiles are 64 tokens high, and a
+ *                     chunk shorter than 64 fills their first C rows, like the
+ *                     short last chunk of a sequence).  The result is the same
+ *                     for every C up to rounding; C trades the length of the
+ *                     sequential chain of chunk steps against the work per step.
  *   out             : [B, T, H, d_v] out_dtype (written).
  *   final_state     : [N, H, d_k, d_v] fp32, or NULL to skip.  It may alias
  *                     init_state exactly (in-place state update); partial
@@ -98,8 +103,11 @@ typedef enum {
  *                     may be NULL when that size is 0.  Owned by the caller,
  *                     used only during the call; calls that overlap on the
  *                     GPU must not share one workspace.
- * Supported: d_k == 128 and d_v in {64, 128} for bf16 (tensor-core path);
- * d_k, d_v in {64, 128} for fp32 (fp32 CUDA-core path, fp32 accuracy).
+ * Supported: d_k, d_v in {64, 128} for both dtypes.  bf16 runs on the tensor-
+ * core path (with d_k == 64 the key channels are zero-padded to 128 inside the
+ * kernel: the padded state rows stay zero and reach no output); fp32 I/O runs
+ * token by token on CUDA cores with the fp32 state (fp32 accuracy; the chunk
+ * length does not apply there).
  * T == 0 is valid (final_state = init_state or zeros).
  * The tensor-core path launches one CTA per SM of the device as a cooperative
  * grid (its CTAs wait on one another, so all must be resident at once); the
@@ -199,9 +207,9 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v, const vo
  *     log_alpha = logsigmoid(g_raw),  beta = sigmoid(b_raw)
  * q_raw, k_raw, g_raw take the places (and layouts) of q, k, log_alpha and
  * b_raw that of beta; everything else is as in kda_chunk_fwd / kda_decode_step.
- * kda_chunk_fwd_fused runs on the tensor-core path only (dtype KDA_BF16,
- * d_k == 128; KDA_ERR_UNSUPPORTED otherwise); kda_decode_step_fused supports
- * what kda_decode_step does.
+ * kda_chunk_fwd_fused runs on the tensor-core path only (dtype KDA_BF16;
+ * KDA_ERR_UNSUPPORTED otherwise); kda_decode_step_fused supports what
+ * kda_decode_step does.
  */
 kda_status kda_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const void *g_raw,
                                const void *b_raw, const float *init_state,
@@ -227,7 +235,7 @@ kda_status kda_decode_step_fused(const void *q_raw, const void *k_raw, const voi
  * only for such callers.
  *
  * Same arguments, layouts and results as kda_chunk_fwd, without workspace /
- * workspace_bytes.  Only the tensor-core path: dtype KDA_BF16, d_k == 128,
+ * workspace_bytes.  Only the tensor-core path: dtype KDA_BF16, d_k in {64, 128},
  * d_v in {64, 128}.  It allocates nothing (no cudaMalloc, no library
  * allocator).  Any number of (sequence, head) pairs fits: the chains' rings
  * are made shallower (down to 3 images) when the array cannot hold 12 each.

@@ -69,7 +69,8 @@ def test_rejects_bad_arguments(lib):
     assert chunk(lib, dk=96) == U
     assert chunk(lib, dv=256) == U
     assert chunk(lib, chunk_size=128) == U
-    assert chunk(lib, dk=64, dtype=_lib.KDA_BF16) == U   # tensor-core path needs d_k = 128
+    assert chunk(lib, dk=64, dtype=_lib.KDA_BF16) != U   # the tensor-core path takes d_k = 64 (zero-padded keys)
+    assert chunk(lib, chunk_size=32) != U                # chunks of up to 64 tokens
     assert chunk(lib, ws=None) == E                      # tensor-core path needs its workspace
     assert chunk(lib, ws_bytes=1024) == E
     rec = lib.kda_recurrent_fwd(FAKE, FAKE, FAKE, FAKE, None, None, None, 0, 1, 8, 1, 64, 64, _lib.KDA_F32,
@@ -94,7 +95,7 @@ def test_gdn_rejects_bad_arguments(lib):
     assert gchunk(gate=ODD) == E                 # a given gate must be 16-byte aligned like every tensor
     assert gchunk(gate=None, ws=None) == E       # a null gate (DeltaNet) is fine; the missing workspace is not
     assert gchunk(dk=96) == U
-    assert gchunk(chunk_size=32) == U
+    assert gchunk(chunk_size=128) == U
     # the per-channel gate of KDA stays mandatory
     assert lib.kda_chunk_fwd(FAKE, FAKE, FAKE, None, FAKE, None, None, 0, 1, 128, 2, 128, 128, 64, _lib.KDA_BF16,
                              _lib.KDA_F32, FAKE, None, FAKE, 1 << 30, None) == E
@@ -117,7 +118,7 @@ def test_fused_rejects_bad_arguments(lib):
     assert fchunk(q=None) == E
     assert fchunk(g=None) == E                    # the gate's pre-activation is required
     assert fchunk(dtype=_lib.KDA_F32, dk=64) == U  # tensor-core path only
-    assert fchunk(dk=64) == U
+    assert fchunk(dk=64) != U
     assert fchunk(ws=None) == E
     dec = lib.kda_decode_step_fused
     assert dec(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 128, 128, _lib.KDA_BF16, _lib.KDA_F32, None) == E
@@ -151,7 +152,8 @@ def test_workspace_size_rejects_what_the_prefill_rejects(lib):
         assert lib.kda_chunk_fwd_workspace_size(2, 16, dk, dv, dt, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
         assert n.value == 0
     # shapes the prefill accepts get a size (fp32: the CUDA-core path, no workspace)
-    for dk, dv, dt in [(128, 64, _lib.KDA_BF16), (64, 64, _lib.KDA_F32), (64, 128, _lib.KDA_F32)]:
+    for dk, dv, dt in [(128, 64, _lib.KDA_BF16), (64, 128, _lib.KDA_BF16), (64, 64, _lib.KDA_F32),
+                       (64, 128, _lib.KDA_F32)]:
         assert lib.kda_chunk_fwd_workspace_size(2, 16, dk, dv, dt, ctypes.byref(n)) == _lib.KDA_OK
 
 

@@ -112,3 +112,15 @@ def test_fused_decode_small(cuda_lib, dk, dv, dtype):
         assert rel_err(o, ref_o) <= tol
         assert rel_err(state, ref_s) <= tol
     assert device_error() == 0
+
+
+def test_fused_chunk_length_32_and_key_width_64(cuda_lib):
+    check_chunk(inputs.make_prefill("prefill_bf16", device="cpu", raw=True, B=1, T=200, H=2, dk=64, init_state=True))
+    x = inputs.make_prefill("prefill_bf16", device="cpu", raw=True, B=1, T=333, H=2, init_state=True)
+    dev = torch.device("cuda")
+    out, fs = kda_chunk_fwd_fused(*(x[n].to(dev) for n in NAMES), initial_state=x["init_state"].to(dev),
+                                  chunk_size=32)
+    torch.cuda.synchronize()
+    q, k, la, beta = oracle.prologue(*(np64(x[n]) for n in ("q", "k", "log_alpha", "beta")))
+    ref_o, ref_s = oracle.recurrent(q, k, np64(x["v"]), la, beta, init_state=np64(x["init_state"]))
+    assert rel_err(out, ref_o) <= BF16_TOL and rel_err(fs, ref_s) <= BF16_TOL

@@ -143,3 +143,10 @@ def test_gdn_decode_equals_kda_decode(cuda_lib):
     o2 = kda_decode_step(*tok, lg[..., None].expand_as(d["log_alpha"][0]).contiguous(), d["beta"][0], s2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_gdn_chunk_length_32_and_key_width_64(cuda_lib):
+    x = gdn_inputs("prefill_bf16", True, B=1, T=333, H=3, init_state=True)
+    run_and_check(lambda *a, **kw: gdn_chunk_fwd(*a, chunk_size=32, **kw), x, BF16_TOL)
+    y = gdn_inputs("prefill_bf16", True, B=2, T=150, H=3, dk=64, dv=64, init_state=True)
+    run_and_check(gdn_chunk_fwd, y, BF16_TOL)

@@ -222,3 +222,44 @@ def test_bf16_output_is_rounded_fp32_output(cuda_lib, fn):
     assert o16.dtype == torch.bfloat16
     assert torch.equal(o16, o32.to(torch.bfloat16))
     assert torch.equal(f16, f32)
+
+
+# ---- chunk length C <= 64 and key width 64 on the tensor-core path ---------------------------------
+
+@pytest.mark.parametrize("C", [16, 32, 48])
+@pytest.mark.parametrize("T", [17, 200, 333])
+def test_chunk_lengths(cuda_lib, C, T):
+    """Chunks of C < 64 tokens (the chunkwise form with another C; the result must not change)."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=T, H=3, init_state=True)
+    run_and_check(lambda *a, **kw: kda_chunk_fwd(*a, chunk_size=C, **kw), x, BF16_TOL)
+
+
+def test_chunk_length_32_varlen_and_many_pairs(cuda_lib):
+    lens = [1, 0, 64, 130, 7, 65, 0, 200]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    y = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=int(cu[-1]), H=10, init_state=False)
+    y["cu_seqlens"] = cu
+    y["init_state"] = torch.randn((len(lens), 10, 128, 128), generator=torch.Generator().manual_seed(8)) * 0.1
+    run_and_check(lambda *a, **kw: kda_chunk_fwd(*a, chunk_size=32, **kw), y, BF16_TOL)
+
+
+def test_chunk_length_128_is_unsupported(cuda_lib):
+    from gated_delta_rule_86_b200 import KdaError
+    x = inputs.make_prefill("prefill_bf16", device="cuda", B=1, T=64, H=1)
+    with pytest.raises(KdaError):
+        kda_chunk_fwd(*(x[n] for n in NAMES), chunk_size=128)
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("T", [1, 65, 333])
+def test_key_width_64_bf16(cuda_lib, dv, T):
+    """bf16 with d_k = 64 on the tensor-core path (keys zero-padded to 128 channels in the kernel)."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=T, H=3, dk=64, dv=dv, init_state=True)
+    run_and_check(kda_chunk_fwd, x, BF16_TOL)
+
+
+def test_key_width_64_strong_decay_and_chunk_32(cuda_lib):
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=300, H=2, dk=64, mu=-3.0, init_state=True)
+    run_and_check(kda_chunk_fwd, x, BF16_TOL)
+    y = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=250, H=5, dk=64, dv=64, init_state=True)
+    run_and_check(lambda *a, **kw: kda_chunk_fwd(*a, chunk_size=32, **kw), y, BF16_TOL)
