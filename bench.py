@@ -326,7 +326,7 @@ def hbm_roofline(alg_bytes, ms, hbm_peak, kernel="kda_chunk_tc_kernel", traffic=
             "traffic": traffic, "kernel": kernel, "alg_bytes_per_launch": alg_bytes}
 
 
-def prefill_block(args, world, x, hbm_peak, entry="kda_chunk_fwd", out_dtype=None, flush=None, label=None):
+def prefill_block(args, world, x, hbm_peak, entry="kda_chunk_fwd", out_dtype=None, flush=None, label=None, chunk=64):
     """Time one prefill entry point on the inputs x (a make_prefill dict on the GPU)."""
     import torch
 
@@ -339,13 +339,14 @@ def prefill_block(args, world, x, hbm_peak, entry="kda_chunk_fwd", out_dtype=Non
     N = B if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
 
     def step(_i):
-        return fn(*a, initial_state=x["init_state"], cu_seqlens=x["cu_seqlens"], out_dtype=out_dtype)
+        return fn(*a, initial_state=x["init_state"], cu_seqlens=x["cu_seqlens"], out_dtype=out_dtype, chunk_size=chunk)
 
     ms = timed_steps(step, args, world, flush)
     tokens = B * T
     alg = prefill_alg_bytes(tokens * H, N * H, dk, dv, out_bytes=4 if out_dtype == torch.float32 else 2)
     w = x["workload"]
     return {"entry": entry, "workload": label or w.name, "B": B, "T": T, "H": H, "N": N, "d_k": dk, "d_v": dv,
+            "chunk": chunk,
             "out_dtype": "f32" if out_dtype == torch.float32 else "bf16", "ms_per_step": ms,
             "tokens_per_s": world * tokens / (ms * 1e-3), "roofline": hbm_roofline(alg, ms, hbm_peak),
             "l2": "flushed before each call" if flush is not None else "inputs larger than L2"}
@@ -367,6 +368,41 @@ def gdn_prefill_block(args, world, a, s0, tokens, token_heads, hbm_peak):
     return {"entry": "gdn_chunk_fwd", "gate": "log_g [B,T,H] = the first key channel of the workload's log_alpha",
             "ms_per_step": ms_step, "tokens_per_s": world * tokens / (ms_step * 1e-3),
             "roofline": hbm_roofline(alg, ms_step, hbm_peak)}
+
+
+def bwd_alg_flops(token_heads, dk=128, dv=128):
+    """Algorithmic flops of the gradient per token-head: the adjoint step (dS += q do^T, dq, du, dk's two
+    terms, dS', dlog_alpha, dS_prev: 15 d_k d_v) plus the forward step it needs (S', w, S: 5 d_k d_v)."""
+    return token_heads * 20 * dk * dv
+
+
+FP32_PEAK_NOTE = "148 SMs x 128 fp32 FMA/clk x 2 flop x 1.965 GHz = 74.4 TFLOP/s (nominal CUDA-core peak)"
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_block(args, world):
+    """kda_chunk_bwd on the shape of the 4K prefill workload (B=2, H=16, T=4096, d=128)."""
+    import torch
+
+    from gated_delta_rule_86_b200 import inputs, kda_chunk_bwd
+    w = inputs.WORKLOADS["prefill_bf16"]
+    x = inputs.make_prefill(w, device="cuda", init_state=True)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    d_out = torch.randn(x["v"].shape, generator=g, device="cuda")
+    a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+
+    def step(_i):
+        return kda_chunk_bwd(*a, d_out, initial_state=x["init_state"])
+
+    ms = timed_steps(step, args, world)
+    th = w.B * w.T * w.H
+    flops = bwd_alg_flops(th)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"entry": "kda_chunk_bwd", "workload": "prefill_bf16 shape (B2 H16 T4096 d128), N(0,0.1) initial state, "
+            "N(0,1) upstream gradient", "ms_per_step": ms, "tokens_per_s": world * w.B * w.T / (ms * 1e-3),
+            "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tf / FP32_PEAK_TFLOPS, "traffic": None, "kernel": "kda_bwd_kernel",
+                         "alg_flops_per_launch": flops, "peak_source": FP32_PEAK_NOTE}}
 
 
 def oracle_single_thread(workload, T_s=4096):
@@ -474,6 +510,21 @@ def run_kda(args):
     del xr
     torch.cuda.empty_cache()
 
+    # ---------------- chunk length ablation and key width 64 on the same workload ----------------
+    ablation = {}
+    xa = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank)
+    for C in (16, 32, 64):
+        blk = prefill_block(args, world, dict(xa, workload=w), hbm_peak, chunk=C)
+        ablation[f"C{C}"] = {"ms_per_step": blk["ms_per_step"], "tokens_per_s": blk["tokens_per_s"],
+                             "chain_steps_per_head": -(-w.T // C), "roofline_frac": blk["roofline"]["frac"]}
+    del xa
+    x64 = inputs.make_prefill(w, device="cuda", seed=inputs.BASE_SEED + w.wid + 1000 * rank, dk=64)
+    dk64 = prefill_block(args, world, x64, hbm_peak, label="long_bf16 with d_k = 64")
+    del x64
+    torch.cuda.empty_cache()
+    bwd = backward_block(args, world)
+    torch.cuda.empty_cache()
+
     # ---------------- the other prefill workloads ----------------
     others = {}
     flush_buf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
@@ -552,10 +603,13 @@ def run_kda(args):
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h},
+                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                        "path": "kda_chunk_fwd on pinned host tensors: 8 token segments whose copies overlap the "
+                                "kernels (copy streams for H2D and D2H)"},
                 # per step: the schedule-table kernel and the chunk kernel
                 "gpu_launches": 2 * args.steps, "clocks": clocks, "decode": decode, "bf16_output": bf16_out,
-                "fused_prologue": fused, "gated_deltanet": gdn, "other_prefill_workloads": others}
+                "fused_prologue": fused, "gated_deltanet": gdn, "other_prefill_workloads": others,
+                "chunk_length_ablation": ablation, "key_width_64": dk64, "backward": bwd}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

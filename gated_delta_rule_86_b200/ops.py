@@ -85,9 +85,80 @@ def _out_dtype(out_dtype):
     return _DTYPES[out_dtype]
 
 
-def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state, chunk_size,
-             out_dtype):
+def _host_pipelined(fn_name, q, k, v, gate, beta, initial_state, chunk_size, out_dtype, segments):
+    """The prefill of one sequence (B == 1) held in pinned host memory, in token segments whose
+    host-to-device copies, kernels and device-to-host copies overlap: segment i's inputs travel on
+    one copy stream while segment i-1 runs and segment i-2's output travels back on another.  The
+    state passes from segment to segment on the device.  Segments start at multiples of the chunk
+    length, so the chunks, and therefore the results, are exactly those of one call."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    seg = -(-T // segments)
+    seg = -(-seg // chunk_size) * chunk_size
+    bounds = [(a, min(a + seg, T)) for a in range(0, T, seg)]
+    hosts = [q, k, v, gate, beta]
+    devs = [None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hosts]
+    out_d = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev)
+    out_h = torch.empty((B, T, H, dv), dtype=out_dtype, pin_memory=True)
+    st = [None, None]
+    state = None
+    if initial_state is not None:
+        state = initial_state.to(dev, non_blocking=True).to(torch.float32).contiguous()
+    compute = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d.wait_stream(compute)   # the device buffers are free for writing
     lib = _lib.load()
+    dt = _io_dtype(*hosts)
+    odt = _out_dtype(out_dtype)
+    ws_bytes = ctypes.c_size_t(0)
+    _lib.check(lib.kda_chunk_fwd_workspace_size(1, H, dk, dv, dt, ctypes.byref(ws_bytes)), "kda_chunk_fwd_workspace_size")
+    ws = torch.empty(max(ws_bytes.value, 16), dtype=torch.uint8, device=dev)
+    for i, (a, b) in enumerate(bounds):
+        ev_in = torch.cuda.Event()
+        with torch.cuda.stream(h2d):
+            for hd, dd in zip(hosts, devs):
+                if hd is not None:
+                    dd[:, a:b].copy_(hd[:, a:b], non_blocking=True)
+            ev_in.record(h2d)
+        compute.wait_event(ev_in)
+        fs = torch.empty((1, H, dk, dv), dtype=torch.float32, device=dev)
+        st[i & 1] = fs
+        segs = [None if dd is None else dd[:, a:b] for dd in devs]
+        status = getattr(lib, fn_name)(*(_ptr(x) for x in segs), _ptr(state), None, ctypes.c_int32(0), 1, b - a, H, dk,
+                                       dv, ctypes.c_int32(chunk_size), dt, odt, _ptr(out_d[:, a:b]), _ptr(fs),
+                                       _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle())
+        _lib.check(status, fn_name)
+        state = fs
+        ev_out = torch.cuda.Event()
+        ev_out.record(compute)
+        d2h.wait_event(ev_out)
+        with torch.cuda.stream(d2h):
+            out_h[:, a:b].copy_(out_d[:, a:b], non_blocking=True)
+    fs_h = None
+    if state is not None:
+        fs_h = torch.empty(state.shape, dtype=torch.float32, pin_memory=True)
+        with torch.cuda.stream(d2h):
+            fs_h.copy_(state, non_blocking=True)
+    d2h.synchronize()
+    compute.wait_stream(d2h)
+    for t in devs + [out_d, ws] + st:
+        if t is not None:
+            t.record_stream(d2h)
+    return out_h, fs_h
+
+
+def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state, chunk_size,
+             out_dtype, host_segments=8):
+    lib = _lib.load()
+    if (host_segments and host_segments > 1 and not q.is_cuda and cu_seqlens is None and "_chunk_fwd" in fn_name
+            and q.dim() == 4 and q.shape[0] == 1 and q.shape[1] >= 2 * host_segments * chunk_size
+            and all(t is None or (t.is_pinned() and t.is_contiguous()) for t in (q, k, v, log_alpha, beta))):
+        if log_alpha is None and not fn_name.startswith("gdn_"):
+            raise ValueError("log_alpha is required")
+        out_h, fs_h = _host_pipelined(fn_name, q, k, v, log_alpha, beta, initial_state, chunk_size, out_dtype,
+                                      host_segments)
+        return out_h, (fs_h if output_final_state else None)
     on_host, (q, k, v, la, beta, s0, cu), (B, T, H, dk, dv, N) = _prefill_prepare(
         q, k, v, log_alpha, beta, initial_state, cu_seqlens, per_head_gate=fn_name.startswith("gdn_"))
     dt = _io_dtype(q, k, v, la, beta)
@@ -119,16 +190,20 @@ def _prefill(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, outpu
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
-                  chunk_size=64, out_dtype=torch.float32):
+                  chunk_size=64, out_dtype=torch.float32, host_segments=8):
     """Chunkwise-parallel KDA prefill; returns ``(out, final_state)``.
 
     q, k, log_alpha: [B, T, H, d_k]; v: [B, T, H, d_v]; beta: [B, T, H] (one
     dtype: bf16 or fp32).  initial_state: fp32 [N, H, d_k, d_v] or None;
     cu_seqlens: int32 [N+1] for packed sequences (B == 1) or None.  out has
     dtype ``out_dtype`` (fp32 by default, the accumulator precision).
+    Inputs in pinned host memory are copied in and the results copied back;
+    for one sequence (B == 1) this runs in ``host_segments`` token segments
+    whose copies overlap the kernels (0 or 1: one copy in, one call, one
+    copy out).
     """
     return _prefill("kda_chunk_fwd", q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state,
-                    chunk_size, out_dtype)
+                    chunk_size, out_dtype, host_segments)
 
 
 def kda_recurrent_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
@@ -179,11 +254,11 @@ def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, out_dtype=torch.f
 
 
 def gdn_chunk_fwd(q, k, v, log_g, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
-                  chunk_size=64, out_dtype=torch.float32):
+                  chunk_size=64, out_dtype=torch.float32, host_segments=8):
     """Gated DeltaNet prefill (one log-decay per head and token): :func:`kda_chunk_fwd` with
     ``log_g`` [B, T, H] in place of log_alpha; ``log_g=None`` is DeltaNet (no decay)."""
     return _prefill("gdn_chunk_fwd", q, k, v, log_g, beta, initial_state, cu_seqlens, output_final_state,
-                    chunk_size, out_dtype)
+                    chunk_size, out_dtype, host_segments)
 
 
 def gdn_recurrent_fwd(q, k, v, log_g, beta, initial_state=None, cu_seqlens=None, output_final_state=True,
@@ -200,12 +275,12 @@ def gdn_decode_step(q, k, v, log_g, beta, state, out=None, out_dtype=torch.float
 
 
 def kda_chunk_fwd_fused(q_raw, k_raw, v, g_raw, b_raw, initial_state=None, cu_seqlens=None,
-                        output_final_state=True, chunk_size=64, out_dtype=torch.float32):
+                        output_final_state=True, chunk_size=64, out_dtype=torch.float32, host_segments=8):
     """:func:`kda_chunk_fwd` from the raw projections, activated inside the kernel's loads:
     q, k = L2-normalised q_raw, k_raw (over d_k, eps 1e-6 under the root), log_alpha =
     logsigmoid(g_raw), beta = sigmoid(b_raw).  Same shapes as kda_chunk_fwd; bf16 only."""
     return _prefill("kda_chunk_fwd_fused", q_raw, k_raw, v, g_raw, b_raw, initial_state, cu_seqlens,
-                    output_final_state, chunk_size, out_dtype)
+                    output_final_state, chunk_size, out_dtype, host_segments)
 
 
 def kda_decode_step_fused(q_raw, k_raw, v, g_raw, b_raw, state, out=None, out_dtype=torch.float32):

@@ -44,7 +44,7 @@ def test_gdn_prefill_block(monkeypatch):
 def test_prefill_block_bytes_follow_out_dtype(monkeypatch):
     seen = []
 
-    def fake_chunk(q, k, v, la, beta, initial_state=None, cu_seqlens=None, out_dtype=None):
+    def fake_chunk(q, k, v, la, beta, initial_state=None, cu_seqlens=None, out_dtype=None, chunk_size=64):
         seen.append(out_dtype)
         return None, None
 

@@ -263,3 +263,25 @@ def test_key_width_64_strong_decay_and_chunk_32(cuda_lib):
     run_and_check(kda_chunk_fwd, x, BF16_TOL)
     y = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=250, H=5, dk=64, dv=64, init_state=True)
     run_and_check(lambda *a, **kw: kda_chunk_fwd(*a, chunk_size=32, **kw), y, BF16_TOL)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_host_buffers_pipelined_equal_device_call(cuda_lib, out_dtype):
+    """Pinned host inputs of one sequence run in token segments whose copies overlap the kernels; the
+    segments start at multiples of the chunk length, so the result is bitwise that of one call on
+    device buffers (and the DeltaNet form, without a gate, takes the same route)."""
+    from gated_delta_rule_86_b200 import gdn_chunk_fwd
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=1000, H=4, init_state=True)
+    host = [x[n].pin_memory() for n in NAMES]
+    s0 = x["init_state"].pin_memory()
+    dev = torch.device("cuda")
+    o_d, f_d = kda_chunk_fwd(*(t.to(dev) for t in host), initial_state=s0.to(dev), out_dtype=out_dtype)
+    o_h, f_h = kda_chunk_fwd(*host, initial_state=s0, out_dtype=out_dtype, host_segments=4)
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    assert not o_h.is_cuda and o_h.is_pinned()
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(f_h, f_d.cpu())
+    g_d, gf_d = gdn_chunk_fwd(*(t.to(dev) for t in host[:3]), None, host[4].to(dev), initial_state=s0.to(dev))
+    g_h, gf_h = gdn_chunk_fwd(*host[:3], None, host[4], initial_state=s0, host_segments=4)
+    torch.cuda.synchronize()
+    assert torch.equal(g_h, g_d.cpu()) and torch.equal(gf_h, gf_d.cpu())
