@@ -119,12 +119,15 @@ __device__ __forceinline__ uint32_t a1_qg(int r, int j) { return a1_nw(r + kChun
 // ---- chain CTA shared memory ------------------------------------------------------------------
 template <int DV> struct ChainSmem {
     using I = Img<DV>;
-    // three image slots (Img layout); a slot is free again once the last MMA of its chunk completed
+    // two image slots (Img layout); a slot is free again once the last MMA of its chunk completed
     static constexpr int kSlotBytes = I::kStride;
-    static constexpr int kSlots = 3;
-    static_assert(kChunk * DV * 4 <= I::kUT - I::kA1, "output staging fits the dead A1 area");
+    static constexpr int kSlots = 2;
+    // two output staging buffers (fp32 or bf16 [DV / 64 blocks][64 tokens][64 values]), so that a
+    // chunk's TMA output store never holds up the reuse of an image slot
+    static constexpr int kStageBytes = kChunk * DV * 4;
+    static constexpr int kStage = kSlots * kSlotBytes;
     // exact path scratch (fp32): per-column partial sums of S^T k and S^T q per channel quarter, k . q
-    static constexpr int kRedPk = kSlots * kSlotBytes;
+    static constexpr int kRedPk = kStage + 2 * kStageBytes;
     static constexpr int kRedPq = kRedPk + 4 * 128 * 4;
     static constexpr int kRedKq = kRedPq + 4 * 128 * 4;
     static constexpr int kBytes = kRedKq + 16;
@@ -366,8 +369,8 @@ struct ChunkCtx {
 
 // Mbarriers of one CTA (each role uses its own subset).
 struct ChunkBars {
-    // chain: image slot full / free, MMA completions
-    uint64_t full[3], slot_free[3], mma1, mma2, mma3[2];
+    // chain: image slot full, MMA completions
+    uint64_t full[2], mma1, mma2, mma3[2];
     // chain: 1 + the chunk in which some state thread saw an fp16 overflow of U~ (ut) or of the state
     // operand (st); set before a plain barrier and compared with the chunk after it
     int ovf_ut, ovf_st;
@@ -1011,40 +1014,38 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
 
     if (warp >= kRoleWarps) {
         // ---- output and image warps 16-19: warp 16 + w reads TMEM lanes 32 w .. 32 w + 31, i.e. value
-        //      columns j = 32 w + lane of O^T (columns 64-127 of D1^T[b]) once [. ; P] U~ completed,
-        //      and stages them for TMA tensor stores (double-buffered); lane 1 of warp 16 copies
-        //      the chunk images from the chain's ring in global memory into the two slots ----
+        //      columns j = 32 w + lane of O^T (columns 64-127 of D1^T[b]) once [. ; P] U~ completed, and
+        //      stages them in their own double buffer for TMA tensor stores; lane 1 of warp 16 copies the
+        //      chunk images from the chain's ring in global memory into the two slots: image t + 2 goes
+        //      into chunk t's slot as soon as chunk t's last MMA has completed ----
         const int jo = (warp & 3) * 32 + lane;
         const bool jov = jo < DV;
         const bool lead = warp == kRoleWarps && lane == 0;
-        // the image copies are issued by another lane than the output stores: its flag waits then do
-        // not wait for the output stores still in flight
+        // the image copies are issued by another lane than the output stores: the image lane's fence and
+        // flag waits then do not wait for the output stores still in flight
         const bool lead_ld = warp == kRoleWarps && lane == 1;
         const uint32_t tlo = tc::tmem_lane_base(warp);
         constexpr uint32_t kOutThreads = kThreads - kRoleThreads;
-        // chunk whose image copy was issued last into each shared-memory slot (-1: none); the CTA
-        // waits for exactly these copies before it leaves
+        // chunk whose image copy was issued last into each slot (-1: none); copies into one slot are
+        // sequential (each waits for the MMAs that read the previous one), so these are the only copies
+        // that may be in flight when the CTA leaves
         int pend[SM::kSlots];
 #pragma unroll
         for (int i = 0; i < SM::kSlots; ++i) pend[i] = -1;
-        auto load_image = [&](int t) -> bool {   // lane 1 of warp 16
-            if (*abort_flag) return false;
-            const int rs = kc * sched.ring + t % sched.ring;
-            if (!tc::flag_wait_ge(sched.ready + rs, t + 1, abort_flag, sched.fw)) return false;
-            if (*abort_flag) return false;
+        auto ready_flag = [&](int t) { return sched.ready + kc * sched.ring + t % sched.ring; };
+        auto copy_image = [&](int t) {   // lane 1 of warp 16, once image t's ready flag has been seen
             tc::fence_async_global();
-            const uint8_t *src = sched.rings + (size_t)rs * I::kStride;
-            uint8_t *slot = sm + (t % SM::kSlots) * SM::kSlotBytes;
+            const uint8_t *src = sched.rings + ((size_t)kc * sched.ring + t % sched.ring) * I::kStride;
             uint64_t *fb = &bars.full[t % SM::kSlots];
             tc::mbar_arrive_expect_tx(fb, I::kBytes);
-            tc::bulk_load(slot, src, I::kBytes, fb);   // the image has the slot's layout: one copy
+            tc::bulk_load(sm + (t % SM::kSlots) * SM::kSlotBytes, src, I::kBytes, fb);   // one copy per image
             pend[t % SM::kSlots] = t;
-            return true;
         };
         if (lead_ld)
-            for (int t = 0; t < 2 && t < ttot; ++t)
-                if (!load_image(t)) break;
-        int stage_pending = -1;   // slot whose output store was issued, its read not yet confirmed
+            for (int t = 0; t < SM::kSlots && t < ttot; ++t) {
+                if (*abort_flag || !tc::flag_wait_ge(ready_flag(t), t + 1, abort_flag, sched.fw)) break;
+                copy_image(t);
+            }
         // a wait by lane 0 of warp 16, whose outcome all four warps share (they leave together)
         auto out_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
             bool ok = true;
@@ -1060,25 +1061,15 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
             const PairInfo pi = pair_info(sched, pr);
             const int h = pi.h;
             for (int c = 0; c < pi.nchunks; ++c, ++t) {
-                const int b = t & 1, s3 = t % SM::kSlots;
-                // the previous chunk's output store has read its staging: that slot may be refilled
-                if (lead && stage_pending >= 0) {
-                    tc::bulk_wait_read_all();
-                    tc::mbar_arrive(&bars.slot_free[stage_pending]);
-                    stage_pending = -1;
-                }
-                // first the image of chunk t + 2, into the slot of chunk t - 1 once that slot is free
-                // (two chunks ahead of its use)
-                bool lok = true;
-                if (lead_ld && t + 2 < ttot) {
-                    const int sp2 = (t + 2) % SM::kSlots;
-                    lok = (t < 1 || tc::mbar_wait(&bars.slot_free[sp2], ((t - 1) / SM::kSlots) & 1, abort_flag)) &&
-                          load_image(t + 2);
-                }
-                if (tc::named_sync_or(kBarOut, kOutThreads, !lok)) {
-                    stop = true;
-                    break;
-                }
+                const int b = t & 1;
+                TO *stage = reinterpret_cast<TO *>(sm + SM::kStage + b * SM::kStageBytes);
+                // the ready flag of image t + 2, read now (an acquire load) and used once chunk t's slot is
+                // free, so that its latency overlaps the waits below
+                const bool next = lead_ld && t + SM::kSlots < ttot;
+                const int seen = next ? tc::ld_acquire_gpu(ready_flag(t + SM::kSlots)) : 0;
+                // staging buffer b was last read by the TMA store of chunk t - 2 (at most one newer store,
+                // chunk t - 1's, may still be reading its buffer); the barrier below publishes this
+                if (lead) tc::bulk_wait_read_1();
                 // the state warps have chosen how chunk t is evaluated (outmode) ...
                 if (!out_wait(&bars.outq[b], ph_q[b])) {
                     stop = true;
@@ -1094,12 +1085,17 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     }
                     ph3[b] ^= 1u;
                 }
+                // every read of chunk t's slot is over (the state warps read it before they issue the
+                // chunk's last MMAs, or before they signal an exactly evaluated chunk): image t + 2 goes
+                // there.  A failed flag wait sets the abort flag, which the next barrier wait turns into a stop.
+                if (next && !*abort_flag &&
+                    (seen >= t + SM::kSlots + 1 ||
+                     tc::flag_wait_ge(ready_flag(t + SM::kSlots), t + SM::kSlots + 1, abort_flag, sched.fw)))
+                    copy_image(t + SM::kSlots);
                 if (mode == 2) {
                     const int64_t tok0 = pi.tok0(c);
                     const int L = pi.len(c);
                     const bool full = L == kChunk;
-                    // staging: the slot's A1 area, dead since MMA1 of this chunk (before [. ; P] U~)
-                    TO *stage = reinterpret_cast<TO *>(sm + s3 * SM::kSlotBytes + I::kA1);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {   // tokens 32 half + [0, 32)
                         float o[32];
@@ -1131,8 +1127,6 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                             for (int blk = 0; blk < DV / 64; ++blk)
                                 tc::tma_store_3d(&maps.o, blk * 64, h, static_cast<int>(tok0),
                                                  stage + blk * (kChunk * 64));
-                            tc::bulk_commit();
-                            stage_pending = s3;
                         }
                     }
                 } else {
@@ -1140,14 +1134,13 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&bars.d1_free[b]);
                 }
-                // no output store reads this chunk's slot (partial chunk, or no tensor output)
-                if (lead && stage_pending != s3) tc::mbar_arrive(&bars.slot_free[s3]);
+                // one bulk group per chunk (empty when the chunk had no TMA store), so that wait_group.read 1
+                // at the top always names chunk t - 1's group
+                if (lead) tc::bulk_commit();
             }
         }
         if (lead) tc::bulk_wait_all();   // every output store has completed before the CTA leaves
         if (lead_ld) {
-            // no image copy may still be in flight either (only copies that were issued are awaited:
-            // after an abort some chunks' copies never were)
             int never = 0;
 #pragma unroll
             for (int i = 0; i < SM::kSlots; ++i)
@@ -1395,7 +1388,6 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                         stop = true;
                         break;
                     }
-                    if (leader) tc::mbar_arrive(&bars.slot_free[s]);   // done with the slot
                     continue;
                 }
             }
@@ -1407,7 +1399,6 @@ __device__ __forceinline__ void chain_role(const ChunkCtx &cx, ChunkBars &bars, 
                 stop = true;
                 break;
             }
-            if (leader) tc::mbar_arrive(&bars.slot_free[s]);
         }
         if (!stop && final_state && *abort_flag == 0 && jv && kin) {
 #pragma unroll
@@ -1436,11 +1427,7 @@ kda_chunk_tc_kernel(const __grid_constant__ RowMaps maps, const __grid_constant_
     const bool is_chain = static_cast<int>(blockIdx.x) < sched.nchain;
     if (tid == 0) {
         if (!is_chain) s_tmax = chain_tmax(sched);
-        for (int i = 0; i < 3; ++i) {
-            tc::mbar_init(&bars.full[i], 1);
-            // the state warps are done with the slot's chunk; its output store has read the slot
-            tc::mbar_init(&bars.slot_free[i], 2);
-        }
+        for (int i = 0; i < 2; ++i) tc::mbar_init(&bars.full[i], 1);
         tc::mbar_init(&bars.mma1, 1);
         tc::mbar_init(&bars.mma2, 1);
         tc::mbar_init(&bars.mma3[0], 1);
