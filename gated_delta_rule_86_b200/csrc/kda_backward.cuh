@@ -18,13 +18,16 @@
 // The result equals the gradient of the chunked forward up to rounding, because the chunked
 // forward equals the recurrence.
 //
-// Schedule.  One CTA per (sequence, head).  Thread (warp w, lane l) owns key rows
-// [32 (w / NCG), +32) and value column 32 (w % NCG) + l of the d_k x d_v state and of its gradient,
-// in fp32 registers, so every sum over d_v or d_k is a shuffle transpose-sum inside a warp plus a
-// deterministic combine across warps in shared memory (no atomics: results are reproducible).
+// Schedule.  One cluster of d_v / 32 CTAs per (sequence, head); CTA s of the cluster owns value
+// columns [32 s, 32 s + 32) of the d_k x d_v state and of its gradient (the columns evolve
+// independently).  Thread (warp w, lane l) owns key rows [32 w, 32 w + 32) and column 32 s + l, in
+// fp32 registers, so every sum over d_k is a combine of the warps' partials in shared memory, and
+// every sum over d_v is a shuffle transpose-sum inside a warp (the CTA's 32 columns) plus a combine
+// of the cluster's slices through distributed shared memory, once per block of 32 tokens.  Both
+// combines run in a fixed order (no atomics: results are reproducible).
 //   1. forward over the sequence, storing the state at the start of every chunk of C tokens
 //      (the checkpoints, in the workspace);
-//   2. chunks in reverse: the chunk's states are recomputed from its checkpoint into a per-CTA
+//   2. chunks in reverse: the chunk's states are recomputed from its checkpoint into a per-pair
 //      scratch (one d_k x d_v state per token), then its tokens are visited in reverse.
 // Token vectors move through shared memory 32 tokens at a time.  Each token costs three passes of
 // the recurrence (checkpoint pass, recompute, reverse), all in fp32.
@@ -54,20 +57,20 @@ __device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
 }
 
 template <int DK, int DV> struct Smem {
-    static constexpr int NRG = DK / 32, NCG = DV / 32;
+    static constexpr int NRG = DK / 32, NCS = DV / 32;   // warps per CTA, CTAs per cluster
     static constexpr int kQ = 0;                       // [kSub][DK]
     static constexpr int kK = kQ + kSub * DK;          // [kSub][DK]
     static constexpr int kA = kK + kSub * DK;          // [kSub][DK]  exp(log_alpha)
-    static constexpr int kV = kA + kSub * DK;          // [kSub][DV]
-    static constexpr int kDo = kV + kSub * DV;         // [kSub][DV]
-    static constexpr int kB = kDo + kSub * DV;         // [kSub]
-    static constexpr int kRedW = kB + kSub;            // [2][NRG][DV]
-    static constexpr int kRedDu = kRedW + 2 * NRG * DV;   // [NRG][DV]
-    static constexpr int kRedQ = kRedDu + NRG * DV;    // [NCG][DK]
-    static constexpr int kRedK = kRedQ + NCG * DK;     // [NCG][DK]
-    static constexpr int kRedG = kRedK + NCG * DK;     // [NCG][DK]
-    static constexpr int kRedB = kRedG + NCG * DK;     // [NCG]
-    static constexpr int kFloats = kRedB + NCG;
+    static constexpr int kV = kA + kSub * DK;          // [kSub][32]  this CTA's value columns
+    static constexpr int kDo = kV + kSub * 32;         // [kSub][32]
+    static constexpr int kB = kDo + kSub * 32;         // [kSub]
+    static constexpr int kRedW = kB + kSub;            // [2][NRG][32]
+    static constexpr int kRedDu = kRedW + 2 * NRG * 32;   // [NRG][32]
+    // this slice's partial sums over its 32 columns, double-buffered by block: dq, dk, dlog_alpha
+    // ([3][kSub][DK]) and dbeta ([kSub])
+    static constexpr int kPart = kRedDu + NRG * 32;
+    static constexpr int kPartFloats = 3 * kSub * DK + kSub;
+    static constexpr int kFloats = kPart + 2 * kPartFloats;
 };
 
 // Checkpoint slots of the sequence whose tokens start at t0: sequences never share one
@@ -78,8 +81,26 @@ inline int64_t ckpts_per_head(int64_t total_tokens, int N, int C) { return total
 
 }  // namespace bwd
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA of the cluster: arrive (release), then wait (acquire).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 load from the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_dsmem(const float *local, uint32_t rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local)), ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
 template <int DK, int DV, typename TIO, typename TDO>
-__global__ void __launch_bounds__(32 * (DK / 32) * (DV / 32))
+__global__ void __launch_bounds__(32 * (DK / 32))
 kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *__restrict__ v,
                const TIO *__restrict__ log_alpha, const TIO *__restrict__ beta, const float *init_state,
                const int32_t *__restrict__ cu, int T, int H, int C, const TDO *__restrict__ dout,
@@ -87,17 +108,17 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
                float *__restrict__ dla, float *__restrict__ dbeta, float *dinit, float *ckpt, float *scratch,
                int64_t nck_head) {
     using SM = bwd::Smem<DK, DV>;
-    constexpr int NRG = SM::NRG, NCG = SM::NCG, NT = 32 * NRG * NCG;
+    constexpr int NRG = SM::NRG, NCS = SM::NCS, NT = 32 * NRG;
     constexpr int kSub = bwd::kSub;
     extern __shared__ float smf[];
     float *sq = smf + SM::kQ, *sk = smf + SM::kK, *sa = smf + SM::kA, *sv = smf + SM::kV, *sdo = smf + SM::kDo;
-    float *sb = smf + SM::kB, *red_w = smf + SM::kRedW, *red_du = smf + SM::kRedDu, *red_q = smf + SM::kRedQ;
-    float *red_k = smf + SM::kRedK, *red_g = smf + SM::kRedG, *red_b = smf + SM::kRedB;
+    float *sb = smf + SM::kB, *red_w = smf + SM::kRedW, *red_du = smf + SM::kRedDu, *part = smf + SM::kPart;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rg = warp / NCG, cg = warp % NCG;
-    const int j = cg * 32 + lane, r0 = rg * 32;
-    const int pair = blockIdx.x, h = pair % H, n = pair / H;
+    const int rg = warp, r0 = rg * 32;
+    const int cs = static_cast<int>(cluster_ctarank());   // == blockIdx.x % NCS
+    const int j = cs * 32 + lane;
+    const int pair = blockIdx.x / NCS, h = pair % H, n = pair / H;
     const int64_t t0 = cu ? (int64_t)cu[n] : (int64_t)n * T;
     const int64_t t1 = cu ? (int64_t)cu[n + 1] : t0 + T;
     const int L = static_cast<int>(t1 - t0);
@@ -118,33 +139,50 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
             sa[tk * DK + c] = expf(to_f32(log_alpha[row * DK + c]));
             if (need_q) sq[tk * DK + c] = to_f32(q[row * DK + c]);
         }
-        for (int idx = tid; idx < nb * DV; idx += NT) {
-            const int tk = idx / DV, c = idx - tk * DV;
+        for (int idx = tid; idx < nb * 32; idx += NT) {
+            const int tk = idx >> 5, c = idx & 31;
             const size_t row = (size_t)(t0 + ts + tk) * H + h;
-            sv[tk * DV + c] = to_f32(v[row * DV + c]);
-            if (need_q) sdo[tk * DV + c] = to_f32(dout[row * DV + c]);
+            sv[tk * 32 + c] = to_f32(v[row * DV + cs * 32 + c]);
+            if (need_q) sdo[tk * 32 + c] = to_f32(dout[row * DV + cs * 32 + c]);
         }
         for (int tk = tid; tk < nb; tk += NT) sb[tk] = to_f32(beta[(size_t)(t0 + ts + tk) * H + h]);
         __syncthreads();
     };
+    // this thread's 32 key rows of a staged token vector (16-byte shared-memory loads, the same
+    // address across the warp)
+    auto rows32 = [&](const float *base, float (&o)[32]) {
+        const float4 *p4 = reinterpret_cast<const float4 *>(base + r0);
+#pragma unroll
+        for (int m4 = 0; m4 < 8; ++m4) {
+            const float4 f = p4[m4];
+            o[4 * m4] = f.x;
+            o[4 * m4 + 1] = f.y;
+            o[4 * m4 + 2] = f.z;
+            o[4 * m4 + 3] = f.w;
+        }
+    };
     // one forward step of the staged token i on the state S (one barrier; red_w is double-buffered)
     int wbuf = 0;
     auto forward_step = [&](float (&S)[32], int i) {
-        float pw = 0.f;
+        float ka[32], aa[32];
+        rows32(sk + i * DK, ka);
+        rows32(sa + i * DK, aa);
+        float pw4[4] = {0.f, 0.f, 0.f, 0.f};   // four interleaved partial sums over the 32 rows
 #pragma unroll
         for (int m = 0; m < 32; ++m) {
-            S[m] *= sa[i * DK + r0 + m];
-            pw = fmaf(S[m], sk[i * DK + r0 + m], pw);
+            S[m] *= aa[m];
+            pw4[m & 3] = fmaf(S[m], ka[m], pw4[m & 3]);
         }
-        red_w[(wbuf * NRG + rg) * DV + j] = pw;
+        const float pw = (pw4[0] + pw4[1]) + (pw4[2] + pw4[3]);
+        red_w[(wbuf * NRG + rg) * 32 + lane] = pw;
         __syncthreads();
         float w = 0.f;
 #pragma unroll
-        for (int g = 0; g < NRG; ++g) w += red_w[(wbuf * NRG + g) * DV + j];
+        for (int g = 0; g < NRG; ++g) w += red_w[(wbuf * NRG + g) * 32 + lane];
         wbuf ^= 1;
-        const float u = sb[i] * (sv[i * DV + j] - w);
+        const float u = sb[i] * (sv[i * 32 + lane] - w);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) S[m] = fmaf(sk[i * DK + r0 + m], u, S[m]);
+        for (int m = 0; m < 32; ++m) S[m] = fmaf(ka[m], u, S[m]);
     };
 
     // ---- 1. forward with a checkpoint at the start of every chunk ----
@@ -168,99 +206,121 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     float dS[32];
 #pragma unroll
     for (int m = 0; m < 32; ++m) dS[m] = dfinal ? dfinal[sbase + el(m)] : 0.f;
+    int blk = 0;   // reverse blocks so far (selects the partial-sum buffer)
     for (int c = nck - 1; c >= 0; --c) {
-        const int cs = c * C, ce = min(L, cs + C);
+        const int cs0 = c * C, ce = min(L, cs0 + C);
         // recompute: the state before every token of the chunk, into the scratch
         {
             float S[32];
 #pragma unroll
             for (int m = 0; m < 32; ++m) S[m] = my_ck[(size_t)c * kv + el(m)];
-            for (int ts = cs; ts < ce; ts += kSub) {
+            for (int ts = cs0; ts < ce; ts += kSub) {
                 const int nb = min(kSub, ce - ts);
                 stage(ts, nb, false);
                 for (int i = 0; i < nb; ++i) {
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) my_scr[(size_t)(ts - cs + i) * kv + el(m)] = S[m];
+                    for (int m = 0; m < 32; ++m) my_scr[(size_t)(ts - cs0 + i) * kv + el(m)] = S[m];
                     forward_step(S, i);
                 }
             }
         }
         // reverse over the chunk's tokens, in staged blocks from the end
-        const int nblk = (ce - cs + kSub - 1) / kSub;
-        for (int bi = nblk - 1; bi >= 0; --bi) {
-            const int ts = cs + bi * kSub, nb = min(kSub, ce - ts);
+        const int nblk = (ce - cs0 + kSub - 1) / kSub;
+        for (int bi = nblk - 1; bi >= 0; --bi, ++blk) {
+            const int ts = cs0 + bi * kSub, nb = min(kSub, ce - ts);
+            float *pq = part + (blk & 1) * SM::kPartFloats, *pk = pq + kSub * DK, *pg = pk + kSub * DK;
+            float *pb = pg + kSub * DK;
             stage(ts, nb, true);
+            // the recomputed state before token i, loaded one token ahead of its use
+            float Sn[32];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + nb - 1) * kv + el(m)];
             for (int i = nb - 1; i >= 0; --i) {
-                const size_t trow = (size_t)(t0 + ts + i) * H + h;
+                float ka[32], aa[32];
+                rows32(sk + i * DK, ka);
+                rows32(sa + i * DK, aa);
                 // S' = Diag(a) S_prev and w = S'^T k
                 float Sp[32];
-                float pw = 0.f;
+                float pw4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int m = 0; m < 32; ++m) {
-                    Sp[m] = sa[i * DK + r0 + m] * my_scr[(size_t)(ts - cs + i) * kv + el(m)];
-                    pw = fmaf(Sp[m], sk[i * DK + r0 + m], pw);
+                    Sp[m] = aa[m] * Sn[m];
+                    pw4[m & 3] = fmaf(Sp[m], ka[m], pw4[m & 3]);
                 }
-                red_w[(wbuf * NRG + rg) * DV + j] = pw;
+                if (i > 0) {
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + i - 1) * kv + el(m)];
+                }
+                const float pw = (pw4[0] + pw4[1]) + (pw4[2] + pw4[3]);
+                red_w[(wbuf * NRG + rg) * 32 + lane] = pw;
                 __syncthreads();
                 float w = 0.f;
 #pragma unroll
-                for (int g = 0; g < NRG; ++g) w += red_w[(wbuf * NRG + g) * DV + j];
+                for (int g = 0; g < NRG; ++g) w += red_w[(wbuf * NRG + g) * 32 + lane];
                 wbuf ^= 1;
-                const float bt = sb[i], vj = sv[i * DV + j], doj = sdo[i * DV + j];
+                const float bt = sb[i], vj = sv[i * 32 + lane], doj = sdo[i * 32 + lane];
                 const float u = bt * (vj - w);
                 // o = S^T q: dS += q do^T, dq = S do (S = S' + k u^T)
                 float x[32];
-                float pdu = 0.f;
+                {
+                    float qa[32];
+                    rows32(sq + i * DK, qa);
+                    float pdu4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    const float km = sk[i * DK + r0 + m];
-                    dS[m] = fmaf(sq[i * DK + r0 + m], doj, dS[m]);
-                    x[m] = fmaf(km, u, Sp[m]) * doj;
-                    pdu = fmaf(dS[m], km, pdu);   // du = dS^T k
+                    for (int m = 0; m < 32; ++m) {
+                        dS[m] = fmaf(qa[m], doj, dS[m]);
+                        x[m] = fmaf(ka[m], u, Sp[m]) * doj;
+                        pdu4[m & 3] = fmaf(dS[m], ka[m], pdu4[m & 3]);   // du = dS^T k
+                    }
+                    red_du[rg * 32 + lane] = (pdu4[0] + pdu4[1]) + (pdu4[2] + pdu4[3]);
                 }
-                red_q[cg * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
-                red_du[rg * DV + j] = pdu;
+                pq[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
                 __syncthreads();
                 float du = 0.f;
 #pragma unroll
-                for (int g = 0; g < NRG; ++g) du += red_du[g * DV + j];
+                for (int g = 0; g < NRG; ++g) du += red_du[g * 32 + lane];
                 if (rg == 0) {
-                    dv[trow * DV + j] = bt * du;
+                    dv[((size_t)(t0 + ts + i) * H + h) * DV + j] = bt * du;
                     float db = du * (vj - w);
 #pragma unroll
                     for (int o = 16; o >= 1; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
-                    if (lane == 0) red_b[cg] = db;
+                    if (lane == 0) pb[i] = db;
                 }
                 // dk = dS u - beta S' du;  dS' = dS - beta k du^T;  dlog_alpha = rowsum(dS' * S');  dS = a dS'
 #pragma unroll
                 for (int m = 0; m < 32; ++m) x[m] = dS[m] * u - bt * Sp[m] * du;
-                red_k[cg * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
+                pk[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
 #pragma unroll
                 for (int m = 0; m < 32; ++m) {
-                    dS[m] = fmaf(-bt * sk[i * DK + r0 + m], du, dS[m]);
+                    dS[m] = fmaf(-bt * ka[m], du, dS[m]);
                     x[m] = dS[m] * Sp[m];
-                    dS[m] *= sa[i * DK + r0 + m];
+                    dS[m] *= aa[m];
                 }
-                red_g[cg * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
-                __syncthreads();
-                if (tid < DK) {
-                    float aq = 0.f, ak = 0.f, ag = 0.f;
+                pg[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
+            }
+            // the block's sums over d_v: every slice's partials are complete (cluster barrier), then
+            // CTA s combines the elements e = s NT + tid, + NCS NT, ... over the slices in order 0, 1, ...
+            // (the buffer is rewritten two blocks later, after every CTA has passed the next barrier)
+            cluster_sync();
+            for (int e = cs * NT + tid; e < nb * DK; e += NCS * NT) {
+                const int i = e / DK, r = e - i * DK;
+                float aq = 0.f, ak = 0.f, ag = 0.f;
 #pragma unroll
-                    for (int g = 0; g < NCG; ++g) {
-                        aq += red_q[g * DK + tid];
-                        ak += red_k[g * DK + tid];
-                        ag += red_g[g * DK + tid];
-                    }
-                    dq[trow * DK + tid] = aq;
-                    dk[trow * DK + tid] = ak;
-                    dla[trow * DK + tid] = ag;
+                for (int g = 0; g < NCS; ++g) {
+                    aq += ld_dsmem(pq + i * DK + r, g);
+                    ak += ld_dsmem(pk + i * DK + r, g);
+                    ag += ld_dsmem(pg + i * DK + r, g);
                 }
-                if (tid == DK % NT) {
-                    float ab = 0.f;
+                const size_t trow = (size_t)(t0 + ts + i) * H + h;
+                dq[trow * DK + r] = aq;
+                dk[trow * DK + r] = ak;
+                dla[trow * DK + r] = ag;
+            }
+            for (int i = cs * NT + tid; i < nb; i += NCS * NT) {
+                float ab = 0.f;
 #pragma unroll
-                    for (int g = 0; g < NCG; ++g) ab += red_b[g];
-                    dbeta[trow] = ab;
-                }
+                for (int g = 0; g < NCS; ++g) ab += ld_dsmem(pb + i, g);
+                dbeta[(size_t)(t0 + ts + i) * H + h] = ab;
             }
         }
     }
@@ -268,6 +328,7 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
 #pragma unroll
         for (int m = 0; m < 32; ++m) dinit[sbase + el(m)] = dS[m];
     }
+    cluster_sync();   // no CTA leaves while another may still read its shared memory
 }
 
 // Workspace of the backward: the checkpoints (one d_k x d_v state per chunk of every sequence and
@@ -292,12 +353,25 @@ cudaError_t launch_bwd_dk_dv(const void *q, const void *k, const void *v, const 
     const int64_t nck_head = bwd::ckpts_per_head(total, N, C);
     float *ck = static_cast<float *>(workspace);
     float *scr = ck + (size_t)H * nck_head * DK * DV;
-    const unsigned grid = static_cast<unsigned>(N) * H;
+    const unsigned grid = static_cast<unsigned>(N) * H * SM::NCS;
     if (grid == 0) return cudaSuccess;
-    kern<<<grid, 32 * (DK / 32) * (DV / 32), smem, stream>>>(
-        static_cast<const TIO *>(q), static_cast<const TIO *>(k), static_cast<const TIO *>(v),
-        static_cast<const TIO *>(la), static_cast<const TIO *>(beta), init_state, cu, T, H, C,
-        static_cast<const TDO *>(dout), dfinal, dq, dk, dv, dla, dbeta, dinit, ck, scr, nck_head);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * SM::NRG);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;   // the d_v slices of one (sequence, head)
+    attr[0].val.clusterDim.x = SM::NCS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const TIO *>(q), static_cast<const TIO *>(k),
+                           static_cast<const TIO *>(v), static_cast<const TIO *>(la), static_cast<const TIO *>(beta),
+                           init_state, cu, T, H, C, static_cast<const TDO *>(dout), dfinal, dq, dk, dv, dla, dbeta,
+                           dinit, ck, scr, nck_head);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -271,9 +271,11 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
  *     dS += q do^T;  dq = S do;  du = dS^T k;  dk = dS u - beta S' du;
  *     dbeta = du . (v - w);  dv = beta du;  dS' = dS - beta k du^T;
  *     dlog_alpha = rowsum(dS' * S');  dS_prev = Diag(alpha) dS'.
- * All arithmetic is fp32 on CUDA cores; one CTA per (sequence, head) keeps
- * the state and its gradient in registers and reduces over d_k and d_v in a
- * fixed order (results are reproducible run to run).
+ * All arithmetic is fp32 on CUDA cores.  One cluster of d_v / 32 CTAs per
+ * (sequence, head) keeps the state and its gradient in registers, each CTA a
+ * 32-column slice; sums over d_k and d_v (the latter across the cluster through
+ * distributed shared memory) run in a fixed order (results are reproducible
+ * run to run).
  *
  *   q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, B, T, H,
  *   d_k, d_v, dtype : as for kda_chunk_fwd (the forward's inputs).
