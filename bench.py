@@ -41,16 +41,28 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LIB_SOURCES = ("gated_delta_rule_86_b200/csrc", "include")
 
 
-def build_hash():
-    """Hash of the library's sources (csrc/*.cu, *.cuh, include/*.h): names the build that a
-    profile summary was captured on."""
+# The csrc files that a profiled kernel's device code and launch come from (the kernel's header and
+# the headers it includes): its DRAM traffic depends on these alone.
+KERNEL_SOURCES = {
+    "kda_chunk_tc_kernel": ("kda_chunk_tc.cuh", "kda_common.cuh", "kda_recurrent.cuh", "tc_utils.cuh"),
+    "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
+    "kda_bwd_kernel": ("kda_backward.cuh", "kda_common.cuh"),
+}
+
+
+def build_hash(kernel=None):
+    """Hash of the library's sources (csrc/*.cu, *.cuh, include/*.h), or of one kernel's sources
+    (KERNEL_SOURCES): names the build that a profile summary was captured on."""
     import glob
     import hashlib
     h = hashlib.sha256()
     files = []
-    for d in LIB_SOURCES:
-        for ext in ("*.cu", "*.cuh", "*.h"):
-            files += glob.glob(os.path.join(ROOT, d, ext))
+    if kernel is not None:
+        files = [os.path.join(ROOT, LIB_SOURCES[0], f) for f in KERNEL_SOURCES[kernel]]
+    else:
+        for d in LIB_SOURCES:
+            for ext in ("*.cu", "*.cuh", "*.h"):
+                files += glob.glob(os.path.join(ROOT, d, ext))
     for f in sorted(files):
         h.update(os.path.relpath(f, ROOT).encode())
         with open(f, "rb") as fh:
@@ -60,10 +72,11 @@ def build_hash():
 
 def traffic_record(kernel, workload):
     """The DRAM traffic record of `kernel` on `workload` from profiles/*.md (a line
-    `traffic-record: {json}` written next to the ncu summary), if it was captured on the current
-    build; else None.  Keys: build, kernel, workload, dram_bytes, units, units_per_launch."""
+    `traffic-record: {json}` written next to the ncu summary), if it was captured on the kernel's
+    current sources (build_hash(kernel)); else None.  Keys: build, kernel, workload, dram_bytes,
+    units."""
     import glob
-    want = build_hash()
+    want = build_hash(kernel)
     for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(f) as fh:
             for line in fh:
@@ -456,8 +469,8 @@ def run_kda(args):
     alg_bytes = prefill_alg_bytes(token_heads, w.B * w.H)
     alg_flops = prefill_alg_flops(token_heads)
     dense_flops = token_heads * (12 * w.chunk * w.dk + 6 * w.dk * w.dv)
-    # DRAM traffic per launch: from an ncu capture of this very build (a traffic-record line in
-    # profiles/, matched by the hash of the library sources), scaled to this launch by the units it
+    # DRAM traffic per launch: from an ncu capture of this very kernel build (a traffic-record line in
+    # profiles/, matched by the hash of the kernel's sources), scaled to this launch by the units it
     # processes; null when no capture of this build exists
     rec = traffic_record("kda_chunk_tc_kernel", PREFILL_WORKLOAD)
     traffic = None
@@ -470,7 +483,7 @@ def run_kda(args):
         "traffic_source": None if rec is None else
         f"{rec['file']}: ncu dram__bytes_read.sum + dram__bytes_write.sum on {rec['units']} token-heads "
         f"(build {rec['build']}), scaled by token-heads",
-        "build": build_hash(),
+        "build": build_hash("kda_chunk_tc_kernel"),
         "tensor": {"alg_flops_per_launch": alg_flops,
                    "achieved_tflops": alg_flops / (ms_step * 1e-3) / 1e12,
                    "frac_of_burst_peak": alg_flops / (ms_step * 1e-3) / 1e12 / tc_peak_burst,
@@ -563,12 +576,17 @@ def run_kda(args):
     heads = dw.B * dw.H
     d_bytes = decode_alg_bytes(heads)
     d_gbs = d_bytes / (dms_step * 1e-3) / 1e9
+    drec = traffic_record("kda_decode_kernel", DECODE_WORKLOAD)   # units: head-steps of the capture
+    d_traffic = None if drec is None else drec["dram_bytes"] * heads / drec["units"]
     decode = {"workload": DECODE_WORKLOAD, "B": dw.B, "H": dw.H, "d_k": dw.dk, "d_v": dw.dv, "steps": nsteps,
               "steps_per_s": world * 1e3 / dms_step, "tokens_per_s": world * dw.B * 1e3 / dms_step,
               "us_per_step": dms_step * 1e3,
               "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": hbm_peak, "unit": "GB/s",
-                           "frac": d_gbs / hbm_peak, "traffic": None, "kernel": "kda_decode_kernel",
-                           "alg_bytes_per_launch": d_bytes}}
+                           "frac": d_gbs / hbm_peak, "traffic": d_traffic, "kernel": "kda_decode_kernel",
+                           "alg_bytes_per_launch": d_bytes,
+                           "traffic_source": None if drec is None else
+                           f"{drec['file']}: ncu dram__bytes_read.sum + dram__bytes_write.sum on {drec['units']} "
+                           f"head-steps (build {drec['build']})"}}
     # decode end to end: tokens from pinned host memory each step, output read back each step
     hq = [d[n][:64].cpu().pin_memory() for n in names]
     hout = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, pin_memory=True)
@@ -621,16 +639,24 @@ def run_profile_case(args):
 
     chunk:  kda_chunk_fwd on B=1, H=32, T=16384 (0.54 GB of bf16 inputs, above L2).
     decode: kda_decode_step on the full decode workload state (B=256, H=32, 512 MiB fp32).
+    bwd:    kda_chunk_bwd on the backward block's shape (B=2, H=16, T=4096).
     """
     import torch
 
-    from gated_delta_rule_86_b200 import inputs, kda_chunk_fwd, kda_decode_step
+    from gated_delta_rule_86_b200 import inputs, kda_chunk_bwd, kda_chunk_fwd, kda_decode_step
     torch.cuda.set_device(0)
     if args.profile == "chunk":
         x = inputs.make_prefill(PREFILL_WORKLOAD, device="cuda", T=16384)
         a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
         for _ in range(3):
             kda_chunk_fwd(*a, initial_state=x["init_state"])
+    elif args.profile == "bwd":
+        x = inputs.make_prefill("prefill_bf16", device="cuda", init_state=True)
+        g = torch.Generator(device="cuda").manual_seed(5)
+        d_out = torch.randn(x["v"].shape, generator=g, device="cuda")
+        a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+        for _ in range(3):
+            kda_chunk_bwd(*a, d_out, initial_state=x["init_state"])
     else:
         d = inputs.make_decode(DECODE_WORKLOAD, device="cuda", steps=4)
         for i in range(4):
@@ -648,7 +674,7 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--ref-seconds", type=float, default=10.0, help="target CPU seconds per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["chunk", "decode"], default=None,
+    ap.add_argument("--profile", choices=["chunk", "decode", "bwd"], default=None,
                     help="run a small fixed launch set for an ncu capture (no timing output)")
     args = ap.parse_args()
     if args.profile:

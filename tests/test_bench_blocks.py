@@ -74,16 +74,29 @@ def test_traffic_record_needs_the_current_build(tmp_path, monkeypatch):
     for d in bench.LIB_SOURCES:
         (tmp_path / d).mkdir(parents=True)
     (tmp_path / "include" / "kda.h").write_text("int x;\n")
+    csrc = tmp_path / bench.LIB_SOURCES[0]
+    for f in {f for fs in bench.KERNEL_SOURCES.values() for f in fs}:
+        (csrc / f).write_text("// " + f + "\n")
+    (csrc / "kda_api.cu").write_text("// api\n")
     h = bench.build_hash()
     assert h == bench.build_hash() and len(h) == 16
-    rec = {"build": h, "kernel": "kda_chunk_tc_kernel", "workload": "long_bf16", "dram_bytes": 1000, "units": 10}
+    hk = bench.build_hash("kda_chunk_tc_kernel")
+    assert len(hk) == 16 and hk != h and hk != bench.build_hash("kda_decode_kernel")
+    rec = {"build": hk, "kernel": "kda_chunk_tc_kernel", "workload": "long_bf16", "dram_bytes": 1000, "units": 10}
     (tmp_path / "profiles" / "k.md").write_text("# summary\ntraffic-record: " + json.dumps(rec) + "\n")
     got = bench.traffic_record("kda_chunk_tc_kernel", "long_bf16")
     assert got is not None and got["dram_bytes"] == 1000 and got["file"] == os.path.join("profiles", "k.md")
     assert bench.traffic_record("kda_chunk_tc_kernel", "prefill_bf16") is None
-    # any change to the library sources makes the record stale
+    assert bench.traffic_record("kda_decode_kernel", "long_bf16") is None
+    # changes outside the kernel's own sources leave the record valid ...
     (tmp_path / "include" / "kda.h").write_text("int y;\n")
-    assert bench.build_hash() != h
+    (csrc / "kda_api.cu").write_text("// api 2\n")
+    (csrc / "kda_backward.cuh").write_text("// changed\n")
+    assert bench.build_hash() != h and bench.build_hash("kda_chunk_tc_kernel") == hk
+    assert bench.traffic_record("kda_chunk_tc_kernel", "long_bf16") is not None
+    # ... and any change to one of them makes it stale
+    (csrc / "tc_utils.cuh").write_text("// changed\n")
+    assert bench.build_hash("kda_chunk_tc_kernel") != hk
     assert bench.traffic_record("kda_chunk_tc_kernel", "long_bf16") is None
 
 
