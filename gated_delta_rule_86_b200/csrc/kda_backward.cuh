@@ -20,10 +20,10 @@
 //
 // Schedule.  One cluster of d_v / 32 CTAs per (sequence, head); CTA s of the cluster owns value
 // columns [32 s, 32 s + 32) of the d_k x d_v state and of its gradient (the columns evolve
-// independently).  Thread (warp w, lane l) owns key rows [32 w, 32 w + 32) and column 32 s + l, in
-// fp32 registers, so every sum over d_k is a combine of the warps' partials in shared memory, and
-// every sum over d_v is a shuffle transpose-sum inside a warp (the CTA's 32 columns) plus a combine
-// of the cluster's slices through distributed shared memory, once per block of 32 tokens.  Both
+// independently).  Thread (warp w, lane l) owns key rows [R w, R w + R) (R = kRows) and column
+// 32 s + l, in fp32 registers, so every sum over d_k is a combine of the warps' partials in shared
+// memory, and every sum over d_v is a shuffle transpose-sum inside a warp (the CTA's 32 columns) plus
+// a combine of the cluster's slices through distributed shared memory, once per block of 32 tokens.  Both
 // combines run in a fixed order (no atomics: results are reproducible).
 //   1. forward over the sequence, storing the state at the start of every chunk of C tokens
 //      (the checkpoints, in the workspace);
@@ -40,11 +40,18 @@ namespace kda {
 namespace bwd {
 
 constexpr int kSub = 32;   // tokens per staged block
+#ifndef KDA_BWD_ROWS
+#define KDA_BWD_ROWS 8
+#endif
+constexpr int kRows = KDA_BWD_ROWS;   // key rows per thread: d_k / kRows warps per CTA
+static_assert(kRows == 8 || kRows == 16 || kRows == 32, "rows per thread");
 
-// Lane l ends with the warp-wide sum of value l (recursive halving, 31 shuffles for 32 values).
-__device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
+// Sum over the warp's 32 lanes of each of the kRows values v[m]: lane l ends with the sum of value
+// l % kRows (recursive halving inside groups of kRows lanes, then adds across the groups:
+// kRows - 1 + log2(32 / kRows) shuffles).
+__device__ __forceinline__ float transpose_sum_rows(float (&v)[kRows], int lane) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
+    for (int off = kRows / 2; off >= 1; off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < off; ++i) {
@@ -53,11 +60,13 @@ __device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
             v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
         }
     }
+#pragma unroll
+    for (int off = kRows; off < 32; off <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
     return v[0];
 }
 
 template <int DK, int DV> struct Smem {
-    static constexpr int NRG = DK / 32, NCS = DV / 32;   // warps per CTA, CTAs per cluster
+    static constexpr int NRG = DK / kRows, NCS = DV / 32;   // warps per CTA, CTAs per cluster
     static constexpr int kQ = 0;                       // [kSub][DK]
     static constexpr int kK = kQ + kSub * DK;          // [kSub][DK]
     static constexpr int kA = kK + kSub * DK;          // [kSub][DK]  exp(log_alpha)
@@ -100,7 +109,7 @@ __device__ __forceinline__ float ld_dsmem(const float *local, uint32_t rank) {
 }
 
 template <int DK, int DV, typename TIO, typename TDO>
-__global__ void __launch_bounds__(32 * (DK / 32))
+__global__ void __launch_bounds__(32 * (DK / bwd::kRows))
 kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *__restrict__ v,
                const TIO *__restrict__ log_alpha, const TIO *__restrict__ beta, const float *init_state,
                const int32_t *__restrict__ cu, int T, int H, int C, const TDO *__restrict__ dout,
@@ -109,13 +118,13 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
                int64_t nck_head) {
     using SM = bwd::Smem<DK, DV>;
     constexpr int NRG = SM::NRG, NCS = SM::NCS, NT = 32 * NRG;
-    constexpr int kSub = bwd::kSub;
+    constexpr int kSub = bwd::kSub, R = bwd::kRows;
     extern __shared__ float smf[];
     float *sq = smf + SM::kQ, *sk = smf + SM::kK, *sa = smf + SM::kA, *sv = smf + SM::kV, *sdo = smf + SM::kDo;
     float *sb = smf + SM::kB, *red_w = smf + SM::kRedW, *red_du = smf + SM::kRedDu, *part = smf + SM::kPart;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rg = warp, r0 = rg * 32;
+    const int rg = warp, r0 = rg * R;
     const int cs = static_cast<int>(cluster_ctarank());   // == blockIdx.x % NCS
     const int j = cs * 32 + lane;
     const int pair = blockIdx.x / NCS, h = pair % H, n = pair / H;
@@ -148,12 +157,12 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
         for (int tk = tid; tk < nb; tk += NT) sb[tk] = to_f32(beta[(size_t)(t0 + ts + tk) * H + h]);
         __syncthreads();
     };
-    // this thread's 32 key rows of a staged token vector (16-byte shared-memory loads, the same
+    // this thread's R key rows of a staged token vector (16-byte shared-memory loads, the same
     // address across the warp)
-    auto rows32 = [&](const float *base, float (&o)[32]) {
+    auto rows = [&](const float *base, float (&o)[R]) {
         const float4 *p4 = reinterpret_cast<const float4 *>(base + r0);
 #pragma unroll
-        for (int m4 = 0; m4 < 8; ++m4) {
+        for (int m4 = 0; m4 < R / 4; ++m4) {
             const float4 f = p4[m4];
             o[4 * m4] = f.x;
             o[4 * m4 + 1] = f.y;
@@ -163,13 +172,13 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     };
     // one forward step of the staged token i on the state S (one barrier; red_w is double-buffered)
     int wbuf = 0;
-    auto forward_step = [&](float (&S)[32], int i) {
-        float ka[32], aa[32];
-        rows32(sk + i * DK, ka);
-        rows32(sa + i * DK, aa);
+    auto forward_step = [&](float (&S)[R], int i) {
+        float ka[R], aa[R];
+        rows(sk + i * DK, ka);
+        rows(sa + i * DK, aa);
         float pw4[4] = {0.f, 0.f, 0.f, 0.f};   // four interleaved partial sums over the 32 rows
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
+        for (int m = 0; m < R; ++m) {
             S[m] *= aa[m];
             pw4[m & 3] = fmaf(S[m], ka[m], pw4[m & 3]);
         }
@@ -182,17 +191,17 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
         wbuf ^= 1;
         const float u = sb[i] * (sv[i * 32 + lane] - w);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) S[m] = fmaf(ka[m], u, S[m]);
+        for (int m = 0; m < R; ++m) S[m] = fmaf(ka[m], u, S[m]);
     };
 
     // ---- 1. forward with a checkpoint at the start of every chunk ----
     {
-        float S[32];
+        float S[R];
 #pragma unroll
-        for (int m = 0; m < 32; ++m) S[m] = init_state ? init_state[sbase + el(m)] : 0.f;
+        for (int m = 0; m < R; ++m) S[m] = init_state ? init_state[sbase + el(m)] : 0.f;
         for (int c = 0; c < nck; ++c) {
 #pragma unroll
-            for (int m = 0; m < 32; ++m) my_ck[(size_t)c * kv + el(m)] = S[m];
+            for (int m = 0; m < R; ++m) my_ck[(size_t)c * kv + el(m)] = S[m];
             if (c == nck - 1) break;   // the last chunk's tokens are recomputed in step 2
             for (int ts = c * C; ts < (c + 1) * C; ts += kSub) {
                 const int nb = min(kSub, (c + 1) * C - ts);
@@ -203,23 +212,23 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     }
 
     // ---- 2. chunks in reverse ----
-    float dS[32];
+    float dS[R];
 #pragma unroll
-    for (int m = 0; m < 32; ++m) dS[m] = dfinal ? dfinal[sbase + el(m)] : 0.f;
+    for (int m = 0; m < R; ++m) dS[m] = dfinal ? dfinal[sbase + el(m)] : 0.f;
     int blk = 0;   // reverse blocks so far (selects the partial-sum buffer)
     for (int c = nck - 1; c >= 0; --c) {
         const int cs0 = c * C, ce = min(L, cs0 + C);
         // recompute: the state before every token of the chunk, into the scratch
         {
-            float S[32];
+            float S[R];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) S[m] = my_ck[(size_t)c * kv + el(m)];
+            for (int m = 0; m < R; ++m) S[m] = my_ck[(size_t)c * kv + el(m)];
             for (int ts = cs0; ts < ce; ts += kSub) {
                 const int nb = min(kSub, ce - ts);
                 stage(ts, nb, false);
                 for (int i = 0; i < nb; ++i) {
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) my_scr[(size_t)(ts - cs0 + i) * kv + el(m)] = S[m];
+                    for (int m = 0; m < R; ++m) my_scr[(size_t)(ts - cs0 + i) * kv + el(m)] = S[m];
                     forward_step(S, i);
                 }
             }
@@ -232,24 +241,24 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
             float *pb = pg + kSub * DK;
             stage(ts, nb, true);
             // the recomputed state before token i, loaded one token ahead of its use
-            float Sn[32];
+            float Sn[R];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + nb - 1) * kv + el(m)];
+            for (int m = 0; m < R; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + nb - 1) * kv + el(m)];
             for (int i = nb - 1; i >= 0; --i) {
-                float ka[32], aa[32];
-                rows32(sk + i * DK, ka);
-                rows32(sa + i * DK, aa);
+                float ka[R], aa[R];
+                rows(sk + i * DK, ka);
+                rows(sa + i * DK, aa);
                 // S' = Diag(a) S_prev and w = S'^T k
-                float Sp[32];
+                float Sp[R];
                 float pw4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
+                for (int m = 0; m < R; ++m) {
                     Sp[m] = aa[m] * Sn[m];
                     pw4[m & 3] = fmaf(Sp[m], ka[m], pw4[m & 3]);
                 }
                 if (i > 0) {
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + i - 1) * kv + el(m)];
+                    for (int m = 0; m < R; ++m) Sn[m] = my_scr[(size_t)(ts - cs0 + i - 1) * kv + el(m)];
                 }
                 const float pw = (pw4[0] + pw4[1]) + (pw4[2] + pw4[3]);
                 red_w[(wbuf * NRG + rg) * 32 + lane] = pw;
@@ -261,20 +270,23 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
                 const float bt = sb[i], vj = sv[i * 32 + lane], doj = sdo[i * 32 + lane];
                 const float u = bt * (vj - w);
                 // o = S^T q: dS += q do^T, dq = S do (S = S' + k u^T)
-                float x[32];
+                float x[R];
                 {
-                    float qa[32];
-                    rows32(sq + i * DK, qa);
+                    float qa[R];
+                    rows(sq + i * DK, qa);
                     float pdu4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) {
+                    for (int m = 0; m < R; ++m) {
                         dS[m] = fmaf(qa[m], doj, dS[m]);
                         x[m] = fmaf(ka[m], u, Sp[m]) * doj;
                         pdu4[m & 3] = fmaf(dS[m], ka[m], pdu4[m & 3]);   // du = dS^T k
                     }
                     red_du[rg * 32 + lane] = (pdu4[0] + pdu4[1]) + (pdu4[2] + pdu4[3]);
                 }
-                pq[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
+                {
+                    const float t = bwd::transpose_sum_rows(x, lane);
+                    if (lane < R) pq[i * DK + r0 + lane] = t;
+                }
                 __syncthreads();
                 float du = 0.f;
 #pragma unroll
@@ -288,15 +300,21 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
                 }
                 // dk = dS u - beta S' du;  dS' = dS - beta k du^T;  dlog_alpha = rowsum(dS' * S');  dS = a dS'
 #pragma unroll
-                for (int m = 0; m < 32; ++m) x[m] = dS[m] * u - bt * Sp[m] * du;
-                pk[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
+                for (int m = 0; m < R; ++m) x[m] = dS[m] * u - bt * Sp[m] * du;
+                {
+                    const float t = bwd::transpose_sum_rows(x, lane);
+                    if (lane < R) pk[i * DK + r0 + lane] = t;
+                }
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
+                for (int m = 0; m < R; ++m) {
                     dS[m] = fmaf(-bt * ka[m], du, dS[m]);
                     x[m] = dS[m] * Sp[m];
                     dS[m] *= aa[m];
                 }
-                pg[i * DK + r0 + lane] = bwd::transpose_sum32(x, lane);
+                {
+                    const float t = bwd::transpose_sum_rows(x, lane);
+                    if (lane < R) pg[i * DK + r0 + lane] = t;
+                }
             }
             // the block's sums over d_v: every slice's partials are complete (cluster barrier), then
             // CTA s combines the elements e = s NT + tid, + NCS NT, ... over the slices in order 0, 1, ...
@@ -326,7 +344,7 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     }
     if (dinit) {
 #pragma unroll
-        for (int m = 0; m < 32; ++m) dinit[sbase + el(m)] = dS[m];
+        for (int m = 0; m < R; ++m) dinit[sbase + el(m)] = dS[m];
     }
     cluster_sync();   // no CTA leaves while another may still read its shared memory
 }
@@ -357,7 +375,7 @@ cudaError_t launch_bwd_dk_dv(const void *q, const void *k, const void *v, const 
     if (grid == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(32 * SM::NRG);
+    cfg.blockDim = dim3(32 * SM::NRG);   // one warp per kRows key rows
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
