@@ -21,8 +21,8 @@
 // resident at once (cooperative launch), one CTA per SM:
 //   * chain CTAs (one per (sequence, head) pair in flight; a chain runs its
 //     pairs one after another) copy each chunk image from the chain's ring in a
-//     global workspace (it stays in L2) into a three-slot shared-memory ring,
-//     two chunks ahead of their use, and
+//     global workspace (it stays in L2) into one of two shared-memory slots (image
+//     t + 2 goes into chunk t's slot once chunk t's last MMA has completed), and
 //     run, per chunk, one MMA group [-W ; Qg] S (rows 0-63 give U~ - U, rows
 //     64-127 give Qg S), the U~ epilogue, the MMAs Kd^T U~ and [. ; P] U~ (adding
 //     P U~ to rows 64-127) and the fp32 state update, while dedicated warps store
@@ -32,8 +32,9 @@
 //     transform, then W and U on the tensor cores.  The finished chunk image (-W,
 //     U, Qg = Q exp(G), Kd = K exp(G_last - G), P, gamma = exp(G_last) and a
 //     flag) is bulk-stored into its ring slot and announced through a flag in
-//     global memory (a release store; the chain polls it with relaxed loads, as
-//     only its asynchronous copies, which read L2, depend on it); the chain
+//     global memory (after the store has completed and the async proxy is fenced,
+//     a GPU-scope release store; the chain reads the flag with acquire loads and
+//     fences the async proxy before its bulk copy of the image); the chain
 //     announces in turn which slots it has copied out.
 // Every producer serves every chain, so the preparation throughput per pair is
 // (SMs - chains) / chains producer CTAs rather than a fixed cluster share.
@@ -244,21 +245,6 @@ template <> __device__ __forceinline__ void store16<float>(float *dst, const flo
 template <> __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16 *dst, const float *f) {
     reinterpret_cast<uint4 *>(dst)[0] = pack8_bf16(f);
     reinterpret_cast<uint4 *>(dst)[1] = pack8_bf16(f + 8);
-}
-
-// Sum 32 per-lane values across the warp so that lane l ends with the warp-wide
-// sum of value l (recursive halving: 31 shuffles for 32 values).
-__device__ __forceinline__ void warp_transpose_sum32(float (&v)[32], int lane) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-            const float send = upper ? v[i] : v[i + off];
-            const float keep = upper ? v[i + off] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
 }
 
 // One thread of a role waits on an mbarrier phase (bounded), then the role's
