@@ -483,6 +483,8 @@ def run_kda(args):
         "traffic_source": None if rec is None else
         f"{rec['file']}: ncu dram__bytes_read.sum + dram__bytes_write.sum on {rec['units']} token-heads "
         f"(build {rec['build']}), scaled by token-heads",
+        # the same capture's utilisation counters (tensor pipe, DRAM throughput; the 16K launch under ncu)
+        "ncu_counters": None if rec is None else rec.get("ncu"),
         "build": build_hash("kda_chunk_tc_kernel"),
         "tensor": {"alg_flops_per_launch": alg_flops,
                    "achieved_tflops": alg_flops / (ms_step * 1e-3) / 1e12,
@@ -586,7 +588,8 @@ def run_kda(args):
                            "alg_bytes_per_launch": d_bytes,
                            "traffic_source": None if drec is None else
                            f"{drec['file']}: ncu dram__bytes_read.sum + dram__bytes_write.sum on {drec['units']} "
-                           f"head-steps (build {drec['build']})"}}
+                           f"head-steps (build {drec['build']})",
+                           "ncu_counters": None if drec is None else drec.get("ncu")}}
     # decode end to end: tokens from pinned host memory each step, output read back each step
     hq = [d[n][:64].cpu().pin_memory() for n in names]
     hout = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, pin_memory=True)
