@@ -26,6 +26,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -135,23 +136,70 @@ def decode_alg_bytes(heads, dk=128, dv=128, in_bytes=2, out_bytes=4):
 # ---- clocks -----------------------------------------------------------------------------------------
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled while the timed region runs: through NVML
+    (read-only queries) every 5 ms from a background thread, else through `nvidia-smi -lms 200`.
+    `nvml` may be given (a module with the pynvml names) for tests."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+    PERIOD_S = 0.005
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, nvml=None):
         self.proc = None
         self.path = None
         self.device_index = device_index
+        self.nvml = nvml
+        self.rows = None       # NVML samples: (sm_mhz, max_mhz, power_w, reason bits)
+        self.thread = None
 
-    def __enter__(self):
+    def _uuid(self):
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
-            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            return uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
         except Exception:
-            ident = str(self.device_index)
+            return None
+
+    def _start_nvml(self):
+        nv = self.nvml
+        if nv is None:
+            try:
+                import pynvml as nv
+            except ImportError:
+                return False
+        try:
+            nv.nvmlInit()
+            uuid = self._uuid()
+            handle = nv.nvmlDeviceGetHandleByUUID(uuid) if uuid else nv.nvmlDeviceGetHandleByIndex(self.device_index)
+            max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        except Exception:
+            return False
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.rows = []
+        self.stop = threading.Event()
+
+        def run():
+            while True:
+                try:
+                    self.rows.append((nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM), max_mhz,
+                                      nv.nvmlDeviceGetPowerUsage(handle) / 1000.0, reasons_fn(handle)))
+                except Exception:
+                    pass
+                if self.stop.wait(self.PERIOD_S):
+                    return
+
+        self.nv = nv
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        return True
+
+    def __enter__(self):
+        if self._start_nvml():
+            return self
+        ident = self._uuid() or str(self.device_index)
         fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
         os.close(fd)
         try:
@@ -164,6 +212,13 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -173,6 +228,15 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        if self.rows is not None:
+            if not self.rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": "nvml"}
+            bits = 0
+            for r in self.rows:
+                bits |= int(r[3])
+            return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
+                    "reasons": sorted(n for n, b in self.REASONS if bits & b), "samples": len(self.rows),
+                    "power_w_max": max(r[2] for r in self.rows), "source": "nvml, every 5 ms"}
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
@@ -196,7 +260,7 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows), "source": "nvidia-smi, every 200 ms"}
 
 
 # ---- distributed plumbing ---------------------------------------------------------------------------

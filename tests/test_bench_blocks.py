@@ -103,3 +103,51 @@ def test_traffic_record_needs_the_current_build(tmp_path, monkeypatch):
 def test_cpu_model_is_text_or_none():
     m = bench.cpu_model()
     assert m is None or (isinstance(m, str) and m)
+
+
+class _FakeNvml:
+    """Stands in for pynvml: fixed clocks and power, reason bits that change after a few samples."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self):
+        self.calls = 0
+        self.shutdown = False
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        self.shutdown = True
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        return "h"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        assert kind == self.NVML_CLOCK_SM
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.calls += 1
+        return 1965 if self.calls % 2 else 1950
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 250000 + 1000 * self.calls   # mW
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 if self.calls > 3 else 0x1   # sw_power_cap after a while; 0x1 (idle) is not reported
+
+
+def test_clock_sampler_nvml_summary():
+    import time
+    fake = _FakeNvml()
+    with bench.ClockSampler(0, nvml=fake) as clk:
+        time.sleep(0.1)
+    s = clk.summary()
+    assert fake.shutdown and s["source"].startswith("nvml")
+    assert s["samples"] >= 5 and s["sm_max_mhz"] == 1965 and s["sm_mhz"] in (1950, 1957.5, 1965)
+    assert s["reasons"] == ["sw_power_cap"]
+    assert s["power_w_max"] >= 250.0
+    json.dumps(s)
