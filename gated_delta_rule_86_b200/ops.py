@@ -335,6 +335,41 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_s
     return tuple(g)
 
 
+class _KdaChunk(torch.autograd.Function):
+    """Autograd wrapper: forward = kda_chunk_fwd, backward = kda_chunk_bwd (both in the library)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk_size, out_dtype):
+        out, fs = kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=initial_state, cu_seqlens=cu_seqlens,
+                                output_final_state=True, chunk_size=chunk_size, out_dtype=out_dtype)
+        ctx.save_for_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+        ctx.chunk_size = chunk_size
+        return out, fs
+
+    @staticmethod
+    def backward(ctx, d_out, d_final_state):
+        q, k, v, log_alpha, beta, s0, cu = ctx.saved_tensors
+        if d_out is None:
+            d_out = torch.zeros(v.shape, dtype=torch.float32, device=v.device)
+        # the backward's chunk_size is its checkpoint interval (it changes no result)
+        grads = kda_chunk_bwd(q, k, v, log_alpha, beta, d_out, initial_state=s0, d_final_state=d_final_state,
+                              cu_seqlens=cu, chunk_size=ctx.chunk_size)
+        dq, dk, dv, dla, db, ds0 = grads
+        cast = [g.to(x.dtype) if (x is not None and ctx.needs_input_grad[i]) else None
+                for i, (g, x) in enumerate(zip((dq, dk, dv, dla, db, ds0), (q, k, v, log_alpha, beta, s0)))]
+        return (*cast, None, None, None)
+
+
+def kda_chunk(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
+              out_dtype=torch.float32):
+    """Differentiable KDA prefill on CUDA tensors: ``(out, final_state)`` of :func:`kda_chunk_fwd`, with
+    gradients (through :func:`kda_chunk_bwd`) for q, k, v, log_alpha, beta and the initial state, cast to
+    their dtypes.  The gradient is that of the exact recurrence, evaluated in fp32."""
+    if not q.is_cuda:
+        raise ValueError("kda_chunk takes CUDA tensors")
+    return _KdaChunk.apply(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk_size, out_dtype)
+
+
 def device_error() -> int:
     """Sync the current stream and return-and-clear the device error word (KDA_OK or KDA_ERR_TIMEOUT)."""
     return _lib.load().kda_get_last_device_error(_stream_handle())

@@ -117,3 +117,32 @@ def test_backward_matches_autograd_free_directional_derivative(cuda_lib):
     grads = kda_chunk_bwd(*base[:5], do, initial_state=base[5])
     an = sum(float((gr.double() * d.double()).sum()) for gr, d in zip(grads, dirs))
     assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), (fd, an)
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_autograd_wrapper(cuda_lib, varlen):
+    """kda_chunk (torch.autograd.Function over kda_chunk_fwd / kda_chunk_bwd): loss.backward() gives the
+    gradients of kda_chunk_bwd called directly (bitwise, cast to each input's dtype), and those are the
+    oracle's; the forward outputs are kda_chunk_fwd's."""
+    from gated_delta_rule_86_b200 import kda_chunk, kda_chunk_fwd
+    if varlen:
+        x = inputs.make_prefill("varlen_bf16", device="cpu", H=2, varlen=3, varlen_range=(40, 150))
+    else:
+        x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=130, H=3, init_state=True)
+    dev = torch.device("cuda")
+    cu = None if x["cu_seqlens"] is None else x["cu_seqlens"].to(dev)
+    leaves = [x[n].to(dev).requires_grad_(True) for n in NAMES]
+    s0 = x["init_state"].to(dev).requires_grad_(True)
+    do, dfin = upstream(x, 11)
+    out, fs = kda_chunk(*leaves, initial_state=s0, cu_seqlens=cu)
+    ((out * do.to(dev)).sum() + (fs * dfin.to(dev)).sum()).backward()
+    ref_out, ref_fs = kda_chunk_fwd(*(t.detach() for t in leaves), initial_state=s0.detach(), cu_seqlens=cu)
+    assert torch.equal(out.detach(), ref_out) and torch.equal(fs.detach(), ref_fs)
+    direct = kda_chunk_bwd(*(t.detach() for t in leaves), do.to(dev), initial_state=s0.detach(),
+                           d_final_state=dfin.to(dev), cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    for name, leaf, want in zip(GRADS, leaves + [s0], direct):
+        assert leaf.grad is not None and leaf.grad.dtype == leaf.dtype, name
+        assert torch.equal(leaf.grad, want.to(leaf.dtype)), name
+    check(x, do, dfin)
