@@ -468,18 +468,24 @@ def backward_block(args, world):
     d_out = torch.randn(x["v"].shape, generator=g, device="cuda")
     a = [x[n] for n in ("q", "k", "v", "log_alpha", "beta")]
 
-    def step(_i):
-        return kda_chunk_bwd(*a, d_out, initial_state=x["init_state"])
+    def step(_i, chunk=64):
+        return kda_chunk_bwd(*a, d_out, initial_state=x["init_state"], chunk_size=chunk)
 
     ms = timed_steps(step, args, world)
+    # the state before every token kept (chunk_size 0): no recompute pass, one state per token-head
+    ms_all = timed_steps(lambda i: step(i, 0), args, world)
     th = w.B * w.T * w.H
     flops = bwd_alg_flops(th)
     tf = flops / (ms * 1e-3) / 1e12
     return {"entry": "kda_chunk_bwd", "workload": "prefill_bf16 shape (B2 H16 T4096 d128), N(0,0.1) initial state, "
-            "N(0,1) upstream gradient", "ms_per_step": ms, "tokens_per_s": world * w.B * w.T / (ms * 1e-3),
+            "N(0,1) upstream gradient", "chunk_size": 64, "ms_per_step": ms,
+            "tokens_per_s": world * w.B * w.T / (ms * 1e-3),
             "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                          "frac": tf / FP32_PEAK_TFLOPS, "traffic": None, "kernel": "kda_bwd_kernel",
-                         "alg_flops_per_launch": flops, "peak_source": FP32_PEAK_NOTE}}
+                         "alg_flops_per_launch": flops, "peak_source": FP32_PEAK_NOTE},
+            "every_state": {"chunk_size": 0, "ms_per_step": ms_all, "tokens_per_s": world * w.B * w.T / (ms_all * 1e-3),
+                            "workspace_bytes": w.H * w.B * w.T * w.dk * w.dv * 4,
+                            "frac_of_fp32_peak": flops / (ms_all * 1e-3) / 1e12 / FP32_PEAK_TFLOPS}}
 
 
 def oracle_single_thread(workload, T_s=4096):

@@ -350,7 +350,7 @@ extern "C" {
 
 kda_status kda_chunk_bwd_workspace_size(int32_t N, int32_t H, int64_t total_tokens, int32_t d_k, int32_t d_v,
                                         int32_t chunk, size_t *bytes) {
-    if (!bytes || N < 1 || H < 1 || total_tokens < 0 || chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (!bytes || N < 1 || H < 1 || total_tokens < 0 || chunk < 0) return KDA_ERR_INVALID_ARG;
     *bytes = 0;
     if (!head_ok(d_k) || !head_ok(d_v) || chunk > 256) return KDA_ERR_UNSUPPORTED;
     *bytes = kda::bwd_workspace_bytes(N, H, total_tokens, d_k, d_v, chunk);
@@ -371,7 +371,7 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void
     const void *outs[] = {dq, dk, dv, dlog_alpha, dbeta, d_init_state};
     for (const void *p : outs)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
-    if (chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (chunk < 0) return KDA_ERR_INVALID_ARG;   // 0: every state stored, no recompute
     if (chunk > 256) return KDA_ERR_UNSUPPORTED;
     const int N = cu_seqlens ? num_seqs : B;
     const int64_t total = cu_seqlens ? (int64_t)T : (int64_t)B * T;

@@ -29,6 +29,9 @@
 //      (the checkpoints, in the workspace);
 //   2. chunks in reverse: the chunk's states are recomputed from its checkpoint into a per-pair
 //      scratch (one d_k x d_v state per token), then its tokens are visited in reverse.
+// With C = 0 ("every state") step 1 stores the state before every token instead and step 2 reads
+// those (no recompute; the workspace then holds one state per token and head); the states, and so
+// the results, are bitwise those of the checkpointed schedule.
 // Token vectors move through shared memory 32 tokens at a time.  Each token costs three passes of
 // the recurrence (checkpoint pass, recompute, reverse), all in fp32.
 #pragma once
@@ -131,10 +134,14 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     const int64_t t0 = cu ? (int64_t)cu[n] : (int64_t)n * T;
     const int64_t t1 = cu ? (int64_t)cu[n + 1] : t0 + T;
     const int L = static_cast<int>(t1 - t0);
-    const int nck = (L + C - 1) / C;
+    const bool every = C == 0;   // the state before every token is stored in step 1: no recompute
+    const int Ce = every ? (L > 0 ? L : 1) : C;
+    const int nck = (L + Ce - 1) / Ce;
     const size_t kv = (size_t)DK * DV;
-    float *my_ck = ckpt + ((size_t)h * nck_head + bwd::ckpt_base(t0, n, C)) * kv;
-    float *my_scr = scratch + (size_t)pair * C * kv;
+    float *my_ck = every ? nullptr : ckpt + ((size_t)h * nck_head + bwd::ckpt_base(t0, n, C)) * kv;
+    // step 2's per-token states: the per-pair scratch of one chunk, or (every) this pair's tokens in
+    // the workspace's [H][total tokens] states
+    float *my_scr = every ? scratch + ((size_t)h * nck_head + t0) * kv : scratch + (size_t)pair * C * kv;
     const size_t sbase = ((size_t)n * H + h) * kv;
     auto el = [&](int m) { return (size_t)(r0 + m) * DV + j; };   // this thread's element of row r0 + m
 
@@ -194,8 +201,21 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
         for (int m = 0; m < R; ++m) S[m] = fmaf(ka[m], u, S[m]);
     };
 
-    // ---- 1. forward with a checkpoint at the start of every chunk ----
-    {
+    // ---- 1. forward with a checkpoint at the start of every chunk (every: before every token) ----
+    if (every) {
+        float S[R];
+#pragma unroll
+        for (int m = 0; m < R; ++m) S[m] = init_state ? init_state[sbase + el(m)] : 0.f;
+        for (int ts = 0; ts < L; ts += kSub) {
+            const int nb = min(kSub, L - ts);
+            stage(ts, nb, false);
+            for (int i = 0; i < nb; ++i) {
+#pragma unroll
+                for (int m = 0; m < R; ++m) my_scr[(size_t)(ts + i) * kv + el(m)] = S[m];
+                if (ts + i + 1 < L) forward_step(S, i);
+            }
+        }
+    } else {
         float S[R];
 #pragma unroll
         for (int m = 0; m < R; ++m) S[m] = init_state ? init_state[sbase + el(m)] : 0.f;
@@ -217,9 +237,9 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
     for (int m = 0; m < R; ++m) dS[m] = dfinal ? dfinal[sbase + el(m)] : 0.f;
     int blk = 0;   // reverse blocks so far (selects the partial-sum buffer)
     for (int c = nck - 1; c >= 0; --c) {
-        const int cs0 = c * C, ce = min(L, cs0 + C);
+        const int cs0 = c * Ce, ce = min(L, cs0 + Ce);
         // recompute: the state before every token of the chunk, into the scratch
-        {
+        if (!every) {
             float S[R];
 #pragma unroll
             for (int m = 0; m < R; ++m) S[m] = my_ck[(size_t)c * kv + el(m)];
@@ -353,6 +373,7 @@ kda_bwd_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *
 // head) and one chunk's per-token states for every (sequence, head) pair.
 inline size_t bwd_workspace_bytes(int64_t N, int64_t H, int64_t total_tokens, int DK, int DV, int C) {
     const size_t kv = (size_t)DK * DV * sizeof(float);
+    if (C == 0) return (size_t)H * (size_t)(total_tokens > 0 ? total_tokens : 1) * kv;   // every state
     return (size_t)H * bwd::ckpts_per_head(total_tokens, (int)N, C) * kv + (size_t)N * H * C * kv;
 }
 
@@ -368,9 +389,11 @@ cudaError_t launch_bwd_dk_dv(const void *q, const void *k, const void *v, const 
     if (e != cudaSuccess) return e;
     const int N = cu ? num_seqs : B;
     const int64_t total = cu ? (int64_t)T : (int64_t)B * T;   // with cu_seqlens, T is the packed length
-    const int64_t nck_head = bwd::ckpts_per_head(total, N, C);
+    // the checkpoints then the per-pair scratch; with C == 0 only the [H][total tokens] states (the
+    // kernel's per-head stride is then total)
+    const int64_t nck_head = C == 0 ? total : bwd::ckpts_per_head(total, N, C);
     float *ck = static_cast<float *>(workspace);
-    float *scr = ck + (size_t)H * nck_head * DK * DV;
+    float *scr = C == 0 ? ck : ck + (size_t)H * nck_head * DK * DV;
     const unsigned grid = static_cast<unsigned>(N) * H * SM::NCS;
     if (grid == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};

@@ -295,7 +295,8 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_s
     Takes the forward's inputs and ``d_out`` = dLoss/dout ([B, T, H, d_v], fp32 or bf16) and,
     optionally, ``d_final_state`` = dLoss/dfinal_state (fp32 [N, H, d_k, d_v]).  Returns
     ``(dq, dk, dv, dlog_alpha, dbeta, d_initial_state)`` in fp32 with the shapes of q, k, v,
-    log_alpha, beta and the initial state.  ``chunk_size`` is the checkpoint interval.
+    log_alpha, beta and the initial state.  ``chunk_size`` is the checkpoint interval (0: the state
+    before every token is kept, no recompute; more workspace, same result).
     """
     lib = _lib.load()
     on_host = not q.is_cuda

@@ -281,7 +281,10 @@ kda_status kda_chunk_fwd_static_ws(const void *q, const void *k, const void *v, 
  *   d_k, d_v, dtype : as for kda_chunk_fwd (the forward's inputs).
  *   chunk           : states are checkpointed every `chunk` tokens and each
  *                     chunk's per-token states recomputed from its checkpoint
- *                     (1 <= chunk <= 256; it changes no result).
+ *                     (1 <= chunk <= 256); 0 keeps the state before every
+ *                     token instead (no recompute: one pass fewer, a workspace
+ *                     of H * total_tokens * d_k * d_v * 4 bytes).  It changes
+ *                     no result: the gradients are bitwise the same.
  *   d_out           : [B, T, H, d_v] d_out_dtype, dLoss/dout.
  *   d_final_state   : [N, H, d_k, d_v] fp32 dLoss/dfinal_state, or NULL (zero).
  *   dq, dk, dlog_alpha : [B, T, H, d_k] fp32 (written).

@@ -193,7 +193,10 @@ def test_backward_argument_checks(lib):
     kv = 128 * 128 * 4
     assert n.value == 4 * (1000 // 64 + 2 + 1) * kv + 2 * 4 * 64 * kv
     assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 96, 128, 64, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
-    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 0, ctypes.byref(n)) == _lib.KDA_ERR_INVALID_ARG
+    # chunk 0: the state before every token is kept (one state per token and head), no recompute
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 0, ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == 4 * 1000 * kv
+    assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, -1, ctypes.byref(n)) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_chunk_bwd_workspace_size(2, 4, 1000, 128, 128, 512, ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
     F = ctypes.c_void_p(4096)
     bwd = lib.kda_chunk_bwd
@@ -206,6 +209,6 @@ def test_backward_argument_checks(lib):
     assert call(dq=None) == _lib.KDA_ERR_INVALID_ARG
     assert call(ws=None) == _lib.KDA_ERR_INVALID_ARG
     assert call(ws_bytes=16) == _lib.KDA_ERR_INVALID_ARG
-    assert call(chunk=0) == _lib.KDA_ERR_INVALID_ARG
+    assert call(chunk=-1) == _lib.KDA_ERR_INVALID_ARG
     assert call(chunk=300) == _lib.KDA_ERR_UNSUPPORTED
     assert call(dq=ctypes.c_void_p(4100)) == _lib.KDA_ERR_INVALID_ARG   # misaligned

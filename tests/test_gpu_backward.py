@@ -146,3 +146,29 @@ def test_autograd_wrapper(cuda_lib, varlen):
         assert leaf.grad is not None and leaf.grad.dtype == leaf.dtype, name
         assert torch.equal(leaf.grad, want.to(leaf.dtype)), name
     check(x, do, dfin)
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_backward_every_state_bitwise(cuda_lib, varlen):
+    """chunk_size = 0 keeps the state before every token (no recompute pass): bitwise the gradients
+    of the checkpointed schedule, and within the bound of the oracle."""
+    if varlen:
+        lens = [1, 0, 64, 130, 7, 65, 0, 100]
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+        x = inputs.make_prefill("prefill_bf16", device="cpu", B=1, T=int(cu[-1]), H=2, init_state=False)
+        x["cu_seqlens"] = cu
+        x["init_state"] = torch.randn((len(lens), 2, 128, 128), generator=torch.Generator().manual_seed(9)) * 0.1
+    else:
+        x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=333, H=3, init_state=True)
+    do, dfin = upstream(x, 12)
+    dev = torch.device("cuda")
+    a = [x[n].to(dev) for n in NAMES]
+    s0 = x["init_state"].to(dev)
+    cu = None if x["cu_seqlens"] is None else x["cu_seqlens"].to(dev)
+    runs = [kda_chunk_bwd(*a, do.to(dev), initial_state=s0, d_final_state=dfin.to(dev), cu_seqlens=cu, chunk_size=c)
+            for c in (64, 0)]
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    for name, g64, g0 in zip(GRADS, *runs):
+        assert torch.equal(g64, g0), name
+    check(x, do, dfin, chunk=0)
