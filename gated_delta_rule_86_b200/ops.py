@@ -85,6 +85,16 @@ def _out_dtype(out_dtype):
     return _DTYPES[out_dtype]
 
 
+def segment_bounds(T, segments, chunk_size):
+    """Token ranges [a, b) of the host-buffer pipeline: at most ``segments`` of them, each starting at
+    a multiple of ``chunk_size`` (so that the chunks are those of one call), covering [0, T)."""
+    if T <= 0:
+        return []
+    seg = -(-T // max(1, segments))
+    seg = -(-seg // chunk_size) * chunk_size
+    return [(a, min(a + seg, T)) for a in range(0, T, seg)]
+
+
 def _host_pipelined(fn_name, q, k, v, gate, beta, initial_state, chunk_size, out_dtype, segments):
     """The prefill of one sequence (B == 1) held in pinned host memory, in token segments whose
     host-to-device copies, kernels and device-to-host copies overlap: segment i's inputs travel on
@@ -94,9 +104,7 @@ def _host_pipelined(fn_name, q, k, v, gate, beta, initial_state, chunk_size, out
     dev = torch.device("cuda", torch.cuda.current_device())
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    seg = -(-T // segments)
-    seg = -(-seg // chunk_size) * chunk_size
-    bounds = [(a, min(a + seg, T)) for a in range(0, T, seg)]
+    bounds = segment_bounds(T, segments, chunk_size)
     hosts = [q, k, v, gate, beta]
     devs = [None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hosts]
     out_d = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev)
