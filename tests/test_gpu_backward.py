@@ -172,3 +172,18 @@ def test_backward_every_state_bitwise(cuda_lib, varlen):
     for name, g64, g0 in zip(GRADS, *runs):
         assert torch.equal(g64, g0), name
     check(x, do, dfin, chunk=0)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_backward_every_state_head_sizes(cuda_lib, dk, dv):
+    """chunk_size = 0 at the other head sizes: bitwise the checkpointed schedule's gradients."""
+    x = inputs.make_prefill("prefill_bf16", device="cpu", B=2, T=97, H=2, dk=dk, dv=dv, init_state=True)
+    do, dfin = upstream(x, dk + 3 * dv)
+    dev = torch.device("cuda")
+    a = [x[n].to(dev) for n in NAMES]
+    runs = [kda_chunk_bwd(*a, do.to(dev), initial_state=x["init_state"].to(dev), d_final_state=dfin.to(dev),
+                          chunk_size=c) for c in (32, 0)]
+    torch.cuda.synchronize()
+    assert device_error() == 0
+    for name, g1, g0 in zip(GRADS, *runs):
+        assert torch.equal(g1, g0), name
